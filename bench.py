@@ -1,0 +1,399 @@
+"""Throughput of the GDN chunked-prefill forward on B200, one JSON line.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+A step is one forward pass of the layer over one batch of the bf16 workload
+B=1, T=4096, H=16, dk=dv=128 (C=64, random fp32 S0) through the C ABI, inputs
+already resident in HBM.  The L2 is flushed (a 2 x L2-size write) before every
+timed step, outside the timed events.  ``value`` is whole-job tokens/s; with N
+GPUs every rank runs its own replica (weak scaling, no collective on the data
+path) and the time is the max over ranks.  ``e2e`` times the same call with the
+inputs in pinned host memory, including the host->device copies of the inputs
+and the device->host copies of o and S_T.  ``bwd`` reports the backward on the
+B=4, T=8192, H=16, d=128 workload.  ``cpu_baseline`` times the float64 oracle on
+a bounded sample of the same workload on the host cores.
+
+``--impl reference`` times the oracle (there is no other implementation of this
+layer to run here) on a bounded sample per step and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN chunked-prefill fwd/bwd tokens/s and TFLOP/s vs BF16 roofline, 1×B200"
+CHUNK = 64
+
+
+def flops_per_token_head(dk, dv, C=CHUNK, backward=False):
+    """(dense MMA-tile FLOPs, triangular-aware FLOPs) per token and value head."""
+    if backward:
+        dense = 16 * dk * dv + 14 * 2 * C * dk + 4 * C * C
+        return dense, dense * 385000 / 507904
+    dense = 6 * dk * dv + 2 * C * (3 * dk + 2 * dv)
+    tri = 6 * dk * dv + C * (3 * dk + 2 * dv) + C * C / 3
+    return dense, tri
+
+
+def fwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
+    """Algorithmic HBM bytes of one forward: read q, k, v, beta, g, S0; write o, S_T."""
+    return T_total * (elt * (Hk * 2 * dk + Hv * 2 * dv) + Hv * 8) + 2 * N * Hv * dk * dv * 4
+
+
+def bwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
+    """Read q, k, v, do, beta, g; write dq, dk, dv, dbeta, dg (+ dS_T read, dS0 write)."""
+    return T_total * (elt * (Hk * 4 * dk + Hv * 3 * dv) + Hv * 16) + 2 * N * Hv * dk * dv * 4
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling (every 200 ms) around the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- oracle arm
+def oracle_sample(inp, nheads, units_total):
+    """Run the oracle on the first ``nheads`` value heads of a fixed-length workload
+    in one call (OpenMP over the heads) and return (seconds, tokens/s scaled to
+    the full workload: tokens x nheads / units_total per second)."""
+    import oracle
+
+    x = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    grp = x["v"].shape[2] // x["q"].shape[2]
+    hk1 = (nheads + grp - 1) // grp
+    nheads = hk1 * grp
+    S0 = None if x.get("initial_state") is None else x["initial_state"][:, :nheads]
+    t0 = time.perf_counter()
+    oracle.fwd(x["q"][:, :, :hk1], x["k"][:, :, :hk1], x["v"][:, :, :nheads],
+               x["beta"][:, :, :nheads], x["g"][:, :, :nheads], initial_state=S0)
+    dt = time.perf_counter() - t0
+    tokens = x["q"].shape[0] * x["q"].shape[1] * nheads / units_total
+    return dt, tokens / dt, nheads
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    from gated_deltanet_chunked_fwd_b200.inputs import make_workload
+
+    inp = make_workload(1, seed=0)
+    Hv = inp["v"].shape[2]
+    nheads = min(Hv, oracle.num_threads())  # bounded sample: one head per host thread
+    for _ in range(args.warmup):
+        oracle_sample(inp, 1, Hv)
+    times = []
+    for _ in range(args.steps):
+        dt, _, nheads = oracle_sample(inp, nheads, Hv)
+        times.append(dt)
+    T_tok = inp["q"].shape[1] * inp["q"].shape[0]
+    tok_per_step = T_tok * nheads / Hv
+    value = tok_per_step * len(times) / sum(times)
+    cores = min(nheads, oracle.num_threads())
+    heads = range(nheads)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "gdn_fwd bf16 B=1 T=4096 H=16 dk=dv=128 C=64 S0~0.1N(0,1)",
+                   "global_batch": 1, "seq_len": 4096, "parallelism": "none (host oracle)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{len(heads)} of {Hv} value heads per step (float64 token loop)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- our arm
+def time_steps(fn, steps, flush, stream):
+    """Per-step device time (ms) with CUDA events on ``stream``; L2 flushed before each step."""
+    ms = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    return ms
+
+
+def run_ours(args, world, rank, local):
+    import ctypes
+
+    import gated_deltanet_chunked_fwd_b200 as gdn
+    from gated_deltanet_chunked_fwd_b200 import _abi
+    from gated_deltanet_chunked_fwd_b200.inputs import make_workload
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    L = _abi.lib()
+    inp = make_workload(1, seed=rank, device=dev)
+    q, k, v, beta, g, S0 = (inp[n] for n in ("q", "k", "v", "beta", "g", "initial_state"))
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    N = B
+    o = torch.empty(B, T, Hv, dv, dtype=q.dtype, device=dev)
+    ST = torch.empty(N, Hv, dk, dv, dtype=torch.float32, device=dev)
+    a = _abi.GdnFwdArgs()
+    gdn._fill_common(a, q, k, v, beta, g, None, None, S0, 0)
+    a.o, a.ST = o.data_ptr(), ST.data_ptr()
+    ws_n = gdn.gdn_chunk_fwd_workspace_size(q, k, v, beta, g, initial_state=S0)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    launches = L.gdn_chunk_fwd_launch_count(ctypes.byref(a))
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def step():
+        st = L.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(ws.data_ptr()), ws_n, sp)
+        if st != 0:
+            raise gdn.GdnError("gdn_chunk_fwd", st)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    scratch = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+
+    def flush():
+        scratch.fill_(1.0)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        ms = time_steps(step, args.steps, flush, stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms_step = max_over_ranks(sum(ms) / len(ms), world)
+    tokens = B * T
+    value = tokens * world / (ms_step * 1e-3)
+
+    # ---- e2e: pinned host inputs, H2D + call + D2H of o and S_T, inside the timed region
+    host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("beta", beta),
+                                                  ("g", g), ("S0", S0))}
+    dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    ST_h = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
+    ae = _abi.GdnFwdArgs()
+    gdn._fill_common(ae, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["beta"], dbuf["g"], None, None,
+                     dbuf["S0"], 0)
+    ae.o, ae.ST = o.data_ptr(), ST.data_ptr()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * ST_h.element_size()
+
+    def e2e_step():
+        for n_, t in host.items():
+            dbuf[n_].copy_(t, non_blocking=True)
+        st = L.gdn_chunk_fwd(ctypes.byref(ae), ctypes.c_void_p(ws.data_ptr()), ws_n, sp)
+        if st != 0:
+            raise gdn.GdnError("gdn_chunk_fwd", st)
+        o_h.copy_(o, non_blocking=True)
+        ST_h.copy_(ST, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(sum(time_steps(e2e_step, args.steps, flush, stream)) / args.steps, world)
+    e2e_value = tokens * world / (ms_e2e * 1e-3)
+
+    # ---- roofline of the dominant kernel (the whole forward when it is one launch)
+    hbm, bf16, src = measured_peaks()
+    byts = fwd_bytes(tokens, Hk, Hv, dk, dv, N)
+    dense, tri = flops_per_token_head(dk, dv)
+    achieved = byts / (ms_step * 1e-3) / 1e9
+    tflops_dense = dense * tokens * Hv / (ms_step * 1e-3) / 1e12
+    tflops_tri = tri * tokens * Hv / (ms_step * 1e-3) / 1e12
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            traffic = json.load(f).get("fwd_bf16_T4096_H16_d128", {}).get("bytes_per_launch")
+
+    # ---- backward on its own workload (one step per measurement)
+    bwd = None
+    if not args.no_bwd:
+        bi = make_workload(4, seed=rank, device=dev)
+        qs = [bi[n] for n in ("q", "k", "v", "beta", "g", "do")]
+        wsb = torch.empty(max(gdn.gdn_chunk_bwd_workspace_size(*qs[:5]), 1), dtype=torch.uint8,
+                          device=dev)
+
+        def bstep():
+            gdn.gdn_chunk_bwd(*qs, dST=bi["dST"], workspace=wsb)
+
+        bstep()
+        torch.cuda.synchronize()
+        bms = max_over_ranks(statistics.mean(time_steps(bstep, max(1, min(args.steps, 5)), flush,
+                                                        stream)), world)
+        bt = bi["q"].shape[0] * bi["q"].shape[1]
+        bd, btri = flops_per_token_head(dk, dv, backward=True)
+        bb = bwd_bytes(bt, Hk, Hv, dk, dv, bi["q"].shape[0])
+        bwd = {"workload": "gdn_bwd bf16 B=4 T=8192 H=16 dk=dv=128 C=64", "tokens_per_s": bt * world / (bms * 1e-3),
+               "ms": bms, "tflops_dense": bd * bt * Hv / (bms * 1e-3) / 1e12,
+               "tflops_tri": btri * bt * Hv / (bms * 1e-3) / 1e12,
+               "hbm_gbs": bb / (bms * 1e-3) / 1e9}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import oracle
+
+        nh = min(Hv, oracle.num_threads())
+        dt, tps, nh = oracle_sample(make_workload(1, seed=0), nh, Hv)
+        cpu_base = {"value": tps, "unit": "tokens/s", "cores": min(nh, oracle.num_threads()),
+                    "kind": "oracle",
+                    "sample": f"{nh} of {Hv} value heads of the same workload (all 4096 tokens), "
+                              f"float64 token loop, {dt:.2f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "gdn_fwd bf16 B=1 T=4096 H=16 dk=dv=128 C=64 S0~0.1N(0,1)",
+                       "global_batch": world, "seq_len": T, "heads": Hv, "head_dim": dk,
+                       "parallelism": f"replicas x{world} (no collective)",
+                       "l2": "flushed before every timed step (2x L2 write, outside the events)",
+                       "path": "tensor-core fused" if launches == 1 else "cuda-core 4-kernel"},
+            "tflops": {"dense": tflops_dense, "triangular": tflops_tri, "peak_bf16": bf16,
+                       "frac_dense": tflops_dense / bf16},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": traffic,
+                         "peak_source": src, "algorithmic_bytes": byts,
+                         "kernel": "whole forward (all launches of one call)"},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu_base,
+            "bwd": bwd,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        # the oracle arm runs on rank 0's host cores only; no process group
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        args.gpus = world
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

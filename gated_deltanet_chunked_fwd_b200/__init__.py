@@ -1,0 +1,186 @@
+"""GDN chunked prefill (forward and backward) on NVIDIA B200 -- Python binding.
+
+``gdn_chunk_fwd`` / ``gdn_chunk_bwd`` mirror the C entry points of
+``include/gdn.h`` one to one.  This module marshals torch tensors into the C
+argument structs, allocates the outputs and the workspace with torch (device
+memory) and passes torch's current CUDA stream.  All arithmetic runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback.
+
+The layer is the gated delta rule of the Gated Delta Network (the GDN layer of
+the FlashQLA pages, news.hamidun.com "What is FlashQLA"):
+    S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t,
+states stored transposed (H = S^T, [dk, dv]).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _abi
+from ._abi import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE, GDN_FLAG_SPLIT_OFF, GdnBwdArgs,
+                   GdnError, GdnFwdArgs)
+
+__all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_chunk_fwd_workspace_size",
+           "gdn_chunk_bwd_workspace_size", "GdnError", "GDN_FLAG_SPLIT_OFF",
+           "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE"]
+
+_DT = {torch.float32: _abi.GDN_F32, torch.bfloat16: _abi.GDN_BF16}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libgdn must be contiguous")
+    return t.data_ptr()
+
+
+def _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags):
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4:
+        raise ValueError("q, k must be [B, T, Hk, dk] and v [B, T, Hv, dv]")
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype: float32 or bfloat16")
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if beta.dtype != torch.float32 or g.dtype != torch.float32:
+        raise ValueError("beta and g must be float32")
+    a.struct_size = ctypes.sizeof(a)
+    a.abi_version = _abi.GDN_ABI_VERSION
+    a.dtype = _DT[q.dtype]
+    a.B, a.T, a.Hk, a.Hv, a.dk, a.dv = B, T, Hk, Hv, dk, dv
+    a.flags = flags
+    a.q, a.k, a.v, a.beta, a.g = _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g)
+    host = None
+    N = B
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise ValueError("cu_seqlens must be int32")
+        host = cu_seqlens_host if cu_seqlens_host is not None else cu_seqlens.cpu()
+        host = host.to(torch.int32).contiguous()
+        N = host.numel() - 1
+        a.num_seqs = N
+        a.cu_seqlens = _ptr(cu_seqlens)
+        a.cu_seqlens_host = host.data_ptr()
+    if initial_state is not None:
+        if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (N, Hv, dk, dv):
+            raise ValueError(f"initial_state must be float32 [{N}, {Hv}, {dk}, {dv}]")
+        a.S0 = _ptr(initial_state)
+    return N, host  # keep `host` alive until the call returns
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn, status):
+    if status != 0:
+        raise GdnError(fn, status)
+
+
+def _dev_status(device, want):
+    return torch.zeros(1, dtype=torch.int32, device=device) if want else None
+
+
+def _raise_dev_status(fn, st):
+    if st is not None:
+        code = int(st.item())  # synchronises
+        if code != 0:
+            raise GdnError(fn + " (device)", code)
+
+
+def gdn_chunk_fwd_workspace_size(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None,
+                                 initial_state=None, flags: int = 0) -> int:
+    a = GdnFwdArgs()
+    _, host = _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags)
+    n = ctypes.c_size_t(0)
+    _check("gdn_chunk_fwd_workspace_size", _abi.lib().gdn_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return n.value
+
+
+def gdn_chunk_fwd(q, k, v, beta, g, cu_seqlens=None, initial_state=None,
+                  output_final_state: bool = True, *, cu_seqlens_host=None, flags: int = 0,
+                  out=None, final_state=None, workspace=None, check_device_status: bool = False):
+    """Chunked-prefill forward.  Returns (o [B,T,Hv,dv] in q's dtype, S_T [N,Hv,dk,dv] fp32 or None).
+
+    q, k: [B,T,Hk,dk]; v: [B,T,Hv,dv]; beta, g: [B,T,Hv] fp32 (g = raw log decay);
+    cu_seqlens: int32 [N+1] on the device for packed variable-length batches
+    (B == 1), with ``cu_seqlens_host`` its host copy (else one D2H copy is made);
+    initial_state: fp32 [N,Hv,dk,dv] (transposed state H = S^T) or None for zeros.
+    Enqueued on torch's current stream; nothing is synchronised unless
+    ``check_device_status`` is set.
+    """
+    a = GdnFwdArgs()
+    N, host = _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags)
+    B, T = q.shape[:2]
+    Hv, dk, dv = v.shape[2], q.shape[3], v.shape[3]
+    o = out if out is not None else torch.empty(B, T, Hv, dv, dtype=q.dtype, device=q.device)
+    ST = None
+    if output_final_state:
+        ST = final_state if final_state is not None else torch.empty(N, Hv, dk, dv, dtype=torch.float32, device=q.device)
+    a.o, a.ST = _ptr(o), _ptr(ST)
+    st = _dev_status(q.device, check_device_status)
+    a.dev_status = _ptr(st)
+    L = _abi.lib()
+    n = ctypes.c_size_t(0)
+    _check("gdn_chunk_fwd_workspace_size", L.gdn_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    if workspace is None or workspace.numel() < n.value:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=q.device)
+    _check("gdn_chunk_fwd", L.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(workspace.data_ptr()),
+                                            n.value, _stream(q.device)))
+    _raise_dev_status("gdn_chunk_fwd", st)
+    del host
+    return o, ST
+
+
+def gdn_chunk_bwd_workspace_size(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None,
+                                 initial_state=None, flags: int = 0) -> int:
+    a = GdnBwdArgs()
+    _, host = _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags)
+    n = ctypes.c_size_t(0)
+    _check("gdn_chunk_bwd_workspace_size", _abi.lib().gdn_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return n.value
+
+
+def gdn_chunk_bwd(q, k, v, beta, g, do, cu_seqlens=None, initial_state=None, dST=None,
+                  output_dS0: bool = True, *, cu_seqlens_host=None, flags: int = 0,
+                  workspace=None, check_device_status: bool = False):
+    """Chunked-prefill backward.  Returns (dq, dk, dv, dbeta, dg, dS0 or None).
+
+    do: [B,T,Hv,dv] in q's dtype; dST: fp32 [N,Hv,dk,dv] or None (zero).
+    dq/dk are summed over the value heads sharing a q/k head; dg is w.r.t. raw g.
+    """
+    a = GdnBwdArgs()
+    N, host = _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags)
+    if do.shape != v.shape or do.dtype != q.dtype:
+        raise ValueError("do must match v's shape and q's dtype")
+    dev = q.device
+    dq, dk = torch.empty_like(q), torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dbeta, dg = torch.empty_like(beta), torch.empty_like(g)
+    dS0 = torch.empty(N, v.shape[2], q.shape[3], v.shape[3], dtype=torch.float32, device=dev) if output_dS0 else None
+    a.dout, a.dST = _ptr(do), _ptr(dST)
+    a.dq, a.dk_out, a.dv_out = _ptr(dq), _ptr(dk), _ptr(dv)
+    a.dbeta, a.dg, a.dS0 = _ptr(dbeta), _ptr(dg), _ptr(dS0)
+    st = _dev_status(dev, check_device_status)
+    a.dev_status = _ptr(st)
+    L = _abi.lib()
+    n = ctypes.c_size_t(0)
+    _check("gdn_chunk_bwd_workspace_size", L.gdn_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    if workspace is None or workspace.numel() < n.value:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=dev)
+    _check("gdn_chunk_bwd", L.gdn_chunk_bwd(ctypes.byref(a), ctypes.c_void_p(workspace.data_ptr()),
+                                            n.value, _stream(dev)))
+    _raise_dev_status("gdn_chunk_bwd", st)
+    del host
+    return dq, dk, dv, dbeta, dg, dS0
+
+
+def launch_count(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None, initial_state=None,
+                 flags: int = 0, backward: bool = False) -> int:
+    """Kernel launches one gdn_chunk_fwd (or _bwd) call enqueues for these arguments."""
+    a = GdnBwdArgs() if backward else GdnFwdArgs()
+    _, host = _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags)
+    fn = _abi.lib().gdn_chunk_bwd_launch_count if backward else _abi.lib().gdn_chunk_fwd_launch_count
+    return int(fn(ctypes.byref(a)))

@@ -1,0 +1,170 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: chunked-prefill forward and backward of the
+ * Gated Delta Network (GDN) linear-attention layer on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  The FlashQLA pages (news.hamidun.com "Qwen FlashQLA ... Hopper",
+ * section "What is FlashQLA"; dothoosh.com FlashQLA article, opening paragraphs)
+ * describe kernels for the forward and backward passes of GDN in chunked-prefill
+ * mode.  Per sequence and value head the layer is the gated delta rule
+ *
+ *     S_t = exp(g_t) * S_{t-1} * (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,
+ *
+ * with an optional initial state S_0 and the final state S_T returned, so that a
+ * long prompt can be fed as consecutive calls, each call's S_T becoming the
+ * next call's S_0 (news.hamidun.com page, "Chunked Prefill" scenario).
+ *
+ * State layout.  Every state array stores H = S^T, i.e. [dk][dv] row-major per
+ * (sequence, value head), so that o_t = H^T q_t.
+ *
+ * Heads.  q/k have Hk heads and v has Hv heads, Hv a multiple of Hk; value
+ * head h reads q/k head h / (Hv / Hk) (contiguous groups).  beta and g are
+ * per (token, value head).  No 1/sqrt(dk) scale is applied to q.
+ *
+ * Tensors (all device memory unless noted, contiguous, row-major):
+ *   q, k   [B, T, Hk, dk]  dtype        v, o     [B, T, Hv, dv]  dtype
+ *   beta, g [B, T, Hv]     fp32         S0, ST   [N, Hv, dk, dv]  fp32
+ * dtype is fp32 or bf16 (GDN_F32 / GDN_BF16).  g is the raw per-token log decay
+ * (not a cumulative sum); it must be finite.
+ * Variable-length batches: pass cu_seqlens (int32 [N+1], device) together with
+ * its host copy cu_seqlens_host; then B must be 1, T is the total token count
+ * and sequence n owns tokens [cu[n], cu[n+1]).  Without cu_seqlens, N = B.
+ *
+ * Ownership and ordering.  The caller owns every buffer, the workspace
+ * included; the library allocates no memory and keeps no state between calls.
+ * Every entry point is asynchronous on the given stream: it enqueues kernels
+ * and returns without synchronising, so buffers must stay valid until the
+ * stream reaches that point.  Calls on different streams may run from
+ * different host threads.  Inputs are never written.
+ *
+ * Errors.  Arguments are checked on the host before anything is launched;
+ * GDN_ERR_INVALID_ARG / GDN_ERR_UNSUPPORTED / GDN_ERR_WORKSPACE then mean that
+ * nothing was enqueued.  GDN_ERR_CUDA means a launch failed (the CUDA error is
+ * not cleared).  Device-side problems (a bounded wait that expired) are written
+ * as a gdn_status value into *dev_status when dev_status is non-NULL; the
+ * caller reads it after its own synchronisation.  Kernels never trap.  Nothing
+ * throws across this interface.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#define GDN_ABI_VERSION 1u
+#define GDN_CHUNK 64 /* tokens per chunk of the chunked algorithm */
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* NULL / inconsistent / misaligned argument      */
+    GDN_ERR_UNSUPPORTED = 2, /* well-formed but outside what is implemented    */
+    GDN_ERR_WORKSPACE = 3,   /* workspace NULL, too small or not 256-B aligned */
+    GDN_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed           */
+    GDN_ERR_TIMEOUT = 5,     /* device: a bounded wait expired                 */
+    GDN_ERR_DEVICE = 6       /* device: an internal consistency check failed   */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* flags (bitwise or); 0 selects the defaults */
+#define GDN_FLAG_SPLIT_OFF (1u << 0)   /* never split one sequence across SMs      */
+#define GDN_FLAG_SPLIT_FORCE (1u << 1) /* split every sequence into short segments */
+#define GDN_FLAG_PORTABLE (1u << 2)    /* CUDA-core kernels only (no tensor cores) */
+
+/* Arguments of the forward.  struct_size = sizeof(gdn_fwd_args),
+ * abi_version = GDN_ABI_VERSION. */
+typedef struct gdn_fwd_args {
+    uint32_t struct_size;
+    uint32_t abi_version;
+    int32_t dtype;    /* gdn_dtype of q, k, v and o                          */
+    int32_t B, T;     /* batch and tokens per sequence (total tokens if varlen) */
+    int32_t Hk, Hv;   /* q/k heads, value heads (Hv % Hk == 0)                 */
+    int32_t dk, dv;   /* head dims, 1..128 (tensor-core path: 128 x 128 bf16)  */
+    int32_t num_seqs; /* N when cu_seqlens != NULL, else ignored (N = B)       */
+    uint32_t flags;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* beta;
+    const float* g;
+    const int32_t* cu_seqlens;      /* device [N+1] or NULL                      */
+    const int32_t* cu_seqlens_host; /* host copy, required with cu_seqlens       */
+    const float* S0;                /* [N,Hv,dk,dv] or NULL (zero initial state) */
+    void* o;                        /* out [B,T,Hv,dv], dtype                    */
+    float* ST;                      /* out [N,Hv,dk,dv] or NULL (not written)    */
+    int32_t* dev_status;            /* device int32 or NULL                      */
+} gdn_fwd_args;
+
+/* Arguments of the backward: the forward's inputs, the upstream gradients
+ * dout (of o) and dST (of S_T, NULL = zero), and the gradient outputs.  The
+ * backward recomputes the forward internally; no forward tape is passed.
+ * dq/dk hold the sum over the value heads that share a q/k head. */
+typedef struct gdn_bwd_args {
+    uint32_t struct_size;
+    uint32_t abi_version;
+    int32_t dtype;
+    int32_t B, T, Hk, Hv, dk, dv;
+    int32_t num_seqs;
+    uint32_t flags;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* beta;
+    const float* g;
+    const int32_t* cu_seqlens;
+    const int32_t* cu_seqlens_host;
+    const float* S0;   /* [N,Hv,dk,dv] or NULL                 */
+    const void* dout;  /* [B,T,Hv,dv], dtype                   */
+    const float* dST;  /* [N,Hv,dk,dv] or NULL (zero)          */
+    void* dq;          /* out [B,T,Hk,dk], dtype               */
+    void* dk_out;      /* out [B,T,Hk,dk], dtype               */
+    void* dv_out;      /* out [B,T,Hv,dv], dtype               */
+    float* dbeta;      /* out [B,T,Hv] fp32                    */
+    float* dg;         /* out [B,T,Hv] fp32 (w.r.t. raw g)     */
+    float* dS0;        /* out [N,Hv,dk,dv] fp32 or NULL (skip) */
+    int32_t* dev_status;
+} gdn_bwd_args;
+
+/* Bytes of device workspace gdn_chunk_fwd needs for these arguments (the
+ * pointers may be NULL here; only sizes, dtype and cu_seqlens_host are read).
+ * Returns GDN_OK and sets *bytes, or an argument error. */
+GDN_API gdn_status gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args, size_t* bytes);
+
+/* Forward: o and (optionally) S_T from q, k, v, beta, g and (optionally) S0.
+ * workspace: device memory of at least gdn_chunk_fwd_workspace_size() bytes,
+ * 256-byte aligned, caller-owned, contents irrelevant on entry.
+ * stream: a cudaStream_t (CUstream) handle, or NULL for the legacy stream. */
+GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Bytes of device workspace gdn_chunk_bwd needs. */
+GDN_API gdn_status gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args, size_t* bytes);
+
+/* Backward: dq, dk, dv, dbeta, dg and (optionally) dS0 of the forward above
+ * for upstream gradients dout and dST.  Same workspace/stream rules. */
+GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args* args, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+GDN_API const char* gdn_status_string(int status);
+
+/* Number of kernel launches gdn_chunk_fwd / gdn_chunk_bwd enqueue for these
+ * arguments (a pure function of the arguments; -1 on an argument error). */
+GDN_API int gdn_chunk_fwd_launch_count(const gdn_fwd_args* args);
+GDN_API int gdn_chunk_bwd_launch_count(const gdn_bwd_args* args);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,85 @@
+"""GPU backward parity: libgdn's gdn_chunk_bwd against the oracle's float64
+adjoint on the same seeded inputs (dq, dk, dv, dbeta, dg, dS0), whole tensors
+at small sizes and sampled heads at the full backward workload size."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_PORTABLE, gdn_chunk_bwd
+from gated_deltanet_chunked_fwd_b200.inputs import make_inputs, make_workload
+from tests._helpers import TOL, cpu, rel_l2
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NAMES = ["dq", "dk", "dv", "dbeta", "dg", "dS0"]
+
+
+def run(inp, flags=0):
+    res = gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["do"],
+                        cu_seqlens=inp.get("cu_seqlens"), initial_state=inp.get("initial_state"),
+                        dST=inp.get("dST"), cu_seqlens_host=inp.get("cu_seqlens_host"),
+                        flags=flags, check_device_status=True)
+    torch.cuda.synchronize()
+    return res
+
+
+def ref(inp):
+    x = cpu(inp)
+    return oracle.bwd(x["q"], x["k"], x["v"], x["beta"], x["g"], x["do"],
+                      cu_seqlens=x.get("cu_seqlens"), initial_state=x.get("initial_state"),
+                      dST=x.get("dST"))
+
+
+def compare(mine, refs, tol, label=""):
+    for name, a, b in zip(NAMES, mine, refs):
+        err = rel_l2(a, b)
+        assert err < tol, f"{label} {name}: rel-L2 {err:.3e} >= {tol}"
+
+
+CASES = [
+    ("fp32", 1, 1, 1, 1, 16, 16, 0.5),
+    ("fp32", 1, 150, 1, 1, 64, 64, 0.5),
+    ("fp32", 2, 65, 2, 4, 32, 48, 0.5),
+    ("fp32", 1, 200, 1, 2, 128, 128, 0.1),
+    ("bf16", 1, 130, 1, 1, 128, 128, 0.1),
+    ("bf16", 2, 64, 2, 4, 128, 128, None),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c)))
+def test_small_shapes(case):
+    dt, B, T, Hk, Hv, dk, dv, s0 = case
+    inp = make_inputs(B, T, Hk, Hv, dk, dv, dtype=dt, seed=7, s0_std=s0, backward=True, device=DEV)
+    compare(run(inp), ref(inp), TOL[inp["q"].dtype], str(case))
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_varlen_ragged(dt):
+    inp = make_inputs(1, 0, 2, 4, 64, 64, dtype=dt, seed=8, s0_std=0.2, backward=True,
+                      lengths=[3, 64, 0, 129, 1], device=DEV)
+    compare(run(inp), ref(inp), TOL[inp["q"].dtype], dt)
+
+
+def test_zero_upstream_state_gradient_and_no_S0():
+    inp = make_inputs(1, 100, 1, 1, 64, 64, dtype="fp32", seed=9, backward=True, device=DEV)
+    inp["dST"] = None
+    compare(run(inp), ref(inp), 1e-4)
+
+
+def test_reduced_backward_workload_full_oracle():
+    """The backward workload's shape reduced to B=1, T=1024, H=2, d=128, whole tensors."""
+    inp = make_workload(4, seed=0, device=DEV, B=1, T=1024, Hk=2, Hv=2)
+    compare(run(inp), ref(inp), 1e-2, "reduced")
+
+
+def test_backward_workload_full_size_sampled_heads():
+    inp = make_workload(4, seed=0, device=DEV)
+    mine = run(inp)
+    x = cpu(inp)
+    for b, h in [(0, 0), (3, 11)]:
+        sl = lambda t: t[b:b + 1, :, h:h + 1]
+        r = oracle.bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["beta"]), sl(x["g"]), sl(x["do"]),
+                       dST=x["dST"][b:b + 1, h:h + 1])
+        got = [sl(t) for t in mine[:5]] + [mine[5][b:b + 1, h:h + 1]]
+        compare(got, r, 1e-2, f"unit ({b},{h})")
