@@ -75,6 +75,7 @@ gdn_status plan_fwd(const gdn_fwd_args* a, FwdPlan* plan) {
     p.o = a->o;
     p.ST = a->ST;
     p.status = a->dev_status;
+    plan->cu_host = a->cu_seqlens ? a->cu_seqlens_host : nullptr;
     plan->split_mode = (a->flags & GDN_FLAG_SPLIT_OFF) ? 1 : (a->flags & GDN_FLAG_SPLIT_FORCE) ? 2 : 0;
     plan->use_tc = !(a->flags & GDN_FLAG_PORTABLE) && tc_fwd_supported(p);
     const int64_t nc = p.num_chunks;

@@ -73,6 +73,7 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
 struct FwdPlan {
     Problem p;
     bool use_tc;         // tensor-core fused kernel
+    const int32_t* cu_host;  // host copy of cu_seqlens (or nullptr)
     int split_mode;      // 0 auto, 1 off, 2 force
     // workspace carve-up (byte offsets); sizes are 0 when unused
     size_t off_table, off_W, off_U, off_gam, off_Hc, total;

@@ -1,9 +1,726 @@
-// gdn_tc_fwd.cu -- tensor-core (tcgen05 / TMEM / TMA) fused forward (sm_100a).
+// gdn_tc_fwd.cu -- fused tensor-core forward of the chunked gated delta rule
+// for bf16 tensors with dk = dv = 128 on sm_100a.
+//
+// One launch does the whole forward.  Each CTA owns one (sequence, value head,
+// segment of chunks) and walks its chunks in order, keeping the fp32 state in
+// TMEM; per chunk of C = 64 tokens (notation of gdn_internal.cuh):
+//   gates      gamma = cumsum g, Gam, E = exp(gamma_r - gamma_s)       CUDA cores
+//   MMA1       [Q;K] K^T -> Q K^T and K K^T  (M=128 rows: 64 q + 64 k)  tensor core
+//   WY / UT    A = strictly-lower(diag(beta) K K^T o E),
+//              T = (I + A)^-1 (16x16 diagonal blocks by substitution,
+//              block merges by level)                                   CUDA cores, fp32
+//   MMA_W/U    W^T = K^T (T diag(beta Gam))^T,  Ut^T = V^T (T diag(beta))^T
+//   MMA_HW     U^T = Ut^T - H^T W^T  (accumulated onto Ut^T, A negated)
+//   MMA_HQ/UP  O^T = Gam * (H^T Q^T) + U^T P^T,  P = lower-incl(Q K^T o E)
+//   MMA_H      H^T <- Gam_n H^T + (U^T diag(exp(gamma_n - gamma))) K
+// All matrices are oriented so that a 128-wide head dimension is the MMA's M
+// (TMEM lane = dv or dk index), so every MMA is M = 128 with N = 64 or 128.
+// Operands live in shared memory as 128-byte-swizzled tiles; q / k / v tiles
+// come in by TMA (double-buffered: chunk c+1 loads while chunk c computes).
+//
+// Long sequences are split into segments that run on different SMs
+// (gate-driven context parallelism, dothoosh.com FlashQLA article, first
+// innovation): a segment that does not start its sequence starts from a zero
+// state w chunks early, with w the fewest whole chunks whose summed log decay
+// is <= log(eps).  While 0 <= beta |k|^2 <= 2 each token's state map has norm
+// <= exp(g_t), so the truncated past contributes at most eps * |H| to the
+// segment's entry state.  If the decay never reaches eps, or some warm-up
+// token breaks the norm condition, the segment starts exactly from the
+// sequence start (from S0) instead.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
 #include "gdn_internal.cuh"
+#include "gdn_sm100.cuh"
+
 
 namespace gdn {
-bool tc_fwd_supported(const Problem&) { return false; }
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTmemCols = 512;
+// TMEM column map (lane = row of the M = 128 MMA)
+constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk   [0, 128)
+constexpr uint32_t kColR1 = 128;  // Q K^T / K K^T, then W^T               [128, 192)
+constexpr uint32_t kColR2 = 192;  // Ut^T, then U^T                        [192, 256)
+constexpr uint32_t kColHQ = 256;  // H^T Q^T                               [256, 320)
+constexpr uint32_t kColUP = 320;  // U^T P^T                               [320, 384)
+
+// shared memory carve-up (bytes from a 1024-aligned base)
+constexpr uint32_t kStageQK = 0;          // 2 stages x 32 KB: [dk atom][q rows 0-63 | k rows 64-127][128 B]
+constexpr uint32_t kStageV = 65536;       // 2 stages x 16 KB: [dv atom][64 rows][128 B]
+constexpr uint32_t kHb = 98304;           // 32 KB  bf16 H^T: [dk atom][128 dv rows][128 B]
+constexpr uint32_t kPt = 131072;          // 8 KB   P: [64 n rows][64 s]
+constexpr uint32_t kBw = 139264;          // 8 KB   T diag(beta Gam): [n][s]
+constexpr uint32_t kBu = 147456;          // 8 KB   T diag(beta): [n][s]
+constexpr uint32_t kWt = 155648;          // 16 KB  W^T: [128 dk rows][64 tokens]
+constexpr uint32_t kUb = 172032;          // 16 KB  U^T: [128 dv rows][64 tokens]
+constexpr uint32_t kUd = 188416;          // 16 KB  U^T diag(decay)
+constexpr uint32_t kAf = kWt;             // fp32 A [64][65] (aliases Wt/Ub/Ud during the solve)
+constexpr uint32_t kTf = kWt + 16640;     // fp32 T [64][65]
+constexpr uint32_t kYs = kWt + 33280;     // fp32 [3][16][17] solve scratch
+constexpr uint32_t kVec = 204800;         // 8 x 64 floats of per-token vectors
+constexpr uint32_t kBar = kVec + 8 * 256; // barriers and TMEM base
+constexpr uint32_t kSmemBytes = kBar + 64 + 1024;  // + alignment slack
+constexpr int kLd = 65;                   // padded row stride of the fp32 solve matrices
+
+struct TcArgs {
+    Problem p;
+    int L;          // chunks per segment
+    int fixed_segs; // segments per sequence when cu_seqlens is absent
+    int auto_warm;  // 1: gate-driven warm-up for segments that do not start a sequence
+    float log_eps;  // warm-up stops once the summed log decay is <= log_eps
+};
+
+__device__ __forceinline__ int nchunks_of(int64_t len) { return (int)((len + kChunk - 1) / kChunk); }
+
+// bf16 row of 64 values (one 128-byte swizzled row) from fp32 registers
+__device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float* v) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 w;
+        w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
+        w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
+        w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
+        w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
+        *reinterpret_cast<uint4*>(tile + sw128_off(row, c)) = w;
+    }
+}
+
+// One 16x16 output block of the level merge: out = -T_ii * (sum_k A_ik T_kj).
+// Phase 1 writes Y = sum_k A_ik T_kj for the blocks of this level into Ys.
+__device__ __forceinline__ void solve_level_Y(const float* Af, const float* Tf, float* Ys, int d,
+                                              int tid) {
+    const int nblk = 4 - d;  // blocks (i, i-d) for i = d..3
+    for (int o = tid; o < nblk * 256; o += kThreads) {
+        const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
+        const int i = blk + d, j0 = i - d;
+        const float* arow = Af + (16 * i + rr) * kLd;
+        float s = 0.f;
+        for (int j = 16 * j0 + cc; j < 16 * i; ++j) s += arow[j] * Tf[j * kLd + 16 * j0 + cc];
+        Ys[blk * 272 + rr * 17 + cc] = s;
+    }
+}
+
+__device__ __forceinline__ void solve_level_T(float* Tf, const float* Ys, int d, int tid) {
+    const int nblk = 4 - d;
+    for (int o = tid; o < nblk * 256; o += kThreads) {
+        const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
+        const int i = blk + d, j0 = i - d;
+        const float* trow = Tf + (16 * i + rr) * kLd + 16 * i;
+        float s = 0.f;
+        for (int j = 0; j <= rr; ++j) s += trow[j] * Ys[blk * 272 + j * 17 + cc];
+        Tf[(16 * i + rr) * kLd + 16 * j0 + cc] = -s;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const TcArgs args) {
+    const Problem& p = args.p;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    float* vbeta = (float*)(sm + kVec);      // beta
+    float* vgam2 = vbeta + 64;               // gamma * log2(e)
+    float* vGam = vgam2 + 64;                // exp(gamma)
+    float* vbG = vGam + 64;                  // beta * Gam
+    float* vdec = vbG + 64;                  // exp(gamma_n - gamma)
+    float* vred = vdec + 64;                 // reductions
+    float* vgam = vred + 64;                 // gamma (natural log)
+    uint64_t* bar_tma = (uint64_t*)(sm + kBar);  // [2]
+    uint64_t* bar_mma = bar_tma + 2;
+    uint32_t* tmem_slot = (uint32_t*)(bar_mma + 1);
+    int* sflag = (int*)(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int Hv = p.Hv, dv = 128, dk = 128;
+
+    // ---- which (sequence, head, segment) this CTA owns
+    const int h = blockIdx.x % Hv;
+    int sidx = blockIdx.x / Hv;
+    int n = 0, seg = 0, segs_n = 1;
+    int64_t bos = 0, len = 0;
+    if (!p.cu) {
+        n = sidx / args.fixed_segs;
+        seg = sidx % args.fixed_segs;
+        segs_n = args.fixed_segs;
+        bos = (int64_t)n * p.T;
+        len = p.T;
+    } else {
+        // warp-cooperative scan of the per-sequence segment counts (every warp
+        // does the same scan, so no shared state is needed)
+        const int lane = tid & 31;
+        int base = 0;
+        bool found = false;
+        for (int n0 = 0; n0 < p.N && !found; n0 += 32) {
+            const int m = n0 + lane;
+            int s_m = 0;
+            int64_t b_m = 0, l_m = 0;
+            if (m < p.N) {
+                b_m = p.cu[m];
+                l_m = max((int64_t)0, (int64_t)p.cu[m + 1] - b_m);
+                s_m = max(1, (nchunks_of(l_m) + args.L - 1) / args.L);
+            }
+            int incl = s_m;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const bool mine = (m < p.N) && (sidx >= base + incl - s_m) && (sidx < base + incl);
+            const unsigned bal = __ballot_sync(0xffffffffu, mine);
+            if (bal) {
+                const int src = __ffs(bal) - 1;
+                n = __shfl_sync(0xffffffffu, m, src);
+                seg = sidx - (base + __shfl_sync(0xffffffffu, incl - s_m, src));
+                segs_n = __shfl_sync(0xffffffffu, s_m, src);
+                bos = __shfl_sync(0xffffffffu, b_m, src);
+                len = __shfl_sync(0xffffffffu, l_m, src);
+                found = true;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (!found) {  // grid larger than the device offsets allow
+            if (tid == 0) report(p.status, GDN_ERR_DEVICE);
+            return;
+        }
+    }
+    const int hk = h / p.group;
+    const int nck = nchunks_of(len);
+    const int c0 = min(nck, seg * args.L);
+    const int c1 = min(nck, (seg + 1) * args.L);
+
+    // ---- warm-up start (gate-driven); exact start from S0 when seg == 0
+    int cstart = 0;
+    if (seg > 0 && args.auto_warm) {
+        float cum = 0.f;
+        int w = c0;
+        int bad = 0;
+        while (w > 0 && cum > args.log_eps) {
+            --w;
+            const int64_t t0 = bos + (int64_t)w * kChunk;
+            const int lw = (int)min((int64_t)kChunk, len - (int64_t)w * kChunk);
+            // summed log decay of chunk w, and the contraction condition beta |k|^2 <= 2
+            float gsum = 0.f;
+            int viol = 0;
+            {
+                const int r = tid >> 1, half = tid & 1;
+                float nrm = 0.f;
+                if (r < lw) {
+                    const uint4* kr = (const uint4*)((const __nv_bfloat16*)p.k +
+                                                     ((t0 + r) * p.Hk + hk) * dk + half * 64);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 u = kr[c];
+                        const __nv_bfloat162* b2 = (const __nv_bfloat162*)&u;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float2 f = __bfloat1622float2(b2[e]);
+                            nrm += f.x * f.x + f.y * f.y;
+                        }
+                    }
+                }
+                nrm += __shfl_xor_sync(0xffffffffu, nrm, 1);
+                if (half == 0 && r < lw) {
+                    const float b = p.beta[(t0 + r) * Hv + h];
+                    gsum = p.g[(t0 + r) * Hv + h];
+                    if (!(b >= 0.f && b * nrm <= 2.f)) viol = 1;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+            viol = __syncthreads_or(viol);
+            if ((tid & 31) == 0) vred[warp] = gsum;
+            __syncthreads();
+            cum += vred[0] + vred[1] + vred[2] + vred[3];
+            __syncthreads();
+            bad |= viol;
+        }
+        cstart = (cum > args.log_eps || bad) ? 0 : w;
+    } else if (seg > 0) {
+        cstart = 0;  // no warm-up rule: replay the whole prefix exactly
+    }
+    const bool exact = (cstart == 0);
+
+    // ---- set-up: barriers, TMEM
+    if (tid == 0) {
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        *sflag = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t sbase = smem_u32(sm);
+    bool ok = true;
+
+    // ---- initial state: H^T (lane = dv index m = tid) from S0 or zero
+    {
+        const int m = tid;
+        const float* s0 = (exact && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
+        float v[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(int64_t)(32 * q4 + e) * dv + m] : 0.f;
+            tmem_st32(tmem + lane_off + kColH + 32 * q4, v);
+            // bf16 copy: row m of Hb, dk chunk (32*q4 .. +31) -> atom q4/2, chunks 4*(q4%2)..+3
+            uint8_t* atom = sm + kHb + (q4 >> 1) * 16384;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint4 w;
+                w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
+                w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
+                w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
+                w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
+                *reinterpret_cast<uint4*>(atom + sw128_off(m, 4 * (q4 & 1) + c)) = w;
+            }
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int nk = c1 - cstart;  // chunks this CTA walks (warm-up + own)
+    auto issue_tma = [&](int k) {
+        const int c = cstart + k;
+        const int stage = k & 1;
+        const int t0 = (int)(bos + (int64_t)c * kChunk);
+        uint8_t* qk = sm + kStageQK + stage * 32768;
+        uint8_t* vv = sm + kStageV + stage * 16384;
+        mbar_arrive_expect_tx(&bar_tma[stage], 49152);
+        for (int a = 0; a < 2; ++a) {
+            tma_load_3d(qk + a * 16384, &tm_q, &bar_tma[stage], 64 * a, hk, t0);
+            tma_load_3d(qk + a * 16384 + 8192, &tm_k, &bar_tma[stage], 64 * a, hk, t0);
+            tma_load_3d(vv + a * 8192, &tm_v, &bar_tma[stage], 64 * a, h, t0);
+        }
+    };
+    if (tid == 0 && nk > 0) issue_tma(0);
+
+    uint32_t mma_phase = 0;
+    const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
+    const uint32_t id_mn_n64 = idesc_bf16(128, 64, 1, 0);        // A MN-major
+    const uint32_t id_neg_bmn_n64 = idesc_bf16(128, 64, 0, 1, 1); // -A, B MN-major
+    const uint32_t id_bmn_n128 = idesc_bf16(128, 128, 0, 1);      // B MN-major, N = 128
+    const float LOG2E = 1.4426950408889634f;
+
+    for (int k = 0; k < nk && ok; ++k) {
+        const int c = cstart + k;
+        const int stage = k & 1;
+        const bool emit = c >= c0;
+        const int64_t t0 = bos + (int64_t)c * kChunk;
+        const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+        const uint32_t sQK = sbase + kStageQK + stage * 32768;
+        const uint32_t sV = sbase + kStageV + stage * 16384;
+
+        // gates of this chunk (threads 0..63): beta, gamma = cumsum g (padding: g = 0)
+        if (tid < 64) {
+            const int r = tid;
+            const float b = r < lc ? p.beta[(t0 + r) * Hv + h] : 0.f;
+            float x = r < lc ? p.g[(t0 + r) * Hv + h] : 0.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if ((r & 31) >= o) x += y;
+            }
+            vbeta[r] = b;
+            vgam[r] = x;  // per-warp inclusive scan, fixed below
+        }
+        __syncthreads();
+        if (tid >= 32 && tid < 64) vgam[tid] += vgam[31];
+        __syncthreads();
+        if (tid < 64) {
+            const int r = tid;
+            const float gl = vgam[63];
+            const float gr = vgam[r];
+            vGam[r] = expf(gr);
+            vbG[r] = vbeta[r] * expf(gr);
+            vdec[r] = expf(gl - gr);
+            vgam2[r] = gr * LOG2E;
+        }
+        __syncthreads();
+
+        // MMA1 (+ MMA_HQ) once this chunk's tiles have landed
+        ok = __syncthreads_and(mbar_wait(&bar_tma[stage], (k >> 1) & 1));
+        if (!ok) break;
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + koff, 16, 1024),
+                            desc_sw128(sQK + 8192 + koff, 16, 1024), id_n64, j > 0);
+            }
+            if (emit) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                    mma_bf16_ss(tmem + kColHQ, desc_sw128(sbase + kHb + koff, 16, 1024),
+                                desc_sw128(sQK + koff, 16, 1024), id_n64, j > 0);
+                }
+            }
+            mma_commit(bar_mma);
+            if (k + 1 < nk) issue_tma(k + 1);  // stage k+1 was freed by chunk k-1's MMAs
+        }
+        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
+        mma_phase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+
+        // P (rows 0..63) and A (rows 64..127) from Q K^T / K K^T
+        {
+            float v[64];
+            tmem_ld32(tmem + lane_off + kColR1, v);
+            tmem_ld32(tmem + lane_off + kColR1 + 32, v + 32);
+            const int r = tid & 63;
+            const float gr = vgam2[r];
+            if (tid < 64) {
+#pragma unroll
+                for (int s = 0; s < 64; ++s)
+                    v[s] = (s <= r && r < lc) ? v[s] * exp2f(gr - vgam2[s]) : 0.f;
+                store_row64(sm + kPt, r, v);
+            } else {
+                float* Af = (float*)(sm + kAf);
+                const float br = vbeta[r];
+#pragma unroll
+                for (int s = 0; s < 64; ++s)
+                    Af[r * kLd + s] = (s < r && r < lc) ? br * v[s] * exp2f(gr - vgam2[s]) : 0.f;
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // T = (I + A)^-1 in fp32: diagonal 16x16 blocks, then three merge levels
+        {
+            const float* Af = (const float*)(sm + kAf);
+            float* Tf = (float*)(sm + kTf);
+            float* Ys = (float*)(sm + kYs);
+            if (tid < 64) {
+                const int b = tid >> 4, cc = tid & 15;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float s = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+                    for (int j = 0; j < r; ++j) s -= Af[(16 * b + r) * kLd + 16 * b + j] * x[j];
+                    x[r] = (r < cc) ? 0.f : s;
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * kLd + 16 * b + cc] = x[r];
+            }
+            __syncthreads();
+            for (int d = 1; d <= 3; ++d) {
+                solve_level_Y(Af, Tf, Ys, d, tid);
+                __syncthreads();
+                solve_level_T(Tf, Ys, d, tid);
+                __syncthreads();
+            }
+            // B operands of MMA_W / MMA_U: rows n, columns s <= n
+            const int nrow = tid >> 1, half = tid & 1;
+            float vw[32], vu[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int s = 32 * half + e;
+                const float t = (s <= nrow) ? Tf[nrow * kLd + s] : 0.f;
+                vw[e] = t * vbG[s];
+                vu[e] = t * vbeta[s];
+            }
+#pragma unroll
+            for (int cch = 0; cch < 4; ++cch) {
+                uint4 w, u;
+                w.x = pack_bf16(vw[8 * cch + 0], vw[8 * cch + 1]);
+                w.y = pack_bf16(vw[8 * cch + 2], vw[8 * cch + 3]);
+                w.z = pack_bf16(vw[8 * cch + 4], vw[8 * cch + 5]);
+                w.w = pack_bf16(vw[8 * cch + 6], vw[8 * cch + 7]);
+                u.x = pack_bf16(vu[8 * cch + 0], vu[8 * cch + 1]);
+                u.y = pack_bf16(vu[8 * cch + 2], vu[8 * cch + 3]);
+                u.z = pack_bf16(vu[8 * cch + 4], vu[8 * cch + 5]);
+                u.w = pack_bf16(vu[8 * cch + 6], vu[8 * cch + 7]);
+                const uint32_t off = sw128_off(nrow, 4 * half + cch);
+                *reinterpret_cast<uint4*>(sm + kBw + off) = w;
+                *reinterpret_cast<uint4*>(sm + kBu + off) = u;
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // MMA_W: W^T = K^T Bw^T  and  MMA_U: Ut^T = V^T Bu^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
+                            desc_sw128(sbase + kBw + j * 32, 16, 1024), id_mn_n64, j > 0);
+                mma_bf16_ss(tmem + kColR2, desc_sw128(sV + j * 2048, 8192, 1024),
+                            desc_sw128(sbase + kBu + j * 32, 16, 1024), id_mn_n64, j > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
+        mma_phase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+
+        // W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
+        {
+            float v[64];
+            tmem_ld32(tmem + lane_off + kColR1, v);
+            tmem_ld32(tmem + lane_off + kColR1 + 32, v + 32);
+            store_row64(sm + kWt, tid, v);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // MMA_HW: U^T = Ut^T - H^T W^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                mma_bf16_ss(tmem + kColR2, desc_sw128(sbase + kHb + koff, 16, 1024),
+                            desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_neg_bmn_n64, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
+        mma_phase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+
+        // U^T (lane = dv index) -> Ub and Ud = U^T diag(decay); H^T <- Gam_n H^T
+        {
+            float v[64];
+            tmem_ld32(tmem + lane_off + kColR2, v);
+            tmem_ld32(tmem + lane_off + kColR2 + 32, v + 32);
+            if (emit) store_row64(sm + kUb, tid, v);
+#pragma unroll
+            for (int s = 0; s < 64; ++s) v[s] *= vdec[s];
+            store_row64(sm + kUd, tid, v);
+            const float Gn = vGam[63];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                tmem_ld32(tmem + lane_off + kColH + 32 * q4, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= Gn;
+                tmem_st32(tmem + lane_off + kColH + 32 * q4, v);
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // MMA_UP: U^T P^T;  MMA_H: H^T += Ud K
+        if (tid == 0) {
+            tc_fence_after();
+            if (emit) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_bf16_ss(tmem + kColUP, desc_sw128(sbase + kUb + j * 32, 16, 1024),
+                                desc_sw128(sbase + kPt + j * 32, 16, 1024), id_n64, j > 0);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                mma_bf16_ss(tmem + kColH, desc_sw128(sbase + kUd + j * 32, 16, 1024),
+                            desc_sw128(sQK + 8192 + j * 2048, 16384, 1024), id_bmn_n128, 1);
+            mma_commit(bar_mma);
+        }
+        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
+        mma_phase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+
+        // output o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n]
+        if (emit) {
+            const int m = tid;
+            __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float hq[32], up[32];
+                tmem_ld32(tmem + lane_off + kColHQ + 32 * half, hq);
+                tmem_ld32(tmem + lane_off + kColUP + 32 * half, up);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int nn = 32 * half + e;
+                    if (nn < lc) op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(vGam[nn] * hq[e] + up[e]);
+                }
+            }
+        }
+        // bf16 copy of the new state for the next chunk's MMAs
+        {
+            float v[32];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                tmem_ld32(tmem + lane_off + kColH + 32 * q4, v);
+                uint8_t* atom = sm + kHb + (q4 >> 1) * 16384;
+#pragma unroll
+                for (int cch = 0; cch < 4; ++cch) {
+                    uint4 w;
+                    w.x = pack_bf16(v[8 * cch + 0], v[8 * cch + 1]);
+                    w.y = pack_bf16(v[8 * cch + 2], v[8 * cch + 3]);
+                    w.z = pack_bf16(v[8 * cch + 4], v[8 * cch + 5]);
+                    w.w = pack_bf16(v[8 * cch + 6], v[8 * cch + 7]);
+                    *reinterpret_cast<uint4*>(atom + sw128_off(tid, 4 * (q4 & 1) + cch)) = w;
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (!ok) {
+        if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
+    } else if (p.ST && seg == segs_n - 1) {
+        // final state S_T = H (stored [dk][dv]): thread m writes column m
+        float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + tid;
+        float v[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            tmem_ld32(tmem + lane_off + kColH + 32 * q4, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) st[(int64_t)(32 * q4 + e) * dv] = v[e];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;  // resolved once per process (a driver entry point)
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)ptr;
+    }
+    return fn;
+}
+
+// [T_total, H, 128] bf16 viewed as (d, head, token); box 64 x 1 x 64, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, int64_t T_total, int H) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)std::max<int64_t>(T_total, 1)};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// Segments of L chunks: count and estimated makespan in chunk-steps.
+struct SplitChoice {
+    int L;
+    int64_t ctas;
+};
+
+SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int split_mode, int nsm) {
+    int maxc = 1;
+    for (int c : nchunks) maxc = std::max(maxc, c);
+    auto count = [&](int L) {
+        int64_t s = 0;
+        for (int c : nchunks) s += std::max(1, (c + L - 1) / L);
+        return s * Hv;
+    };
+    if (split_mode == 1) return {maxc, count(maxc)};
+    if (split_mode == 2) {
+        const int L = std::max(1, std::min(maxc, 2));
+        return {L, count(L)};
+    }
+    int bestL = maxc;
+    double best = 1e300;
+    for (int L = 1; L <= maxc; ++L) {
+        const int64_t S = count(L);
+        const double waves = std::ceil((double)S / nsm);
+        const double est = waves * (L + (L < maxc ? 1.5 : 0.0));
+        if (est < best - 1e-9 || (std::fabs(est - best) < 1e-9 && L > bestL)) {
+            best = est;
+            bestL = L;
+        }
+    }
+    return {bestL, count(bestL)};
+}
+
+std::vector<int> chunk_counts(const Problem& p, const int32_t* cu_host) {
+    std::vector<int> v;
+    if (!p.cu) {
+        v.assign(p.N, (p.T + kChunk - 1) / kChunk);
+    } else {
+        v.resize(p.N);
+        for (int n = 0; n < p.N; ++n) v[n] = (cu_host[n + 1] - cu_host[n] + kChunk - 1) / kChunk;
+    }
+    return v;
+}
+
+}  // namespace
+
+bool tc_fwd_supported(const Problem& p) {
+    return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128;
+}
+
 size_t tc_fwd_workspace(const Problem&) { return 0; }
-int tc_fwd_launches(const Problem&) { return 0; }
-gdn_status launch_fwd_tc(const FwdPlan&, char*, cudaStream_t) { return GDN_ERR_UNSUPPORTED; }
+int tc_fwd_launches(const Problem&) { return 1; }
+
+gdn_status launch_fwd_tc(const FwdPlan& plan, char*, cudaStream_t s) {
+    const Problem& p = plan.p;
+    TcArgs a;
+    a.p = p;
+    const std::vector<int> nck = chunk_counts(p, plan.cu_host);
+    const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count());
+    a.L = sc.L;
+    a.fixed_segs = p.cu ? 0 : std::max(1, (nck.empty() ? 1 : (nck[0] + sc.L - 1) / sc.L));
+    a.auto_warm = plan.split_mode == 1 ? 0 : 1;
+    a.log_eps = (float)(-30.0 * std::log(2.0));
+    CUtensorMap mq, mk, mv;
+    const int64_t Tt = std::max<int64_t>(p.T_total, 1);
+    if (!make_map(&mq, p.q, Tt, p.Hk) || !make_map(&mk, p.k, Tt, p.Hk) || !make_map(&mv, p.v, Tt, p.Hv))
+        return GDN_ERR_CUDA;
+    if (cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    gdn_fwd_tc_kernel<<<(unsigned)sc.ctas, kThreads, kSmemBytes, s>>>(mq, mk, mv, a);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 }  // namespace gdn

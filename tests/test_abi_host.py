@@ -80,7 +80,9 @@ def test_misaligned_tensor_is_rejected(field, offset):
 
 
 def test_workspace_checks():
-    a = fwd_args()
+    # the tensor-core path (bf16, 128 x 128) needs no workspace; the portable one does
+    assert ws_size(fwd_args()) == (OK, 0)
+    a = fwd_args(flags=_abi.GDN_FLAG_PORTABLE)
     st, need = ws_size(a)
     assert st == OK and need > 0 and need % 256 == 0
     assert call_fwd(a, ws=0) == WORKSPACE
@@ -104,8 +106,8 @@ def test_varlen_host_offsets_are_checked():
 
 def test_workspace_grows_with_tokens_and_launch_count():
     L = _abi.lib()
-    s1 = ws_size(fwd_args(T=256))[1]
-    s2 = ws_size(fwd_args(T=1024))[1]
+    s1 = ws_size(fwd_args(T=256, flags=_abi.GDN_FLAG_PORTABLE))[1]
+    s2 = ws_size(fwd_args(T=1024, flags=_abi.GDN_FLAG_PORTABLE))[1]
     assert s2 > s1
     assert L.gdn_chunk_fwd_launch_count(ctypes.byref(fwd_args())) >= 1
     assert L.gdn_chunk_fwd_launch_count(ctypes.byref(fwd_args(Hv=3))) == -1
