@@ -44,7 +44,7 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // 8 warps: warps w and w+4 share TMEM lane quarter w%4
 constexpr int kTmemCols = 512;
 // TMEM column map (lane = row of the M = 128 MMA)
 constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk   [0, 128)
@@ -63,13 +63,14 @@ constexpr uint32_t kBu = 147456;          // 8 KB   T diag(beta): [n][s]
 constexpr uint32_t kWt = 155648;          // 16 KB  W^T: [128 dk rows][64 tokens]
 constexpr uint32_t kUb = 172032;          // 16 KB  U^T: [128 dv rows][64 tokens]
 constexpr uint32_t kUd = 188416;          // 16 KB  U^T diag(decay)
-constexpr uint32_t kAf = kWt;             // fp32 A [64][65] (aliases Wt/Ub/Ud during the solve)
-constexpr uint32_t kTf = kWt + 16640;     // fp32 T [64][65]
-constexpr uint32_t kYs = kWt + 33280;     // fp32 [3][16][17] solve scratch
-constexpr uint32_t kVec = 204800;         // 8 x 64 floats of per-token vectors
-constexpr uint32_t kBar = kVec + 8 * 256; // barriers and TMEM base
+constexpr int kLd = 68;                   // row stride (floats) of the fp32 solve matrices
+constexpr uint32_t kAf = kWt;             // fp32 A [64][68] (aliases Wt/Ub/Ud during the solve)
+constexpr uint32_t kTf = kWt + 64 * kLd * 4;  // fp32 T [64][68]
+constexpr uint32_t kYs = kTf + 64 * kLd * 4;  // fp32 [3][16][17] solve scratch
+constexpr uint32_t kVec = 204800;         // 16 x 64 floats of per-token vectors
+constexpr uint32_t kBar = kVec + 16 * 256; // barriers and TMEM base
 constexpr uint32_t kSmemBytes = kBar + 64 + 1024;  // + alignment slack
-constexpr int kLd = 65;                   // padded row stride of the fp32 solve matrices
+static_assert(kYs + 3 * 272 * 4 <= kVec, "solve scratch overlaps the vectors");
 
 struct TcArgs {
     Problem p;
@@ -81,43 +82,61 @@ struct TcArgs {
 
 __device__ __forceinline__ int nchunks_of(int64_t len) { return (int)((len + kChunk - 1) / kChunk); }
 
-// bf16 row of 64 values (one 128-byte swizzled row) from fp32 registers
-__device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float* v) {
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    uint4 w;
+    w.x = pack_bf16(v[0], v[1]);
+    w.y = pack_bf16(v[2], v[3]);
+    w.z = pack_bf16(v[4], v[5]);
+    w.w = pack_bf16(v[6], v[7]);
+    return w;
+}
+
+// 32 fp32 values -> 4 swizzled 16-byte chunks (chunk0..chunk0+3) of one 128-byte row
+__device__ __forceinline__ void store_row32(uint8_t* tile, int row, int chunk0, const float* v) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 w;
-        w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
-        w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
-        w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
-        w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
-        *reinterpret_cast<uint4*>(tile + sw128_off(row, c)) = w;
+    for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(tile + sw128_off(row, chunk0 + c)) = pack8(v + 8 * c);
+}
+
+// Level-D merge of the blocked inverse (D = 1, 2, 3), for the blocks (i, i-D), i = D..3:
+//   Y = sum_{k=i-D}^{i-1} A_ik T_k,i-D   then   T_i,i-D = -T_ii Y.
+// The diagonal blocks of T store their upper triangles as zeros, so both sums
+// run over full 16-wide blocks with fixed trip counts.
+template <int D>
+__device__ __forceinline__ void solve_level_Y(const float* Af, const float* Tf, float* Ys, int tid) {
+    constexpr int kOut = (4 - D) * 256;
+#pragma unroll
+    for (int q = 0; q < (kOut + kThreads - 1) / kThreads; ++q) {
+        const int o = tid + q * kThreads;
+        if (o < kOut) {
+            const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
+            const int i = blk + D, j0 = i - D;
+            const float* arow = Af + (16 * i + rr) * kLd + 16 * j0;
+            const float* tcol = Tf + (16 * j0) * kLd + 16 * j0 + cc;
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 16 * D; ++j) s[j & 3] += arow[j] * tcol[j * kLd];
+            Ys[blk * 272 + rr * 17 + cc] = (s[0] + s[1]) + (s[2] + s[3]);
+        }
     }
 }
 
-// One 16x16 output block of the level merge: out = -T_ii * (sum_k A_ik T_kj).
-// Phase 1 writes Y = sum_k A_ik T_kj for the blocks of this level into Ys.
-__device__ __forceinline__ void solve_level_Y(const float* Af, const float* Tf, float* Ys, int d,
-                                              int tid) {
-    const int nblk = 4 - d;  // blocks (i, i-d) for i = d..3
-    for (int o = tid; o < nblk * 256; o += kThreads) {
-        const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-        const int i = blk + d, j0 = i - d;
-        const float* arow = Af + (16 * i + rr) * kLd;
-        float s = 0.f;
-        for (int j = 16 * j0 + cc; j < 16 * i; ++j) s += arow[j] * Tf[j * kLd + 16 * j0 + cc];
-        Ys[blk * 272 + rr * 17 + cc] = s;
-    }
-}
-
-__device__ __forceinline__ void solve_level_T(float* Tf, const float* Ys, int d, int tid) {
-    const int nblk = 4 - d;
-    for (int o = tid; o < nblk * 256; o += kThreads) {
-        const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-        const int i = blk + d, j0 = i - d;
-        const float* trow = Tf + (16 * i + rr) * kLd + 16 * i;
-        float s = 0.f;
-        for (int j = 0; j <= rr; ++j) s += trow[j] * Ys[blk * 272 + j * 17 + cc];
-        Tf[(16 * i + rr) * kLd + 16 * j0 + cc] = -s;
+template <int D>
+__device__ __forceinline__ void solve_level_T(float* Tf, const float* Ys, int tid) {
+    constexpr int kOut = (4 - D) * 256;
+#pragma unroll
+    for (int q = 0; q < (kOut + kThreads - 1) / kThreads; ++q) {
+        const int o = tid + q * kThreads;
+        if (o < kOut) {
+            const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
+            const int i = blk + D, j0 = i - D;
+            const float* trow = Tf + (16 * i + rr) * kLd + 16 * i;
+            const float* ycol = Ys + blk * 272 + cc;
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) s[j & 3] += trow[j] * ycol[j * 17];
+            Tf[(16 * i + rr) * kLd + 16 * j0 + cc] = -((s[0] + s[1]) + (s[2] + s[3]));
+        }
     }
 }
 
@@ -128,18 +147,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* vbeta = (float*)(sm + kVec);      // beta
-    float* vgam2 = vbeta + 64;               // gamma * log2(e)
-    float* vGam = vgam2 + 64;                // exp(gamma)
+    float* vgam = vbeta + 64;                // gamma (natural log)
+    float* vGam = vgam + 64;                 // exp(gamma)
     float* vbG = vGam + 64;                  // beta * Gam
     float* vdec = vbG + 64;                  // exp(gamma_n - gamma)
-    float* vred = vdec + 64;                 // reductions
-    float* vgam = vred + 64;                 // gamma (natural log)
+    float* va = vdec + 64;                   // row factor of E (or gamma * log2 e)
+    float* vb = va + 64;                     // column factor of E
+    float* vred = vb + 64;                   // reductions (8 warps)
     uint64_t* bar_tma = (uint64_t*)(sm + kBar);  // [2]
     uint64_t* bar_mma = bar_tma + 2;
     uint32_t* tmem_slot = (uint32_t*)(bar_mma + 1);
-    int* sflag = (int*)(tmem_slot + 1);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = warp >> 2;                    // which half of the columns this thread takes
+    const int row = ((warp & 3) << 5) | lane;    // TMEM lane (= MMA row) this thread reads
     const int Hv = p.Hv, dv = 128, dk = 128;
 
     // ---- which (sequence, head, segment) this CTA owns
@@ -156,7 +177,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // warp-cooperative scan of the per-sequence segment counts (every warp
         // does the same scan, so no shared state is needed)
-        const int lane = tid & 31;
         int base = 0;
         bool found = false;
         for (int n0 = 0; n0 < p.N && !found; n0 += 32) {
@@ -208,44 +228,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t t0 = bos + (int64_t)w * kChunk;
             const int lw = (int)min((int64_t)kChunk, len - (int64_t)w * kChunk);
             // summed log decay of chunk w, and the contraction condition beta |k|^2 <= 2
-            float gsum = 0.f;
+            const int r = tid >> 2, q = tid & 3;
+            float nrm = 0.f, gsum = 0.f;
             int viol = 0;
-            {
-                const int r = tid >> 1, half = tid & 1;
-                float nrm = 0.f;
-                if (r < lw) {
-                    const uint4* kr = (const uint4*)((const __nv_bfloat16*)p.k +
-                                                     ((t0 + r) * p.Hk + hk) * dk + half * 64);
+            if (r < lw) {
+                const uint4* kr = (const uint4*)((const __nv_bfloat16*)p.k +
+                                                 ((t0 + r) * p.Hk + hk) * dk + q * 32);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 u = kr[c];
-                        const __nv_bfloat162* b2 = (const __nv_bfloat162*)&u;
+                for (int c = 0; c < 4; ++c) {
+                    uint4 u = kr[c];
+                    const __nv_bfloat162* b2 = (const __nv_bfloat162*)&u;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float2 f = __bfloat1622float2(b2[e]);
-                            nrm += f.x * f.x + f.y * f.y;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        float2 f = __bfloat1622float2(b2[e]);
+                        nrm += f.x * f.x + f.y * f.y;
                     }
                 }
-                nrm += __shfl_xor_sync(0xffffffffu, nrm, 1);
-                if (half == 0 && r < lw) {
-                    const float b = p.beta[(t0 + r) * Hv + h];
-                    gsum = p.g[(t0 + r) * Hv + h];
-                    if (!(b >= 0.f && b * nrm <= 2.f)) viol = 1;
-                }
+            }
+            nrm += __shfl_xor_sync(0xffffffffu, nrm, 1);
+            nrm += __shfl_xor_sync(0xffffffffu, nrm, 2);
+            if (q == 0 && r < lw) {
+                const float b = p.beta[(t0 + r) * Hv + h];
+                gsum = p.g[(t0 + r) * Hv + h];
+                if (!(b >= 0.f && b * nrm <= 2.f)) viol = 1;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
             viol = __syncthreads_or(viol);
-            if ((tid & 31) == 0) vred[warp] = gsum;
+            if (lane == 0) vred[warp] = gsum;
             __syncthreads();
-            cum += vred[0] + vred[1] + vred[2] + vred[3];
+            float tot = 0.f;
+#pragma unroll
+            for (int i = 0; i < kThreads / 32; ++i) tot += vred[i];
+            cum += tot;
             __syncthreads();
             bad |= viol;
         }
         cstart = (cum > args.log_eps || bad) ? 0 : w;
-    } else if (seg > 0) {
-        cstart = 0;  // no warm-up rule: replay the whole prefix exactly
     }
     const bool exact = (cstart == 0);
 
@@ -258,7 +277,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        *sflag = 0;
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -268,31 +286,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lane quarter
     const uint32_t sbase = smem_u32(sm);
     bool ok = true;
 
-    // ---- initial state: H^T (lane = dv index m = tid) from S0 or zero
+    // ---- initial state: H^T (lane = dv index m) from S0 or zero; this thread
+    //      takes dk columns [64 wg, 64 wg + 64)
     {
-        const int m = tid;
+        const int m = row;
         const float* s0 = (exact && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
         float v[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int hf = 0; hf < 2; ++hf) {
+            const int col0 = 64 * wg + 32 * hf;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(int64_t)(32 * q4 + e) * dv + m] : 0.f;
-            tmem_st32(tmem + lane_off + kColH + 32 * q4, v);
-            // bf16 copy: row m of Hb, dk chunk (32*q4 .. +31) -> atom q4/2, chunks 4*(q4%2)..+3
-            uint8_t* atom = sm + kHb + (q4 >> 1) * 16384;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint4 w;
-                w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
-                w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
-                w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
-                w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
-                *reinterpret_cast<uint4*>(atom + sw128_off(m, 4 * (q4 & 1) + c)) = w;
-            }
+            for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(int64_t)(col0 + e) * dv + m] : 0.f;
+            tmem_st32(tl + kColH + col0, v);
+            store_row32(sm + kHb + wg * 16384, m, 4 * hf, v);
         }
     }
     fence_proxy_async();
@@ -316,6 +326,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     if (tid == 0 && nk > 0) issue_tma(0);
 
+    // gates of the next chunk, loaded one chunk ahead (threads 0..63)
+    float nxt_b = 0.f, nxt_g = 0.f;
+    auto load_gates = [&](int k) {
+        const int c = cstart + k;
+        const int64_t t0 = bos + (int64_t)c * kChunk;
+        const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+        nxt_b = tid < lc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
+        nxt_g = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;  // padding: g = 0
+    };
+    if (tid < 64 && nk > 0) load_gates(0);
+
     uint32_t mma_phase = 0;
     const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
     const uint32_t id_mn_n64 = idesc_bf16(128, 64, 1, 0);        // A MN-major
@@ -332,34 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sQK = sbase + kStageQK + stage * 32768;
         const uint32_t sV = sbase + kStageV + stage * 16384;
 
-        // gates of this chunk (threads 0..63): beta, gamma = cumsum g (padding: g = 0)
-        if (tid < 64) {
-            const int r = tid;
-            const float b = r < lc ? p.beta[(t0 + r) * Hv + h] : 0.f;
-            float x = r < lc ? p.g[(t0 + r) * Hv + h] : 0.f;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if ((r & 31) >= o) x += y;
-            }
-            vbeta[r] = b;
-            vgam[r] = x;  // per-warp inclusive scan, fixed below
-        }
-        __syncthreads();
-        if (tid >= 32 && tid < 64) vgam[tid] += vgam[31];
-        __syncthreads();
-        if (tid < 64) {
-            const int r = tid;
-            const float gl = vgam[63];
-            const float gr = vgam[r];
-            vGam[r] = expf(gr);
-            vbG[r] = vbeta[r] * expf(gr);
-            vdec[r] = expf(gl - gr);
-            vgam2[r] = gr * LOG2E;
-        }
-        __syncthreads();
-
-        // MMA1 (+ MMA_HQ) once this chunk's tiles have landed
+        // ---- MMA1 once this chunk's tiles have landed (the gates below overlap it)
         ok = __syncthreads_and(mbar_wait(&bar_tma[stage], (k >> 1) & 1));
         if (!ok) break;
         if (tid == 0) {
@@ -370,46 +364,81 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + koff, 16, 1024),
                             desc_sw128(sQK + 8192 + koff, 16, 1024), id_n64, j > 0);
             }
-            if (emit) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                    mma_bf16_ss(tmem + kColHQ, desc_sw128(sbase + kHb + koff, 16, 1024),
-                                desc_sw128(sQK + koff, 16, 1024), id_n64, j > 0);
-                }
-            }
             mma_commit(bar_mma);
             if (k + 1 < nk) issue_tma(k + 1);  // stage k+1 was freed by chunk k-1's MMAs
         }
+        // ---- gates: gamma = cumsum g (per-warp scan, then warp 1 adds warp 0's total)
+        if (tid < 64) {
+            float x = nxt_g;
+            const float b = nxt_b;
+            if (k + 1 < nk) load_gates(k + 1);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            vbeta[tid] = b;
+            vgam[tid] = x;
+        }
+        __syncthreads();
+        // E_rs = exp(gamma_r - gamma_s) = a_r * b_s with a_r = exp(gamma_r - gamma_31),
+        // b_s = exp(gamma_31 - gamma_s), used when every |gamma - gamma_31| < 80 (both
+        // factors then stay far inside the fp32 range); else E is one exp2 per entry.
+        float gr = 0.f, gm = 0.f;
+        if (tid < 64) {
+            const int r = tid;
+            gr = vgam[r] + (r >= 32 ? vgam[31] : 0.f);
+            gm = vgam[31];
+            const float gl = vgam[63] + vgam[31];
+            vGam[r] = expf(gr);
+            vbG[r] = vbeta[r] * expf(gr);
+            vdec[r] = expf(gl - gr);
+        }
+        const bool fac = !__syncthreads_or(tid < 64 && !(fabsf(gr - gm) < 80.f));
+        if (tid < 64) {
+            va[tid] = fac ? expf(gr - gm) : gr * LOG2E;
+            vb[tid] = fac ? expf(gm - gr) : gr * LOG2E;
+        }
+        __syncthreads();
+
         ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
         mma_phase ^= 1;
         if (!ok) break;
         tc_fence_after();
 
-        // P (rows 0..63) and A (rows 64..127) from Q K^T / K K^T
+        // ---- P (rows 0..63) and A (rows 64..127); this thread: columns [32 wg, 32 wg + 32)
         {
-            float v[64];
-            tmem_ld32(tmem + lane_off + kColR1, v);
-            tmem_ld32(tmem + lane_off + kColR1 + 32, v + 32);
-            const int r = tid & 63;
-            const float gr = vgam2[r];
-            if (tid < 64) {
+            float v[32];
+            tmem_ld32(tl + kColR1 + 32 * wg, v);
+            const int r = row & 63;
+            const int s0 = 32 * wg;
+            const float ar = va[r];
+            if (row < 64) {
 #pragma unroll
-                for (int s = 0; s < 64; ++s)
-                    v[s] = (s <= r && r < lc) ? v[s] * exp2f(gr - vgam2[s]) : 0.f;
-                store_row64(sm + kPt, r, v);
+                for (int e = 0; e < 32; ++e) {
+                    const int s = s0 + e;
+                    const float E = fac ? ar * vb[s] : exp2f(ar - vb[s]);
+                    v[e] = (s <= r && r < lc) ? v[e] * E : 0.f;
+                }
+                store_row32(sm + kPt, r, 4 * wg, v);
             } else {
-                float* Af = (float*)(sm + kAf);
                 const float br = vbeta[r];
 #pragma unroll
-                for (int s = 0; s < 64; ++s)
-                    Af[r * kLd + s] = (s < r && r < lc) ? br * v[s] * exp2f(gr - vgam2[s]) : 0.f;
+                for (int e = 0; e < 32; ++e) {
+                    const int s = s0 + e;
+                    const float E = fac ? ar * vb[s] : exp2f(ar - vb[s]);
+                    v[e] = (s < r && r < lc) ? br * v[e] * E : 0.f;
+                }
+                float4* dst = reinterpret_cast<float4*>(sm + kAf + (r * kLd + s0) * 4);
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                    dst[c4] = make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
             }
         }
         tc_fence_before();
         __syncthreads();
 
-        // T = (I + A)^-1 in fp32: diagonal 16x16 blocks, then three merge levels
+        // ---- T = (I + A)^-1 in fp32: diagonal 16x16 blocks, then three merge levels
         {
             const float* Af = (const float*)(sm + kAf);
             float* Tf = (float*)(sm + kTf);
@@ -419,53 +448,66 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float x[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    float s = (r == cc) ? 1.f : 0.f;
+                    float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
-                    for (int j = 0; j < r; ++j) s -= Af[(16 * b + r) * kLd + 16 * b + j] * x[j];
-                    x[r] = (r < cc) ? 0.f : s;
+                    for (int j = 0; j + 1 < r; j += 2) {
+                        s0 -= Af[(16 * b + r) * kLd + 16 * b + j] * x[j];
+                        s1 -= Af[(16 * b + r) * kLd + 16 * b + j + 1] * x[j + 1];
+                    }
+                    if (r & 1) s0 -= Af[(16 * b + r) * kLd + 16 * b + r - 1] * x[r - 1];
+                    x[r] = (r < cc) ? 0.f : s0 + s1;
                 }
 #pragma unroll
                 for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * kLd + 16 * b + cc] = x[r];
             }
             __syncthreads();
-            for (int d = 1; d <= 3; ++d) {
-                solve_level_Y(Af, Tf, Ys, d, tid);
-                __syncthreads();
-                solve_level_T(Tf, Ys, d, tid);
-                __syncthreads();
-            }
-            // B operands of MMA_W / MMA_U: rows n, columns s <= n
-            const int nrow = tid >> 1, half = tid & 1;
-            float vw[32], vu[32];
+            solve_level_Y<1>(Af, Tf, Ys, tid);
+            __syncthreads();
+            solve_level_T<1>(Tf, Ys, tid);
+            __syncthreads();
+            solve_level_Y<2>(Af, Tf, Ys, tid);
+            __syncthreads();
+            solve_level_T<2>(Tf, Ys, tid);
+            __syncthreads();
+            solve_level_Y<3>(Af, Tf, Ys, tid);
+            __syncthreads();
+            solve_level_T<3>(Tf, Ys, tid);
+            __syncthreads();
+            // B operands of MMA_W / MMA_U: row n, columns s in [16 q, 16 q + 16), s <= n
+            const int nrow = tid >> 2, q = tid & 3;
+            float vw[16], vu[16];
+            const float4* trow = reinterpret_cast<const float4*>(Tf + nrow * kLd + 16 * q);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int s = 32 * half + e;
-                const float t = (s <= nrow) ? Tf[nrow * kLd + s] : 0.f;
-                vw[e] = t * vbG[s];
-                vu[e] = t * vbeta[s];
-            }
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 t4 = trow[c4];
+                const float tt[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
-            for (int cch = 0; cch < 4; ++cch) {
-                uint4 w, u;
-                w.x = pack_bf16(vw[8 * cch + 0], vw[8 * cch + 1]);
-                w.y = pack_bf16(vw[8 * cch + 2], vw[8 * cch + 3]);
-                w.z = pack_bf16(vw[8 * cch + 4], vw[8 * cch + 5]);
-                w.w = pack_bf16(vw[8 * cch + 6], vw[8 * cch + 7]);
-                u.x = pack_bf16(vu[8 * cch + 0], vu[8 * cch + 1]);
-                u.y = pack_bf16(vu[8 * cch + 2], vu[8 * cch + 3]);
-                u.z = pack_bf16(vu[8 * cch + 4], vu[8 * cch + 5]);
-                u.w = pack_bf16(vu[8 * cch + 6], vu[8 * cch + 7]);
-                const uint32_t off = sw128_off(nrow, 4 * half + cch);
-                *reinterpret_cast<uint4*>(sm + kBw + off) = w;
-                *reinterpret_cast<uint4*>(sm + kBu + off) = u;
+                for (int e = 0; e < 4; ++e) {
+                    const int s = 16 * q + 4 * c4 + e;
+                    const float t = (s <= nrow) ? tt[e] : 0.f;
+                    vw[4 * c4 + e] = t * vbG[s];
+                    vu[4 * c4 + e] = t * vbeta[s];
+                }
             }
+            *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q)) = pack8(vw);
+            *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
+            *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q)) = pack8(vu);
+            *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q + 1)) = pack8(vu + 8);
         }
         fence_proxy_async();
         __syncthreads();
 
-        // MMA_W: W^T = K^T Bw^T  and  MMA_U: Ut^T = V^T Bu^T
+        // ---- MMA_W: W^T = K^T Bw^T  and  MMA_U: Ut^T = V^T Bu^T
         if (tid == 0) {
             tc_fence_after();
+            if (emit) {  // MMA_HQ: H^T Q^T with the chunk-entry state (read by the epilogue)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                    mma_bf16_ss(tmem + kColHQ, desc_sw128(sbase + kHb + koff, 16, 1024),
+                                desc_sw128(sQK + koff, 16, 1024), id_n64, j > 0);
+                }
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
@@ -480,18 +522,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 
-        // W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
+        // ---- W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
         {
-            float v[64];
-            tmem_ld32(tmem + lane_off + kColR1, v);
-            tmem_ld32(tmem + lane_off + kColR1 + 32, v + 32);
-            store_row64(sm + kWt, tid, v);
+            float v[32];
+            tmem_ld32(tl + kColR1 + 32 * wg, v);
+            store_row32(sm + kWt, row, 4 * wg, v);
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // MMA_HW: U^T = Ut^T - H^T W^T
+        // ---- MMA_HW: U^T = Ut^T - H^T W^T
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -507,29 +548,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 
-        // U^T (lane = dv index) -> Ub and Ud = U^T diag(decay); H^T <- Gam_n H^T
+        // ---- U^T (lane = dv index) -> Ub and Ud = U^T diag(decay); H^T <- Gam_n H^T
         {
-            float v[64];
-            tmem_ld32(tmem + lane_off + kColR2, v);
-            tmem_ld32(tmem + lane_off + kColR2 + 32, v + 32);
-            if (emit) store_row64(sm + kUb, tid, v);
+            float v[32];
+            tmem_ld32(tl + kColR2 + 32 * wg, v);
+            if (emit) store_row32(sm + kUb, row, 4 * wg, v);
 #pragma unroll
-            for (int s = 0; s < 64; ++s) v[s] *= vdec[s];
-            store_row64(sm + kUd, tid, v);
+            for (int e = 0; e < 32; ++e) v[e] *= vdec[32 * wg + e];
+            store_row32(sm + kUd, row, 4 * wg, v);
             const float Gn = vGam[63];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                tmem_ld32(tmem + lane_off + kColH + 32 * q4, v);
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t col = kColH + 64 * wg + 32 * hf;
+                tmem_ld32(tl + col, v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] *= Gn;
-                tmem_st32(tmem + lane_off + kColH + 32 * q4, v);
+                tmem_st32(tl + col, v);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // MMA_UP: U^T P^T;  MMA_H: H^T += Ud K
+        // ---- MMA_UP: U^T P^T;  MMA_H: H^T += Ud K
         if (tid == 0) {
             tc_fence_after();
             if (emit) {
@@ -549,38 +590,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 
-        // output o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n]
+        // ---- output o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n], n in this half
         if (emit) {
-            const int m = tid;
-            __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+            const int m = row;
+            float hq[32], up[32];
+            tmem_ld32(tl + kColHQ + 32 * wg, hq);
+            tmem_ld32(tl + kColUP + 32 * wg, up);
+            __nv_bfloat16* op = (__nv_bfloat16*)p.o + ((t0 + 32 * wg) * Hv + h) * dv + m;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float hq[32], up[32];
-                tmem_ld32(tmem + lane_off + kColHQ + 32 * half, hq);
-                tmem_ld32(tmem + lane_off + kColUP + 32 * half, up);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int nn = 32 * half + e;
-                    if (nn < lc) op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(vGam[nn] * hq[e] + up[e]);
-                }
+            for (int e = 0; e < 32; ++e) {
+                const int nn = 32 * wg + e;
+                if (nn < lc) op[(int64_t)e * Hv * dv] = __float2bfloat16_rn(vGam[nn] * hq[e] + up[e]);
             }
         }
-        // bf16 copy of the new state for the next chunk's MMAs
+        // ---- bf16 copy of the new state (dk columns [64 wg, 64 wg + 64)) for the next chunk
         {
             float v[32];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                tmem_ld32(tmem + lane_off + kColH + 32 * q4, v);
-                uint8_t* atom = sm + kHb + (q4 >> 1) * 16384;
-#pragma unroll
-                for (int cch = 0; cch < 4; ++cch) {
-                    uint4 w;
-                    w.x = pack_bf16(v[8 * cch + 0], v[8 * cch + 1]);
-                    w.y = pack_bf16(v[8 * cch + 2], v[8 * cch + 3]);
-                    w.z = pack_bf16(v[8 * cch + 4], v[8 * cch + 5]);
-                    w.w = pack_bf16(v[8 * cch + 6], v[8 * cch + 7]);
-                    *reinterpret_cast<uint4*>(atom + sw128_off(tid, 4 * (q4 & 1) + cch)) = w;
-                }
+            for (int hf = 0; hf < 2; ++hf) {
+                tmem_ld32(tl + kColH + 64 * wg + 32 * hf, v);
+                store_row32(sm + kHb + wg * 16384, row, 4 * hf, v);
             }
         }
         fence_proxy_async();
@@ -591,14 +620,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
         if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
     } else if (p.ST && seg == segs_n - 1) {
-        // final state S_T = H (stored [dk][dv]): thread m writes column m
-        float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + tid;
+        // final state S_T = H (stored [dk][dv]): thread (m, wg) writes column m, dk half wg
+        float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + row;
         float v[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            tmem_ld32(tmem + lane_off + kColH + 32 * q4, v);
+        for (int hf = 0; hf < 2; ++hf) {
+            const int col0 = 64 * wg + 32 * hf;
+            tmem_ld32(tl + kColH + col0, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) st[(int64_t)(32 * q4 + e) * dv] = v[e];
+            for (int e = 0; e < 32; ++e) st[(int64_t)(col0 + e) * dv] = v[e];
         }
     }
     tc_fence_before();
