@@ -44,33 +44,47 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 256;  // 8 warps: warps w and w+4 share TMEM lane quarter w%4
+// Two groups of warps run a two-stage software pipeline over the chunks of a segment:
+//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T / K K^T,
+//                                       P and A, T = (I + A)^-1, W^T and Ut^T, W^T -> smem
+//   group S (threads 256-383, 4 warps)  the state chain of chunk k-1..k: U^T = Ut^T - H^T W^T,
+//                                       H^T <- Gam_n H^T + U^T Kd, outputs, bf16 copy of H
+// Each group has one tcgen05 issuer (threads 0 and 256) and its own commit
+// barrier; they hand chunks over through mbarriers (full / empty pairs).  Warp w
+// reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so group P's two warps per lane
+// quarter split the columns.
+constexpr int kThreads = 384;
+constexpr int kThreadsP = 256;
+constexpr int kThreadsS = 128;
 constexpr int kTmemCols = 512;
 // TMEM column map (lane = row of the M = 128 MMA)
-constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk   [0, 128)
-constexpr uint32_t kColR1 = 128;  // Q K^T / K K^T, then W^T               [128, 192)
-constexpr uint32_t kColR2 = 192;  // Ut^T, then U^T                        [192, 256)
-constexpr uint32_t kColHQ = 256;  // H^T Q^T                               [256, 320)
-constexpr uint32_t kColUP = 320;  // U^T P^T                               [320, 384)
+constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk     [0, 128)
+constexpr uint32_t kColR1 = 128;  // Q K^T / K K^T, then W^T (warpgroup P)   [128, 192)
+constexpr uint32_t kColR2 = 192;  // 2 x (Ut^T -> U^T), by chunk parity      [192, 320)
+constexpr uint32_t kColHQ = 320;  // H^T Q^T                                 [320, 384)
+constexpr uint32_t kColUP = 384;  // U^T P^T                                 [384, 448)
 
 // shared memory carve-up (bytes from a 1024-aligned base)
-constexpr uint32_t kStageQK = 0;          // 2 stages x 32 KB: [dk atom][q rows 0-63 | k rows 64-127][128 B]
-constexpr uint32_t kStageV = 65536;       // 2 stages x 16 KB: [dv atom][64 rows][128 B]
-constexpr uint32_t kHb = 98304;           // 32 KB  bf16 H^T: [dk atom][128 dv rows][128 B]
-constexpr uint32_t kPt = 131072;          // 8 KB   P: [64 n rows][64 s]
-constexpr uint32_t kBw = 139264;          // 8 KB   T diag(beta Gam): [n][s]
-constexpr uint32_t kBu = 147456;          // 8 KB   T diag(beta): [n][s]
-constexpr uint32_t kWt = 155648;          // 16 KB  W^T: [128 dk rows][64 tokens]
-constexpr uint32_t kUb = 172032;          // 16 KB  U^T: [128 dv rows][64 tokens]
-constexpr uint32_t kUd = 188416;          // 16 KB  U^T diag(decay)
-constexpr int kLd = 68;                   // row stride (floats) of the fp32 solve matrices
-constexpr uint32_t kAf = kWt;             // fp32 A [64][68] (aliases Wt/Ub/Ud during the solve)
-constexpr uint32_t kTf = kWt + 64 * kLd * 4;  // fp32 T [64][68]
-constexpr uint32_t kYs = kTf + 64 * kLd * 4;  // fp32 [3][16][17] solve scratch
-constexpr uint32_t kVec = 204800;         // 16 x 64 floats of per-token vectors
-constexpr uint32_t kBar = kVec + 16 * 256; // barriers and TMEM base
-constexpr uint32_t kSmemBytes = kBar + 64 + 1024;  // + alignment slack
-static_assert(kYs + 3 * 272 * 4 <= kVec, "solve scratch overlaps the vectors");
+constexpr uint32_t kStageQK = 0;       // 2 x 32 KB: [dk atom][q rows 0-63 | k rows 64-127][128 B]
+constexpr uint32_t kStageV = 65536;    // 2 x 16 KB: [dv atom][64 rows][128 B]
+constexpr uint32_t kHb = 98304;        // 32 KB  bf16 H^T: [dk atom][128 dv rows][128 B]
+constexpr uint32_t kPt = 131072;       // 2 x 8 KB  P: [64 n rows][64 s], by chunk parity
+constexpr uint32_t kBw = 147456;       // 8 KB   T diag(beta Gam): [n][s]
+constexpr uint32_t kBu = 155648;       // 8 KB   T diag(beta): [n][s]
+constexpr uint32_t kWt = 163840;       // 16 KB  W^T: [128 dk rows][64 tokens]
+constexpr uint32_t kUb = 180224;       // 16 KB  U^T: [128 dv rows][64 tokens]
+constexpr int kLd = 68;                // row stride (floats) of the fp32 solve matrix
+constexpr uint32_t kAs = kBw;         // fp32 [64][64] A, float4-XOR-swizzled (Bw/Bu are written
+                                       // only after the solve has read A for the last time)
+constexpr uint32_t kM = 196608;        // fp32 [64][68] T (lower triangle; diagonal blocks hold zeros above)
+constexpr int kLdY = 20;               // row stride (floats) of the level scratch
+constexpr uint32_t kYs = kM + 64 * kLd * 4;  // fp32 [3][16][20] solve scratch
+constexpr uint32_t kVec = 218112;      // 2 x 2 KB of per-token vectors, by chunk parity
+constexpr uint32_t kVecStride = 512;   // floats per parity
+constexpr uint32_t kRed = kVec + 2 * kVecStride * 4;  // 8 floats
+constexpr uint32_t kBar = kRed + 64;   // 8 mbarriers + TMEM base
+constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
+static_assert(kYs + 3 * 16 * kLdY * 4 <= kVec, "solve scratch overlaps the vectors");
 
 struct TcArgs {
     Problem p;
@@ -98,45 +112,98 @@ __device__ __forceinline__ void store_row32(uint8_t* tile, int row, int chunk0, 
         *reinterpret_cast<uint4*>(tile + sw128_off(row, chunk0 + c)) = pack8(v + 8 * c);
 }
 
-// Level-D merge of the blocked inverse (D = 1, 2, 3), for the blocks (i, i-D), i = D..3:
+// group-wide barrier (named barrier `id` over `cnt` threads), plain and with an AND / OR vote
+__device__ __forceinline__ void wg_sync(int id, int cnt) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(cnt) : "memory");
+}
+__device__ __forceinline__ bool wg_and(int id, int cnt, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(cnt)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool wg_or(int id, int cnt, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(cnt)
+        : "memory");
+    return r != 0;
+}
+
+// A (64 x 64, strictly lower) lives in As with float4 granules XOR-swizzled by row, so that a
+// warp writing 32 rows at one column, or reading 8 rows at one column, hits distinct banks.
+__device__ __forceinline__ int as_idx(int r, int s) { return r * 64 + ((((s >> 2) ^ (r & 15))) << 2) + (s & 3); }
+
+// Level-D merge of the blocked inverse (D = 1, 2, 3) over the blocks (i, i-D), i = D..3:
 //   Y = sum_{k=i-D}^{i-1} A_ik T_k,i-D   then   T_i,i-D = -T_ii Y.
-// The diagonal blocks of T store their upper triangles as zeros, so both sums
-// run over full 16-wide blocks with fixed trip counts.
+// T (in M, stride kLd) stores zeros above the diagonal of its diagonal blocks, so all sums
+// run over full blocks.  A task is one row of a block and 4 consecutive columns; the
+// j-range of Y is split over `kSplit` threads and combined with shuffles.
 template <int D>
-__device__ __forceinline__ void solve_level_Y(const float* Af, const float* Tf, float* Ys, int tid) {
-    constexpr int kOut = (4 - D) * 256;
+__device__ __forceinline__ void solve_level_Y(const float* As, const float* M, float* Ys, int t) {
+    constexpr int kTasks = (4 - D) * 64;  // (block, row, column quad)
+    constexpr int kSplit = kThreadsP / kTasks >= 4 ? 4 : kThreadsP / kTasks;  // 1, 2 or 4
+    constexpr int kLen = 16 * D / kSplit;
+    const int task = t / kSplit, part = t % kSplit;
+    if (task < kTasks) {
+        const int blk = task >> 6, rr = (task >> 2) & 15, quad = task & 3;
+        const int i = blk + D, j0 = i - D;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int q = 0; q < (kOut + kThreads - 1) / kThreads; ++q) {
-        const int o = tid + q * kThreads;
-        if (o < kOut) {
-            const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-            const int i = blk + D, j0 = i - D;
-            const float* arow = Af + (16 * i + rr) * kLd + 16 * j0;
-            const float* tcol = Tf + (16 * j0) * kLd + 16 * j0 + cc;
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int j = 0; j < 16 * D; ++j) s[j & 3] += arow[j] * tcol[j * kLd];
-            Ys[blk * 272 + rr * 17 + cc] = (s[0] + s[1]) + (s[2] + s[3]);
+        for (int jj = 0; jj < kLen; ++jj) {
+            const int j = part * kLen + jj;
+            const float a = As[as_idx(16 * i + rr, 16 * j0 + j)];
+            const float4 tv = *reinterpret_cast<const float4*>(M + (16 * j0 + j) * kLd + 16 * j0 + 4 * quad);
+            acc.x += a * tv.x;
+            acc.y += a * tv.y;
+            acc.z += a * tv.z;
+            acc.w += a * tv.w;
         }
+#pragma unroll
+        for (int o = 1; o < kSplit; o <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+        }
+        if (part == 0) *reinterpret_cast<float4*>(Ys + (blk * 16 + rr) * kLdY + 4 * quad) = acc;
     }
 }
 
 template <int D>
-__device__ __forceinline__ void solve_level_T(float* Tf, const float* Ys, int tid) {
-    constexpr int kOut = (4 - D) * 256;
+__device__ __forceinline__ void solve_level_T(float* M, const float* Ys, int t) {
+    constexpr int kTasks = (4 - D) * 64;
+    if (t < kTasks) {
+        const int blk = t >> 6, rr = (t >> 2) & 15, quad = t & 3;
+        const int i = blk + D, j0 = i - D;
+        const float* trow = M + (16 * i + rr) * kLd + 16 * i;  // T_ii row rr (zeros above)
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int q = 0; q < (kOut + kThreads - 1) / kThreads; ++q) {
-        const int o = tid + q * kThreads;
-        if (o < kOut) {
-            const int blk = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-            const int i = blk + D, j0 = i - D;
-            const float* trow = Tf + (16 * i + rr) * kLd + 16 * i;
-            const float* ycol = Ys + blk * 272 + cc;
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 tt = *reinterpret_cast<const float4*>(trow + 4 * j4);
+            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
 #pragma unroll
-            for (int j = 0; j < 16; ++j) s[j & 3] += trow[j] * ycol[j * 17];
-            Tf[(16 * i + rr) * kLd + 16 * j0 + cc] = -((s[0] + s[1]) + (s[2] + s[3]));
+            for (int e = 0; e < 4; ++e) {
+                const float4 y = *reinterpret_cast<const float4*>(Ys + (blk * 16 + 4 * j4 + e) * kLdY + 4 * quad);
+                acc.x += tv[e] * y.x;
+                acc.y += tv[e] * y.y;
+                acc.z += tv[e] * y.z;
+                acc.w += tv[e] * y.w;
+            }
         }
+        *reinterpret_cast<float4*>(M + (16 * i + rr) * kLd + 16 * j0 + 4 * quad) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
 }
 
@@ -146,21 +213,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Problem& p = args.p;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* vbeta = (float*)(sm + kVec);      // beta
-    float* vgam = vbeta + 64;                // gamma (natural log)
-    float* vGam = vgam + 64;                 // exp(gamma)
-    float* vbG = vGam + 64;                  // beta * Gam
-    float* vdec = vbG + 64;                  // exp(gamma_n - gamma)
-    float* va = vdec + 64;                   // row factor of E (or gamma * log2 e)
-    float* vb = va + 64;                     // column factor of E
-    float* vred = vb + 64;                   // reductions (8 warps)
-    uint64_t* bar_tma = (uint64_t*)(sm + kBar);  // [2]
-    uint64_t* bar_mma = bar_tma + 2;
-    uint32_t* tmem_slot = (uint32_t*)(bar_mma + 1);
+    float* vred = (float*)(sm + kRed);
+    uint64_t* bars = (uint64_t*)(sm + kBar);
+    uint64_t* bar_tma = bars;          // [2] stage full (TMA transaction bytes)
+    uint64_t* bar_mma_p = bars + 2;    // warpgroup P's MMA completions
+    uint64_t* bar_mma_s = bars + 3;    // warpgroup S's MMA completions
+    uint64_t* bar_wt_full = bars + 4;  // W^T of chunk k in smem, Ut^T of chunk k in TMEM
+    uint64_t* bar_wt_empty = bars + 5; // MMA_HW of chunk k has read W^T
+    uint64_t* bar_s_done = bars + 6;   // [2] warpgroup S finished chunk k (parity buffers free)
+    uint32_t* tmem_slot = (uint32_t*)(bars + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wg = warp >> 2;                    // which half of the columns this thread takes
-    const int row = ((warp & 3) << 5) | lane;    // TMEM lane (= MMA row) this thread reads
     const int Hv = p.Hv, dv = 128, dk = 128;
 
     // ---- which (sequence, head, segment) this CTA owns
@@ -267,12 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         cstart = (cum > args.log_eps || bad) ? 0 : w;
     }
     const bool exact = (cstart == 0);
+    const int nk = c1 - cstart;  // chunks this CTA walks (warm-up + own)
 
     // ---- set-up: barriers, TMEM
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -288,29 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lane quarter
     const uint32_t sbase = smem_u32(sm);
-    bool ok = true;
 
-    // ---- initial state: H^T (lane = dv index m) from S0 or zero; this thread
-    //      takes dk columns [64 wg, 64 wg + 64)
-    {
-        const int m = row;
-        const float* s0 = (exact && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
-        float v[32];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int col0 = 64 * wg + 32 * hf;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(int64_t)(col0 + e) * dv + m] : 0.f;
-            tmem_st32(tl + kColH + col0, v);
-            store_row32(sm + kHb + wg * 16384, m, 4 * hf, v);
-        }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    const int nk = c1 - cstart;  // chunks this CTA walks (warm-up + own)
     auto issue_tma = [&](int k) {
         const int c = cstart + k;
         const int stage = k & 1;
@@ -324,313 +364,404 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(vv + a * 8192, &tm_v, &bar_tma[stage], 64 * a, h, t0);
         }
     };
-    if (tid == 0 && nk > 0) issue_tma(0);
 
-    // gates of the next chunk, loaded one chunk ahead (threads 0..63)
-    float nxt_b = 0.f, nxt_g = 0.f;
-    auto load_gates = [&](int k) {
-        const int c = cstart + k;
-        const int64_t t0 = bos + (int64_t)c * kChunk;
-        const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-        nxt_b = tid < lc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
-        nxt_g = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;  // padding: g = 0
-    };
-    if (tid < 64 && nk > 0) load_gates(0);
+    // ---- initial state (warpgroup S): H^T (lane = dv index m) from S0 or zero
+    if (tid >= kThreadsP) {
+        const int m = tid - kThreadsP;
+        const float* s0 = (exact && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
+        float v[64];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e] = s0 ? s0[(int64_t)(64 * a + e) * dv + m] : 0.f;
+            tmem_st64(tl + kColH + 64 * a, v);
+            store_row32(sm + kHb + a * 16384, m, 0, v);
+            store_row32(sm + kHb + a * 16384, m, 4, v + 32);
+        }
+    } else if (tid == 0) {
+        if (nk > 0) issue_tma(0);
+        if (nk > 1) issue_tma(1);
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    uint32_t mma_phase = 0;
     const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
     const uint32_t id_mn_n64 = idesc_bf16(128, 64, 1, 0);        // A MN-major
     const uint32_t id_neg_bmn_n64 = idesc_bf16(128, 64, 0, 1, 1); // -A, B MN-major
     const uint32_t id_bmn_n128 = idesc_bf16(128, 128, 0, 1);      // B MN-major, N = 128
-    const float LOG2E = 1.4426950408889634f;
+    bool ok = true;
 
-    for (int k = 0; k < nk && ok; ++k) {
-        const int c = cstart + k;
-        const int stage = k & 1;
-        const bool emit = c >= c0;
-        const int64_t t0 = bos + (int64_t)c * kChunk;
-        const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-        const uint32_t sQK = sbase + kStageQK + stage * 32768;
-        const uint32_t sV = sbase + kStageV + stage * 16384;
+    if (tid < kThreadsP) {
+        // ======================= group P: chunk-local work ======================
+        const int t = tid;
+        const int hf = t >> 7;                       // which 32-column half of a TMEM row
+        const int row = ((warp & 3) << 5) | lane;    // TMEM lane (= MMA row) this thread reads
+        uint32_t ph = 0;  // parity of bar_mma_p
+        float nxt_b = 0.f, nxt_g = 0.f;
+        auto load_gates = [&](int k) {
+            const int c = cstart + k;
+            const int64_t t0 = bos + (int64_t)c * kChunk;
+            const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+            nxt_b = t < lc ? p.beta[(t0 + t) * Hv + h] : 0.f;
+            nxt_g = t < lc ? p.g[(t0 + t) * Hv + h] : 0.f;  // padding: g = 0
+        };
+        if (t < 64 && nk > 0) load_gates(0);
+        const float LOG2E = 1.4426950408889634f;
 
-        // ---- MMA1 once this chunk's tiles have landed (the gates below overlap it)
-        ok = __syncthreads_and(mbar_wait(&bar_tma[stage], (k >> 1) & 1));
-        if (!ok) break;
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + koff, 16, 1024),
-                            desc_sw128(sQK + 8192 + koff, 16, 1024), id_n64, j > 0);
+        for (int k = 0; k < nk; ++k) {
+            const int c = cstart + k;
+            const int stage = k & 1;
+            const bool emit = c >= c0;
+            const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+            const uint32_t sQK = sbase + kStageQK + stage * 32768;
+            const uint32_t sV = sbase + kStageV + stage * 16384;
+            float* vec = (float*)(sm + kVec) + stage * kVecStride;
+            float* vbeta = vec;
+            float* vgam = vec + 64;
+            float* vGam = vec + 128;
+            float* vbG = vec + 192;
+            float* vdec = vec + 256;
+            float* va = vec + 320;
+            float* vb = vec + 384;
+
+            // buffers of parity `stage` are free once warpgroup S finished chunk k-2
+            if (k >= 2) {
+                ok = wg_and(1, kThreadsP, mbar_wait(&bar_s_done[stage], ((k - 2) >> 1) & 1));
+                if (!ok) break;
             }
-            mma_commit(bar_mma);
-            if (k + 1 < nk) issue_tma(k + 1);  // stage k+1 was freed by chunk k-1's MMAs
-        }
-        // ---- gates: gamma = cumsum g (per-warp scan, then warp 1 adds warp 0's total)
-        if (tid < 64) {
-            float x = nxt_g;
-            const float b = nxt_b;
-            if (k + 1 < nk) load_gates(k + 1);
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            vbeta[tid] = b;
-            vgam[tid] = x;
-        }
-        __syncthreads();
-        // E_rs = exp(gamma_r - gamma_s) = a_r * b_s with a_r = exp(gamma_r - gamma_31),
-        // b_s = exp(gamma_31 - gamma_s), used when every |gamma - gamma_31| < 80 (both
-        // factors then stay far inside the fp32 range); else E is one exp2 per entry.
-        float gr = 0.f, gm = 0.f;
-        if (tid < 64) {
-            const int r = tid;
-            gr = vgam[r] + (r >= 32 ? vgam[31] : 0.f);
-            gm = vgam[31];
-            const float gl = vgam[63] + vgam[31];
-            vGam[r] = expf(gr);
-            vbG[r] = vbeta[r] * expf(gr);
-            vdec[r] = expf(gl - gr);
-        }
-        const bool fac = !__syncthreads_or(tid < 64 && !(fabsf(gr - gm) < 80.f));
-        if (tid < 64) {
-            va[tid] = fac ? expf(gr - gm) : gr * LOG2E;
-            vb[tid] = fac ? expf(gm - gr) : gr * LOG2E;
-        }
-        __syncthreads();
-
-        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
-        mma_phase ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-
-        // ---- P (rows 0..63) and A (rows 64..127); this thread: columns [32 wg, 32 wg + 32)
-        {
-            float v[32];
-            tmem_ld32(tl + kColR1 + 32 * wg, v);
-            const int r = row & 63;
-            const int s0 = 32 * wg;
-            const float ar = va[r];
-            if (row < 64) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int s = s0 + e;
-                    const float E = fac ? ar * vb[s] : exp2f(ar - vb[s]);
-                    v[e] = (s <= r && r < lc) ? v[e] * E : 0.f;
-                }
-                store_row32(sm + kPt, r, 4 * wg, v);
-            } else {
-                const float br = vbeta[r];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int s = s0 + e;
-                    const float E = fac ? ar * vb[s] : exp2f(ar - vb[s]);
-                    v[e] = (s < r && r < lc) ? br * v[e] * E : 0.f;
-                }
-                float4* dst = reinterpret_cast<float4*>(sm + kAf + (r * kLd + s0) * 4);
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                    dst[c4] = make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- T = (I + A)^-1 in fp32: diagonal 16x16 blocks, then three merge levels
-        {
-            const float* Af = (const float*)(sm + kAf);
-            float* Tf = (float*)(sm + kTf);
-            float* Ys = (float*)(sm + kYs);
-            if (tid < 64) {
-                const int b = tid >> 4, cc = tid & 15;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
-#pragma unroll
-                    for (int j = 0; j + 1 < r; j += 2) {
-                        s0 -= Af[(16 * b + r) * kLd + 16 * b + j] * x[j];
-                        s1 -= Af[(16 * b + r) * kLd + 16 * b + j + 1] * x[j + 1];
-                    }
-                    if (r & 1) s0 -= Af[(16 * b + r) * kLd + 16 * b + r - 1] * x[r - 1];
-                    x[r] = (r < cc) ? 0.f : s0 + s1;
-                }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * kLd + 16 * b + cc] = x[r];
-            }
-            __syncthreads();
-            solve_level_Y<1>(Af, Tf, Ys, tid);
-            __syncthreads();
-            solve_level_T<1>(Tf, Ys, tid);
-            __syncthreads();
-            solve_level_Y<2>(Af, Tf, Ys, tid);
-            __syncthreads();
-            solve_level_T<2>(Tf, Ys, tid);
-            __syncthreads();
-            solve_level_Y<3>(Af, Tf, Ys, tid);
-            __syncthreads();
-            solve_level_T<3>(Tf, Ys, tid);
-            __syncthreads();
-            // B operands of MMA_W / MMA_U: row n, columns s in [16 q, 16 q + 16), s <= n
-            const int nrow = tid >> 2, q = tid & 3;
-            float vw[16], vu[16];
-            const float4* trow = reinterpret_cast<const float4*>(Tf + nrow * kLd + 16 * q);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const float4 t4 = trow[c4];
-                const float tt[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int s = 16 * q + 4 * c4 + e;
-                    const float t = (s <= nrow) ? tt[e] : 0.f;
-                    vw[4 * c4 + e] = t * vbG[s];
-                    vu[4 * c4 + e] = t * vbeta[s];
-                }
-            }
-            *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q)) = pack8(vw);
-            *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
-            *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q)) = pack8(vu);
-            *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q + 1)) = pack8(vu + 8);
-        }
-        fence_proxy_async();
-        __syncthreads();
-
-        // ---- MMA_W: W^T = K^T Bw^T  and  MMA_U: Ut^T = V^T Bu^T
-        if (tid == 0) {
-            tc_fence_after();
-            if (emit) {  // MMA_HQ: H^T Q^T with the chunk-entry state (read by the epilogue)
+            ok = wg_and(1, kThreadsP, mbar_wait(&bar_tma[stage], (k >> 1) & 1));
+            if (!ok) break;
+            if (t == 0) {  // MMA1: [Q;K] K^T -> Q K^T (lanes 0-63), K K^T (lanes 64-127)
+                tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                    mma_bf16_ss(tmem + kColHQ, desc_sw128(sbase + kHb + koff, 16, 1024),
-                                desc_sw128(sQK + koff, 16, 1024), id_n64, j > 0);
+                    mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + koff, 16, 1024),
+                                desc_sw128(sQK + 8192 + koff, 16, 1024), id_n64, j > 0);
+                }
+                mma_commit(bar_mma_p);
+            }
+
+            // gates (threads 0..63): gamma = cumsum g; overlaps MMA1
+            float gr = 0.f, gm = 0.f;
+            if (t < 64) {
+                float x = nxt_g;
+                const float b = nxt_b;
+                if (k + 1 < nk) load_gates(k + 1);
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                vbeta[t] = b;
+                vgam[t] = x;
+            }
+            wg_sync(1, kThreadsP);
+            if (t < 64) {
+                gr = vgam[t] + (t >= 32 ? vgam[31] : 0.f);
+                gm = vgam[31];
+                const float gl = vgam[63] + vgam[31];
+                const float eg = expf(gr);
+                vGam[t] = eg;
+                vbG[t] = vbeta[t] * eg;
+                vdec[t] = expf(gl - gr);
+            }
+            // E_rs = exp(gamma_r - gamma_s) = a_r * b_s with a_r = exp(gamma_r - gamma_31),
+            // b_s = exp(gamma_31 - gamma_s) while every |gamma - gamma_31| < 80 (both factors
+            // far inside the fp32 range); otherwise one exp2 per entry.
+            const bool fac = !wg_or(1, kThreadsP, t < 64 && !(fabsf(gr - gm) < 80.f));
+            if (t < 64) {
+                va[t] = fac ? expf(gr - gm) : gr * LOG2E;
+                vb[t] = fac ? expf(gm - gr) : gr * LOG2E;
+            }
+            wg_sync(1, kThreadsP);
+
+            ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
+            ph ^= 1;
+            if (!ok) break;
+            tc_fence_after();
+
+            // P (rows 0..63, into Pt[stage]) and A (rows 64..127, into As);
+            // this thread: TMEM lane `row`, columns [32 hf, 32 hf + 32)
+            {
+                float v[32];
+                tmem_ld32(tl + kColR1 + 32 * hf, v);
+                const int r = row & 63;
+                const int s0 = 32 * hf;
+                const float ar = va[r];
+                float E[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
+                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) E[4 * c4 + e] = fac ? ar * bb[e] : exp2f(ar - bb[e]);
+                }
+                if (row < 64) {
+                    if (emit) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int s = s0 + e;
+                            v[e] = (s <= r && r < lc) ? v[e] * E[e] : 0.f;
+                        }
+                        store_row32(sm + kPt + stage * 8192, r, 4 * hf, v);
+                    }
+                } else {
+                    const float br = vbeta[r];
+                    float* As = (float*)(sm + kAs);
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        float4 w;
+                        const int sb = s0 + 4 * c4;
+                        w.x = (sb + 0 < r && r < lc) ? br * v[4 * c4 + 0] * E[4 * c4 + 0] : 0.f;
+                        w.y = (sb + 1 < r && r < lc) ? br * v[4 * c4 + 1] * E[4 * c4 + 1] : 0.f;
+                        w.z = (sb + 2 < r && r < lc) ? br * v[4 * c4 + 2] * E[4 * c4 + 2] : 0.f;
+                        w.w = (sb + 3 < r && r < lc) ? br * v[4 * c4 + 3] * E[4 * c4 + 3] : 0.f;
+                        *reinterpret_cast<float4*>(As + as_idx(r, sb)) = w;
+                    }
                 }
             }
+            tc_fence_before();
+            wg_sync(1, kThreadsP);
+
+            // T = (I + A)^-1 in fp32: diagonal 16x16 blocks by substitution, then 3 merge levels
+            {
+                const float* As = (const float*)(sm + kAs);
+                float* M = (float*)(sm + kM);
+                float* Ys = (float*)(sm + kYs);
+                if (t < 64) {  // column cc of diagonal block b
+                    const int b = t >> 4, cc = t & 15;
+                    float x[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
-                            desc_sw128(sbase + kBw + j * 32, 16, 1024), id_mn_n64, j > 0);
-                mma_bf16_ss(tmem + kColR2, desc_sw128(sV + j * 2048, 8192, 1024),
-                            desc_sw128(sbase + kBu + j * 32, 16, 1024), id_mn_n64, j > 0);
+                    for (int r = 0; r < 16; ++r) {
+                        float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+                        for (int j = 0; j + 1 < r; j += 2) {
+                            s0 -= As[as_idx(16 * b + r, 16 * b + j)] * x[j];
+                            s1 -= As[as_idx(16 * b + r, 16 * b + j + 1)] * x[j + 1];
+                        }
+                        if (r & 1) s0 -= As[as_idx(16 * b + r, 16 * b + r - 1)] * x[r - 1];
+                        x[r] = (r < cc) ? 0.f : s0 + s1;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) M[(16 * b + r) * kLd + 16 * b + cc] = x[r];
+                }
+                wg_sync(1, kThreadsP);
+                solve_level_Y<1>(As, M, Ys, t);
+                wg_sync(1, kThreadsP);
+                solve_level_T<1>(M, Ys, t);
+                wg_sync(1, kThreadsP);
+                solve_level_Y<2>(As, M, Ys, t);
+                wg_sync(1, kThreadsP);
+                solve_level_T<2>(M, Ys, t);
+                wg_sync(1, kThreadsP);
+                solve_level_Y<3>(As, M, Ys, t);
+                wg_sync(1, kThreadsP);
+                solve_level_T<3>(M, Ys, t);
+                wg_sync(1, kThreadsP);
+                // B operands of MMA_W / MMA_U: row n = t/4, columns s in [16 q, 16 q + 16), s <= n
+                // (written over As, which is no longer read)
+                const int nrow = t >> 2, q = t & 3;
+                float vw[16], vu[16];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int sb = 16 * q + 4 * c4;
+                    const float4 tt = *reinterpret_cast<const float4*>(M + nrow * kLd + sb);
+                    const float4 g4 = *reinterpret_cast<const float4*>(vbG + sb);
+                    const float4 b4 = *reinterpret_cast<const float4*>(vbeta + sb);
+                    const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
+                    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float tv_e = (sb + e <= nrow) ? tv[e] : 0.f;
+                        vw[4 * c4 + e] = tv_e * gv[e];
+                        vu[4 * c4 + e] = tv_e * bv[e];
+                    }
+                }
+                wg_sync(1, kThreadsP);  // As overlaps Bw / Bu
+                *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q)) = pack8(vw);
+                *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
+                *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q)) = pack8(vu);
+                *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q + 1)) = pack8(vu + 8);
             }
-            mma_commit(bar_mma);
-        }
-        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
-        mma_phase ^= 1;
-        if (!ok) break;
-        tc_fence_after();
+            fence_proxy_async();
+            wg_sync(1, kThreadsP);
 
-        // ---- W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
-        {
-            float v[32];
-            tmem_ld32(tl + kColR1 + 32 * wg, v);
-            store_row32(sm + kWt, row, 4 * wg, v);
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- MMA_HW: U^T = Ut^T - H^T W^T
-        if (tid == 0) {
+            if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1);  MMA_U: Ut^T = V^T Bu^T (R2[stage])
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
+                                desc_sw128(sbase + kBw + j * 32, 16, 1024), id_mn_n64, j > 0);
+                    mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
+                                desc_sw128(sbase + kBu + j * 32, 16, 1024), id_mn_n64, j > 0);
+                }
+                mma_commit(bar_mma_p);
+            }
+            ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
+            ph ^= 1;
+            if (!ok) break;
+            // Wt is free once MMA_HW of chunk k-1 has read it
+            if (k >= 1) {
+                ok = wg_and(1, kThreadsP, mbar_wait(bar_wt_empty, (k - 1) & 1));
+                if (!ok) break;
+            }
             tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                mma_bf16_ss(tmem + kColR2, desc_sw128(sbase + kHb + koff, 16, 1024),
-                            desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_neg_bmn_n64, 1);
+            {  // W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
+                float v[32];
+                tmem_ld32(tl + kColR1 + 32 * hf, v);
+                store_row32(sm + kWt, row, 4 * hf, v);
             }
-            mma_commit(bar_mma);
+            fence_proxy_async();
+            tc_fence_before();
+            wg_sync(1, kThreadsP);
+            if (t == 0) mbar_arrive(bar_wt_full);
         }
-        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
-        mma_phase ^= 1;
-        if (!ok) break;
-        tc_fence_after();
+    } else {
+        // ======================= group S: the state chain =======================
+        const int m = tid - kThreadsP;
+        uint32_t ph = 0;  // parity of bar_mma_s
+        for (int k = 0; k < nk; ++k) {
+            const int c = cstart + k;
+            const int stage = k & 1;
+            const bool emit = c >= c0;
+            const int64_t t0 = bos + (int64_t)c * kChunk;
+            const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+            const uint32_t sQK = sbase + kStageQK + stage * 32768;
+            const float* vec = (const float*)(sm + kVec) + stage * kVecStride;
+            const float* vGam = vec + 128;
+            const float* vdec = vec + 256;
 
-        // ---- U^T (lane = dv index) -> Ub and Ud = U^T diag(decay); H^T <- Gam_n H^T
-        {
-            float v[32];
-            tmem_ld32(tl + kColR2 + 32 * wg, v);
-            if (emit) store_row32(sm + kUb, row, 4 * wg, v);
+            ok = wg_and(2, kThreadsS, mbar_wait(bar_wt_full, k & 1));
+            if (!ok) break;
+            if (m == 0) {  // MMA_HQ: H^T Q^T;  MMA_HW: U^T = Ut^T - H^T W^T
+                tc_fence_after();
+                if (emit) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= vdec[32 * wg + e];
-            store_row32(sm + kUd, row, 4 * wg, v);
-            const float Gn = vGam[63];
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                        mma_bf16_ss(tmem + kColHQ, desc_sw128(sbase + kHb + koff, 16, 1024),
+                                    desc_sw128(sQK + koff, 16, 1024), id_n64, j > 0);
+                    }
+                }
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const uint32_t col = kColH + 64 * wg + 32 * hf;
-                tmem_ld32(tl + col, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] *= Gn;
-                tmem_st32(tl + col, v);
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                    mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sbase + kHb + koff, 16, 1024),
+                                desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_neg_bmn_n64, 1);
+                }
+                mma_commit(bar_mma_s);
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- MMA_UP: U^T P^T;  MMA_H: H^T += Ud K
-        if (tid == 0) {
+            ok = wg_and(2, kThreadsS, mbar_wait(bar_mma_s, ph));
+            ph ^= 1;
+            if (!ok) break;
             tc_fence_after();
-            if (emit) {
+            if (m == 0) mbar_arrive(bar_wt_empty);
+
+            {  // U^T (lane = dv index) -> Ub;  H^T <- Gam_n H^T;  K rows <- decay * K rows
+                float v[64];
+                tmem_ld64(tl + kColR2 + 64 * stage, v);
+                store_row32(sm + kUb, m, 0, v);
+                store_row32(sm + kUb, m, 4, v + 32);
+                const float Gn = vGam[63];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    tmem_ld64(tl + kColH + 64 * a, v);
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] *= Gn;
+                    tmem_st64(tl + kColH + 64 * a, v);
+                }
+                // K row s (tile rows 64..127), dk half `a`: 8 chunks of 8 bf16, scaled by decay_s
+                const int s = m >> 1, a = m & 1;
+                uint8_t* krow = sm + kStageQK + stage * 32768 + a * 16384 + (64 + s) * 128;
+                const float d = vdec[s];
+#pragma unroll
+                for (int i8 = 0; i8 < 8; ++i8) {
+                    const int c8 = (i8 + s) & 7;  // rotate so that the rows of a warp hit distinct banks
+                    uint4 u = *reinterpret_cast<uint4*>(krow + 16 * c8);
+                    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float2 f = __bfloat1622float2(b2[e]);
+                        b2[e] = __floats2bfloat162_rn(f.x * d, f.y * d);
+                    }
+                    *reinterpret_cast<uint4*>(krow + 16 * c8) = u;
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            wg_sync(2, kThreadsS);
+            if (m == 0) {  // MMA_UP: U^T P^T;  MMA_H: H^T += U^T Kd
+                tc_fence_after();
+                if (emit) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mma_bf16_ss(tmem + kColUP, desc_sw128(sbase + kUb + j * 32, 16, 1024),
+                                    desc_sw128(sbase + kPt + stage * 8192 + j * 32, 16, 1024), id_n64,
+                                    j > 0);
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    mma_bf16_ss(tmem + kColUP, desc_sw128(sbase + kUb + j * 32, 16, 1024),
-                                desc_sw128(sbase + kPt + j * 32, 16, 1024), id_n64, j > 0);
+                    mma_bf16_ss(tmem + kColH, desc_sw128(sbase + kUb + j * 32, 16, 1024),
+                                desc_sw128(sQK + 8192 + j * 2048, 16384, 1024), id_bmn_n128, 1);
+                mma_commit(bar_mma_s);
             }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_bf16_ss(tmem + kColH, desc_sw128(sbase + kUd + j * 32, 16, 1024),
-                            desc_sw128(sQK + 8192 + j * 2048, 16384, 1024), id_bmn_n128, 1);
-            mma_commit(bar_mma);
-        }
-        ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase));
-        mma_phase ^= 1;
-        if (!ok) break;
-        tc_fence_after();
+            ok = wg_and(2, kThreadsS, mbar_wait(bar_mma_s, ph));
+            ph ^= 1;
+            if (!ok) break;
+            tc_fence_after();
+            if (m == 0 && k + 2 < nk) issue_tma(k + 2);  // stage `stage` is no longer read
 
-        // ---- output o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n], n in this half
-        if (emit) {
-            const int m = row;
-            float hq[32], up[32];
-            tmem_ld32(tl + kColHQ + 32 * wg, hq);
-            tmem_ld32(tl + kColUP + 32 * wg, up);
-            __nv_bfloat16* op = (__nv_bfloat16*)p.o + ((t0 + 32 * wg) * Hv + h) * dv + m;
+            {  // bf16 copy of the new state for the next chunk's MMAs
+                float v[64];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int nn = 32 * wg + e;
-                if (nn < lc) op[(int64_t)e * Hv * dv] = __float2bfloat16_rn(vGam[nn] * hq[e] + up[e]);
+                for (int a = 0; a < 2; ++a) {
+                    tmem_ld64(tl + kColH + 64 * a, v);
+                    store_row32(sm + kHb + a * 16384, m, 0, v);
+                    store_row32(sm + kHb + a * 16384, m, 4, v + 32);
+                }
+            }
+            if (emit) {  // o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n]
+                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float hq[32], up[32];
+                    tmem_ld32x2(tl + kColHQ + 32 * hf, hq, tl + kColUP + 32 * hf, up);
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(vGam + 32 * hf + 4 * e4);
+                        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                        for (int e1 = 0; e1 < 4; ++e1) {
+                            const int e = 4 * e4 + e1, nn = 32 * hf + e;
+                            if (nn < lc)
+                                op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(gv[e1] * hq[e] + up[e]);
+                        }
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            wg_sync(2, kThreadsS);
+            if (m == 0) mbar_arrive(&bar_s_done[stage]);
+        }
+        if (ok && p.ST && seg == segs_n - 1) {
+            // final state S_T = H (stored [dk][dv]): thread m writes column m
+            float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + m;
+            float v[64];
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                tmem_ld64(tl + kColH + 64 * a, v);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) st[(int64_t)(64 * a + e) * dv] = v[e];
             }
         }
-        // ---- bf16 copy of the new state (dk columns [64 wg, 64 wg + 64)) for the next chunk
-        {
-            float v[32];
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                tmem_ld32(tl + kColH + 64 * wg + 32 * hf, v);
-                store_row32(sm + kHb + wg * 16384, row, 4 * hf, v);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
     }
 
-    if (!ok) {
-        if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
-    } else if (p.ST && seg == segs_n - 1) {
-        // final state S_T = H (stored [dk][dv]): thread (m, wg) writes column m, dk half wg
-        float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + row;
-        float v[32];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int col0 = 64 * wg + 32 * hf;
-            tmem_ld32(tl + kColH + col0, v);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) st[(int64_t)(col0 + e) * dv] = v[e];
-        }
-    }
+    if (!ok && (tid == 0 || tid == kThreadsP)) report(p.status, GDN_ERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
