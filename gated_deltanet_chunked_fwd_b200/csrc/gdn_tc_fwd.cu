@@ -63,6 +63,8 @@ constexpr uint32_t kColR1 = 128;  // Q K^T / K K^T, then W^T (warpgroup P)   [12
 constexpr uint32_t kColR2 = 192;  // 2 x (Ut^T -> U^T), by chunk parity      [192, 320)
 constexpr uint32_t kColHQ = 320;  // H^T Q^T                                 [320, 384)
 constexpr uint32_t kColUP = 384;  // U^T P^T                                 [384, 448)
+constexpr uint32_t kColHb = 448;  // bf16 H^T, A operand (K pairs per column) [448, 512)
+// U^T in bf16 (A operand of MMA_UP / MMA_H) overwrites the first 32 columns of its R2 buffer.
 
 // shared memory carve-up (bytes from a 1024-aligned base)
 constexpr uint32_t kStageQK = 0;       // 2 x 32 KB: [dk atom][q rows 0-63 | k rows 64-127][128 B]
@@ -79,10 +81,10 @@ constexpr uint32_t kAs = kBw;         // fp32 [64][64] A, float4-XOR-swizzled (B
 constexpr uint32_t kM = 196608;        // fp32 [64][68] T (lower triangle; diagonal blocks hold zeros above)
 constexpr int kLdY = 20;               // row stride (floats) of the level scratch
 constexpr uint32_t kYs = kM + 64 * kLd * 4;  // fp32 [3][16][20] solve scratch
-constexpr uint32_t kVec = 218112;      // 2 x 2 KB of per-token vectors, by chunk parity
-constexpr uint32_t kVecStride = 512;   // floats per parity
-constexpr uint32_t kRed = kVec + 2 * kVecStride * 4;  // 8 floats
-constexpr uint32_t kBar = kRed + 64;   // 8 mbarriers + TMEM base
+constexpr uint32_t kVec = 218112;      // 3 x 2 KB of per-token vectors, by chunk index mod 3
+constexpr uint32_t kVecStride = 512;   // floats per buffer
+constexpr uint32_t kRed = kVec + 3 * kVecStride * 4;  // 16 floats
+constexpr uint32_t kBar = kRed + 64;   // 9 mbarriers + TMEM base
 constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
 static_assert(kYs + 3 * 16 * kLdY * 4 <= kVec, "solve scratch overlaps the vectors");
 
@@ -220,8 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bar_mma_s = bars + 3;    // warpgroup S's MMA completions
     uint64_t* bar_wt_full = bars + 4;  // W^T of chunk k in smem, Ut^T of chunk k in TMEM
     uint64_t* bar_wt_empty = bars + 5; // MMA_HW of chunk k has read W^T
-    uint64_t* bar_s_done = bars + 6;   // [2] warpgroup S finished chunk k (parity buffers free)
-    uint32_t* tmem_slot = (uint32_t*)(bars + 8);
+    uint64_t* bar_s_done = bars + 6;   // [2] group S finished chunk k (parity buffers free)
+    uint64_t* bar_gates = bars + 8;    // group P wrote the per-token vectors of chunk k
+    uint32_t* tmem_slot = (uint32_t*)(bars + 9);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hv = p.Hv, dv = 128, dk = 128;
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- set-up: barriers, TMEM
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -370,13 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int m = tid - kThreadsP;
         const float* s0 = (exact && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
         float v[64];
+        uint32_t w[32];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
 #pragma unroll
             for (int e = 0; e < 64; ++e) v[e] = s0 ? s0[(int64_t)(64 * a + e) * dv + m] : 0.f;
             tmem_st64(tl + kColH + 64 * a, v);
-            store_row32(sm + kHb + a * 16384, m, 0, v);
-            store_row32(sm + kHb + a * 16384, m, 4, v + 32);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+            tmem_st32u(tl + kColHb + 32 * a, w);
         }
     } else if (tid == 0) {
         if (nk > 0) issue_tma(0);
@@ -389,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
     const uint32_t id_mn_n64 = idesc_bf16(128, 64, 1, 0);        // A MN-major
-    const uint32_t id_neg_bmn_n64 = idesc_bf16(128, 64, 0, 1, 1); // -A, B MN-major
+    const uint32_t id_bmn_n64 = idesc_bf16(128, 64, 0, 1);        // B MN-major
     const uint32_t id_bmn_n128 = idesc_bf16(128, 128, 0, 1);      // B MN-major, N = 128
     bool ok = true;
 
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t sV = sbase + kStageV + stage * 16384;
-            float* vec = (float*)(sm + kVec) + stage * kVecStride;
+            float* vec = (float*)(sm + kVec) + (k % 3) * kVecStride;
             float* vbeta = vec;
             float* vgam = vec + 64;
             float* vGam = vec + 128;
@@ -477,6 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 vb[t] = fac ? expf(gm - gr) : gr * LOG2E;
             }
             wg_sync(1, kThreadsP);
+            if (t == 0) mbar_arrive(bar_gates);
 
             ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
             ph ^= 1;
@@ -613,74 +619,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             {  // W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
                 float v[32];
                 tmem_ld32(tl + kColR1 + 32 * hf, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = -v[e];  // MMA_HW accumulates -H^T W^T
                 store_row32(sm + kWt, row, 4 * hf, v);
             }
-            fence_proxy_async();
-            tc_fence_before();
-            wg_sync(1, kThreadsP);
-            if (t == 0) mbar_arrive(bar_wt_full);
-        }
-    } else {
-        // ======================= group S: the state chain =======================
-        const int m = tid - kThreadsP;
-        uint32_t ph = 0;  // parity of bar_mma_s
-        for (int k = 0; k < nk; ++k) {
-            const int c = cstart + k;
-            const int stage = k & 1;
-            const bool emit = c >= c0;
-            const int64_t t0 = bos + (int64_t)c * kChunk;
-            const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-            const uint32_t sQK = sbase + kStageQK + stage * 32768;
-            const float* vec = (const float*)(sm + kVec) + stage * kVecStride;
-            const float* vGam = vec + 128;
-            const float* vdec = vec + 256;
-
-            ok = wg_and(2, kThreadsS, mbar_wait(bar_wt_full, k & 1));
-            if (!ok) break;
-            if (m == 0) {  // MMA_HQ: H^T Q^T;  MMA_HW: U^T = Ut^T - H^T W^T
-                tc_fence_after();
-                if (emit) {
+            {  // K rows <- exp(gamma_n - gamma_s) * K rows (B operand of MMA_H; MMA1 / MMA_W are done)
+                const int srow = t >> 2, q = t & 3;
+                uint8_t* krow = sm + kStageQK + stage * 32768 + (q >> 1) * 16384 + (64 + srow) * 128;
+                const float d = vdec[srow];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                        mma_bf16_ss(tmem + kColHQ, desc_sw128(sbase + kHb + koff, 16, 1024),
-                                    desc_sw128(sQK + koff, 16, 1024), id_n64, j > 0);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                    mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sbase + kHb + koff, 16, 1024),
-                                desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_neg_bmn_n64, 1);
-                }
-                mma_commit(bar_mma_s);
-            }
-            ok = wg_and(2, kThreadsS, mbar_wait(bar_mma_s, ph));
-            ph ^= 1;
-            if (!ok) break;
-            tc_fence_after();
-            if (m == 0) mbar_arrive(bar_wt_empty);
-
-            {  // U^T (lane = dv index) -> Ub;  H^T <- Gam_n H^T;  K rows <- decay * K rows
-                float v[64];
-                tmem_ld64(tl + kColR2 + 64 * stage, v);
-                store_row32(sm + kUb, m, 0, v);
-                store_row32(sm + kUb, m, 4, v + 32);
-                const float Gn = vGam[63];
-#pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    tmem_ld64(tl + kColH + 64 * a, v);
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) v[e] *= Gn;
-                    tmem_st64(tl + kColH + 64 * a, v);
-                }
-                // K row s (tile rows 64..127), dk half `a`: 8 chunks of 8 bf16, scaled by decay_s
-                const int s = m >> 1, a = m & 1;
-                uint8_t* krow = sm + kStageQK + stage * 32768 + a * 16384 + (64 + s) * 128;
-                const float d = vdec[s];
-#pragma unroll
-                for (int i8 = 0; i8 < 8; ++i8) {
-                    const int c8 = (i8 + s) & 7;  // rotate so that the rows of a warp hit distinct banks
+                for (int i4 = 0; i4 < 4; ++i4) {
+                    const int c8 = 4 * (q & 1) + ((i4 + srow) & 3);  // rotated: rows spread over banks
                     uint4 u = *reinterpret_cast<uint4*>(krow + 16 * c8);
                     __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
@@ -693,19 +642,106 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async();
             tc_fence_before();
+            wg_sync(1, kThreadsP);
+            if (t == 0) mbar_arrive(bar_wt_full);
+        }
+    } else {
+        // ======================= group S: the state chain =======================
+        // Per chunk k: MMA_HW, then (overlapping it) the outputs of chunk k-1; U^T -> bf16 in
+        // TMEM; MMA_HQ / MMA_UP / MMA_H (A operands from TMEM); then one pass over H that
+        // writes its bf16 copy and pre-scales it by the next chunk's Gam_n (MMA_H of chunk
+        // k+1 accumulates onto it).
+        const int m = tid - kThreadsP;
+        uint32_t ph = 0;  // parity of bar_mma_s
+        auto epilogue = [&](int kk) {  // o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n]
+            const int cc = cstart + kk;
+            const int64_t t0 = bos + (int64_t)cc * kChunk;
+            const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
+            const float* vGam = (const float*)(sm + kVec) + (kk % 3) * kVecStride + 128;
+            __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float hq[32], up[32];
+                tmem_ld32x2(tl + kColHQ + 32 * hf, hq, tl + kColUP + 32 * hf, up);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(vGam + 32 * hf + 4 * e4);
+                    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                    for (int e1 = 0; e1 < 4; ++e1) {
+                        const int e = 4 * e4 + e1, nn = 32 * hf + e;
+                        if (nn < lc)
+                            op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(gv[e1] * hq[e] + up[e]);
+                    }
+                }
+            }
+        };
+        for (int k = 0; k < nk && ok; ++k) {
+            const int c = cstart + k;
+            const int stage = k & 1;
+            const bool emit = c >= c0;
+            const bool emit_prev = k > 0 && (c - 1) >= c0;
+            const uint32_t sQK = sbase + kStageQK + stage * 32768;
+            const uint32_t colR2 = kColR2 + 64 * stage;
+
+            ok = wg_and(2, kThreadsS, mbar_wait(bar_wt_full, k & 1));
+            if (!ok) break;
+            if (k == 0) {
+                // scale the initial state by Gam_n of the first chunk (its vectors were written
+                // before the hand-off); MMA_H of chunk 0 accumulates onto it
+                const float Gn = ((const float*)(sm + kVec))[128 + 63];
+                float v[64];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    tmem_ld64(tl + kColH + 64 * a, v);
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] *= Gn;
+                    tmem_st64(tl + kColH + 64 * a, v);
+                }
+            }
+            if (m == 0) {  // MMA_HW: U^T = Ut^T + H^T (-W^T)
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    mma_bf16_ts(tmem + colR2, tmem + kColHb + 8 * j,
+                                desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_bmn_n64, 1);
+                mma_commit(bar_mma_s);
+            }
+            if (emit_prev) epilogue(k - 1);  // overlaps MMA_HW of this chunk
+            ok = wg_and(2, kThreadsS, mbar_wait(bar_mma_s, ph));
+            ph ^= 1;
+            if (!ok) break;
+            tc_fence_after();
+            if (m == 0) mbar_arrive(bar_wt_empty);
+
+            {  // U^T (lane = dv index, fp32) -> bf16 pairs in the first 32 columns of the same buffer
+                float v[64];
+                uint32_t w[32];
+                tmem_ld64(tl + colR2, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+                tmem_st32u(tl + colR2, w);
+            }
+            tc_fence_before();
             wg_sync(2, kThreadsS);
-            if (m == 0) {  // MMA_UP: U^T P^T;  MMA_H: H^T += U^T Kd
+            if (m == 0) {  // MMA_HQ: H^T Q^T;  MMA_UP: U^T P^T;  MMA_H: H^T += U^T Kd
                 tc_fence_after();
                 if (emit) {
 #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                        mma_bf16_ts(tmem + kColHQ, tmem + kColHb + 8 * j, desc_sw128(sQK + koff, 16, 1024),
+                                    id_n64, j > 0);
+                    }
+#pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        mma_bf16_ss(tmem + kColUP, desc_sw128(sbase + kUb + j * 32, 16, 1024),
+                        mma_bf16_ts(tmem + kColUP, tmem + colR2 + 8 * j,
                                     desc_sw128(sbase + kPt + stage * 8192 + j * 32, 16, 1024), id_n64,
                                     j > 0);
                 }
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    mma_bf16_ss(tmem + kColH, desc_sw128(sbase + kUb + j * 32, 16, 1024),
+                    mma_bf16_ts(tmem + kColH, tmem + colR2 + 8 * j,
                                 desc_sw128(sQK + 8192 + j * 2048, 16384, 1024), id_bmn_n128, 1);
                 mma_commit(bar_mma_s);
             }
@@ -715,39 +751,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             if (m == 0 && k + 2 < nk) issue_tma(k + 2);  // stage `stage` is no longer read
 
-            {  // bf16 copy of the new state for the next chunk's MMAs
+            // bf16 copy of the new state (A operand of the next chunk's MMAs); pre-scale by its Gam_n
+            const bool more = k + 1 < nk;
+            if (more) {
+                ok = wg_and(2, kThreadsS, mbar_wait(bar_gates, (k + 1) & 1));
+                if (!ok) break;
+            }
+            {
+                const float Gn = more ? ((const float*)(sm + kVec))[((k + 1) % 3) * kVecStride + 128 + 63] : 1.f;
                 float v[64];
+                uint32_t w[32];
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     tmem_ld64(tl + kColH + 64 * a, v);
-                    store_row32(sm + kHb + a * 16384, m, 0, v);
-                    store_row32(sm + kHb + a * 16384, m, 4, v + 32);
-                }
-            }
-            if (emit) {  // o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n]
-                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float hq[32], up[32];
-                    tmem_ld32x2(tl + kColHQ + 32 * hf, hq, tl + kColUP + 32 * hf, up);
+                    for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+                    tmem_st32u(tl + kColHb + 32 * a, w);
+                    if (more) {
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 g4 = *reinterpret_cast<const float4*>(vGam + 32 * hf + 4 * e4);
-                        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-                        for (int e1 = 0; e1 < 4; ++e1) {
-                            const int e = 4 * e4 + e1, nn = 32 * hf + e;
-                            if (nn < lc)
-                                op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(gv[e1] * hq[e] + up[e]);
-                        }
+                        for (int e = 0; e < 64; ++e) v[e] *= Gn;
+                        tmem_st64(tl + kColH + 64 * a, v);
                     }
                 }
             }
-            fence_proxy_async();
             tc_fence_before();
             wg_sync(2, kThreadsS);
             if (m == 0) mbar_arrive(&bar_s_done[stage]);
         }
+        if (ok && nk > 0 && cstart + nk - 1 >= c0) epilogue(nk - 1);
         if (ok && p.ST && seg == segs_n - 1) {
             // final state S_T = H (stored [dk][dv]): thread m writes column m
             float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + m;
