@@ -27,6 +27,7 @@ STATUS = {
     4: "GDN_ERR_CUDA",
     5: "GDN_ERR_TIMEOUT",
     6: "GDN_ERR_DEVICE",
+    7: "GDN_ERR_TOO_LARGE",
 }
 
 _u32, _i32, _p = ctypes.c_uint32, ctypes.c_int32, ctypes.c_void_p
@@ -54,7 +55,7 @@ class GdnBwdArgs(ctypes.Structure):
 EXPORTS = [
     "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_launch_count",
     "gdn_chunk_bwd_workspace_size", "gdn_chunk_bwd", "gdn_chunk_bwd_launch_count",
-    "gdn_status_string",
+    "gdn_status_string", "gdn_chunk_fwd_noalloc",
 ]
 
 _lib = None
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
         for fn in ("gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
                    "gdn_chunk_bwd", "gdn_chunk_fwd_launch_count", "gdn_chunk_bwd_launch_count"):
             getattr(L, fn).restype = ctypes.c_int
+        L.gdn_chunk_fwd_noalloc.argtypes = [F, _p]
+        L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         _lib = L

@@ -250,6 +250,7 @@ const char* gdn_status_string(int status) {
         case GDN_ERR_CUDA: return "CUDA launch or runtime error";
         case GDN_ERR_TIMEOUT: return "device wait timed out";
         case GDN_ERR_DEVICE: return "device-side consistency check failed";
+        case GDN_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of gdn_chunk_fwd_noalloc";
         default: return "unknown status";
     }
 }

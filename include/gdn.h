@@ -71,7 +71,8 @@ typedef enum gdn_status {
     GDN_ERR_WORKSPACE = 3,   /* workspace NULL, too small or not 256-B aligned */
     GDN_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed           */
     GDN_ERR_TIMEOUT = 5,     /* device: a bounded wait expired                 */
-    GDN_ERR_DEVICE = 6       /* device: an internal consistency check failed   */
+    GDN_ERR_DEVICE = 6,      /* device: an internal consistency check failed   */
+    GDN_ERR_TOO_LARGE = 7    /* gdn_chunk_fwd_noalloc: problem exceeds its scratch */
 } gdn_status;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -157,6 +158,29 @@ GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args* args, void* workspace, size
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 GDN_API const char* gdn_status_string(int status);
+
+/* Forward without a workspace argument, for callers that cannot allocate device
+ * memory: code inside a framework plugin or an inference server whose device
+ * memory is pooled and frozen after start-up, or any runtime that forbids
+ * cudaMalloc on the request path.  (The FlashQLA pages have no counterpart; this
+ * is an interface convenience of this library.)
+ *
+ * It computes exactly what gdn_chunk_fwd computes, always with the CUDA-core
+ * kernels (the path that needs scratch memory), and keeps that scratch in a
+ * fixed device array of GDN_NOALLOC_SCRATCH_BYTES that is part of libgdn.so:
+ * every GPU that loads the library holds it until the process exits.  It calls
+ * no cudaMalloc / cudaFree.  Problems whose scratch would exceed the array are
+ * rejected with GDN_ERR_TOO_LARGE before anything is enqueued (at dk = dv = 128
+ * the array holds about 500 chunk x value-head pairs, e.g. 8 heads x 4000 tokens).
+ *
+ * All calls share the one array per device, so calls whose kernels overlap on
+ * the GPU (different streams, or different threads) race on it; serialise them.
+ * The kernels write every scratch byte before reading it, so nothing needs
+ * clearing between calls.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current) and caches
+ * it; make that first call before any stream capture. */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, void* stream);
 
 /* Number of kernel launches gdn_chunk_fwd / gdn_chunk_bwd enqueue for these
  * arguments (a pure function of the arguments; -1 on an argument error). */
