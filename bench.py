@@ -57,6 +57,28 @@ def bwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
     return T_total * (elt * (Hk * 4 * dk + Hv * 3 * dv) + Hv * 16) + 2 * N * Hv * dk * dv * 4
 
 
+def kernel_sha16():
+    """Fingerprint of the fused forward kernel's source (matches profiles/traffic.json)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("gdn_tc_fwd.cu", "gdn_sm100.cuh"):
+        with open(os.path.join(ROOT, "gated_deltanet_chunked_fwd_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes (read + write) of one fused-forward launch from the committed ncu capture,
+    or None when the kernel source changed since that capture."""
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tp):
+        return None
+    with open(tp) as f:
+        rec = json.load(f).get("fwd_bf16_T4096_H16_d128", {})
+    return rec.get("bytes_per_launch") if rec.get("kernel_sha16") == kernel_sha16() else None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -302,11 +324,7 @@ def run_ours(args, world, rank, local):
     achieved = byts / (ms_step * 1e-3) / 1e9
     tflops_dense = dense * tokens * Hv / (ms_step * 1e-3) / 1e12
     tflops_tri = tri * tokens * Hv / (ms_step * 1e-3) / 1e12
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        with open(tp) as f:
-            traffic = json.load(f).get("fwd_bf16_T4096_H16_d128", {}).get("bytes_per_launch")
+    traffic = traffic_per_launch() if launches == 1 else None
 
     # ---- backward on its own workload (one step per measurement)
     bwd = None
