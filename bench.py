@@ -62,7 +62,7 @@ def kernel_sha16():
     import hashlib
 
     h = hashlib.sha256()
-    for f in ("gdn_tc_fwd.cu", "gdn_sm100.cuh"):
+    for f in ("gdn_tc_fwd.cu", "gdn_tc_common.cuh", "gdn_sm100.cuh"):
         with open(os.path.join(ROOT, "gated_deltanet_chunked_fwd_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -347,7 +347,8 @@ def run_ours(args, world, rank, local):
         bwd = {"workload": "gdn_bwd bf16 B=4 T=8192 H=16 dk=dv=128 C=64", "tokens_per_s": bt * world / (bms * 1e-3),
                "ms": bms, "tflops_dense": bd * bt * Hv / (bms * 1e-3) / 1e12,
                "tflops_tri": btri * bt * Hv / (bms * 1e-3) / 1e12,
-               "hbm_gbs": bb / (bms * 1e-3) / 1e9}
+               "hbm_gbs": bb / (bms * 1e-3) / 1e9,
+               "launches": gdn.launch_count(*qs[:5], backward=True)}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu_base = None

@@ -138,6 +138,13 @@ gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan) {
     b.dg = a->dg;
     b.dS0 = a->dS0;
     const int64_t nc = p.num_chunks;
+    plan->use_tc = !(a->flags & GDN_FLAG_PORTABLE) && tc_bwd_supported(p);
+    if (plan->use_tc) {
+        size_t o1, o2, o3, o4;
+        plan->total = align_up(tc_bwd_workspace(p, &o1, &o2, &o3, &o4), kAlign);
+        plan->launches = p.T_total > 0 ? 2 : 1;
+        return GDN_OK;
+    }
     size_t off = 0;
     plan->off_table = off;
     off = align_up(off + sizeof(int32_t) * (3 * nc + p.N + 1), kAlign);
@@ -238,7 +245,8 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* args, void* workspace, size_t works
     if ((st = check_bwd_pointers(args, plan.b.f))) return st;
     if ((st = check_workspace(workspace, workspace_bytes, plan.total))) return st;
     (void)cudaGetLastError();
-    return launch_bwd_simt(plan, (char*)workspace, (cudaStream_t)stream);
+    return plan.use_tc ? launch_bwd_tc(plan, (char*)workspace, (cudaStream_t)stream)
+                       : launch_bwd_simt(plan, (char*)workspace, (cudaStream_t)stream);
 }
 
 const char* gdn_status_string(int status) {

@@ -89,11 +89,17 @@ bool tc_fwd_supported(const Problem& p);
 
 struct BwdPlan {
     BwdProblem b;
+    bool use_tc;  // tensor-core backward
     size_t off_table, off_W, off_U, off_gam, off_Hc, off_dHc, off_dU, off_dqw, off_dkw, total;
     int launches;
 };
 gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan);
 gdn_status launch_bwd_simt(const BwdPlan& plan, char* ws, cudaStream_t s);
+gdn_status launch_bwd_reduce(const BwdProblem& b, const float* dqw, const float* dkw, cudaStream_t s);
+bool tc_bwd_supported(const Problem& p);
+size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, size_t* off_dqw,
+                        size_t* off_dkw);
+gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s);
 
 // shared SIMT pieces (also used by the backward's forward recompute)
 gdn_status launch_chunk_table(const Problem& p, const ChunkTable& ct, cudaStream_t s);

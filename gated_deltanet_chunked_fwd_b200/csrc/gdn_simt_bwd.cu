@@ -460,6 +460,17 @@ static gdn_status launch_bwd_typed(const BwdPlan& plan, char* ws, cudaStream_t s
     return GDN_OK;
 }
 
+gdn_status launch_bwd_reduce(const BwdProblem& b, const float* dqw, const float* dkw, cudaStream_t s) {
+    const Problem& p = b.f;
+    const int64_t total = p.T_total * p.Hk * p.dk;
+    const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
+    if (p.dtype == GDN_BF16)
+        simt_bwd_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(b, dqw, dkw);
+    else
+        simt_bwd_reduce_kernel<float><<<blocks, 256, 0, s>>>(b, dqw, dkw);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status launch_bwd_simt(const BwdPlan& plan, char* ws, cudaStream_t s) {
     return plan.b.f.dtype == GDN_BF16 ? launch_bwd_typed<__nv_bfloat16>(plan, ws, s)
                                       : launch_bwd_typed<float>(plan, ws, s);

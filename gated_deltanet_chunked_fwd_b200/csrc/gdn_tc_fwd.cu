@@ -36,11 +36,13 @@
 
 #include "gdn_internal.cuh"
 #include "gdn_sm100.cuh"
+#include "gdn_tc_common.cuh"
 
 
 namespace gdn {
 
 using namespace sm100;
+using namespace tc;
 
 namespace {
 
@@ -75,11 +77,9 @@ constexpr uint32_t kBw = 147456;       // 8 KB   T diag(beta Gam): [n][s]
 constexpr uint32_t kBu = 155648;       // 8 KB   T diag(beta): [n][s]
 constexpr uint32_t kWt = 163840;       // 16 KB  W^T: [128 dk rows][64 tokens]
 constexpr uint32_t kUb = 180224;       // 16 KB  U^T: [128 dv rows][64 tokens]
-constexpr int kLd = 68;                // row stride (floats) of the fp32 solve matrix
 constexpr uint32_t kAs = kBw;         // fp32 [64][64] A, float4-XOR-swizzled (Bw/Bu are written
                                        // only after the solve has read A for the last time)
 constexpr uint32_t kM = 196608;        // fp32 [64][68] T (lower triangle; diagonal blocks hold zeros above)
-constexpr int kLdY = 20;               // row stride (floats) of the level scratch
 constexpr uint32_t kYs = kM + 64 * kLd * 4;  // fp32 [3][16][20] solve scratch
 constexpr uint32_t kVec = 218112;      // 3 x 2 KB of per-token vectors, by chunk index mod 3
 constexpr uint32_t kVecStride = 512;   // floats per buffer
@@ -95,119 +95,6 @@ struct TcArgs {
     int auto_warm;  // 1: gate-driven warm-up for segments that do not start a sequence
     float log_eps;  // warm-up stops once the summed log decay is <= log_eps
 };
-
-__device__ __forceinline__ int nchunks_of(int64_t len) { return (int)((len + kChunk - 1) / kChunk); }
-
-__device__ __forceinline__ uint4 pack8(const float* v) {
-    uint4 w;
-    w.x = pack_bf16(v[0], v[1]);
-    w.y = pack_bf16(v[2], v[3]);
-    w.z = pack_bf16(v[4], v[5]);
-    w.w = pack_bf16(v[6], v[7]);
-    return w;
-}
-
-// 32 fp32 values -> 4 swizzled 16-byte chunks (chunk0..chunk0+3) of one 128-byte row
-__device__ __forceinline__ void store_row32(uint8_t* tile, int row, int chunk0, const float* v) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(tile + sw128_off(row, chunk0 + c)) = pack8(v + 8 * c);
-}
-
-// group-wide barrier (named barrier `id` over `cnt` threads), plain and with an AND / OR vote
-__device__ __forceinline__ void wg_sync(int id, int cnt) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(cnt) : "memory");
-}
-__device__ __forceinline__ bool wg_and(int id, int cnt, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, %2, %3, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(cnt)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ bool wg_or(int id, int cnt, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, %2, %3, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(cnt)
-        : "memory");
-    return r != 0;
-}
-
-// A (64 x 64, strictly lower) lives in As with float4 granules XOR-swizzled by row, so that a
-// warp writing 32 rows at one column, or reading 8 rows at one column, hits distinct banks.
-__device__ __forceinline__ int as_idx(int r, int s) { return r * 64 + ((((s >> 2) ^ (r & 15))) << 2) + (s & 3); }
-
-// Level-D merge of the blocked inverse (D = 1, 2, 3) over the blocks (i, i-D), i = D..3:
-//   Y = sum_{k=i-D}^{i-1} A_ik T_k,i-D   then   T_i,i-D = -T_ii Y.
-// T (in M, stride kLd) stores zeros above the diagonal of its diagonal blocks, so all sums
-// run over full blocks.  A task is one row of a block and 4 consecutive columns; the
-// j-range of Y is split over `kSplit` threads and combined with shuffles.
-template <int D>
-__device__ __forceinline__ void solve_level_Y(const float* As, const float* M, float* Ys, int t) {
-    constexpr int kTasks = (4 - D) * 64;  // (block, row, column quad)
-    constexpr int kSplit = kThreadsP / kTasks >= 4 ? 4 : kThreadsP / kTasks;  // 1, 2 or 4
-    constexpr int kLen = 16 * D / kSplit;
-    const int task = t / kSplit, part = t % kSplit;
-    if (task < kTasks) {
-        const int blk = task >> 6, rr = (task >> 2) & 15, quad = task & 3;
-        const int i = blk + D, j0 = i - D;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int jj = 0; jj < kLen; ++jj) {
-            const int j = part * kLen + jj;
-            const float a = As[as_idx(16 * i + rr, 16 * j0 + j)];
-            const float4 tv = *reinterpret_cast<const float4*>(M + (16 * j0 + j) * kLd + 16 * j0 + 4 * quad);
-            acc.x += a * tv.x;
-            acc.y += a * tv.y;
-            acc.z += a * tv.z;
-            acc.w += a * tv.w;
-        }
-#pragma unroll
-        for (int o = 1; o < kSplit; o <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
-        }
-        if (part == 0) *reinterpret_cast<float4*>(Ys + (blk * 16 + rr) * kLdY + 4 * quad) = acc;
-    }
-}
-
-template <int D>
-__device__ __forceinline__ void solve_level_T(float* M, const float* Ys, int t) {
-    constexpr int kTasks = (4 - D) * 64;
-    if (t < kTasks) {
-        const int blk = t >> 6, rr = (t >> 2) & 15, quad = t & 3;
-        const int i = blk + D, j0 = i - D;
-        const float* trow = M + (16 * i + rr) * kLd + 16 * i;  // T_ii row rr (zeros above)
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-            const float4 tt = *reinterpret_cast<const float4*>(trow + 4 * j4);
-            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 y = *reinterpret_cast<const float4*>(Ys + (blk * 16 + 4 * j4 + e) * kLdY + 4 * quad);
-                acc.x += tv[e] * y.x;
-                acc.y += tv[e] * y.y;
-                acc.z += tv[e] * y.z;
-                acc.w += tv[e] * y.w;
-            }
-        }
-        *reinterpret_cast<float4*>(M + (16 * i + rr) * kLd + 16 * j0 + 4 * quad) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -537,35 +424,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* As = (const float*)(sm + kAs);
                 float* M = (float*)(sm + kM);
                 float* Ys = (float*)(sm + kYs);
-                if (t < 64) {  // column cc of diagonal block b
-                    const int b = t >> 4, cc = t & 15;
-                    float x[16];
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
-#pragma unroll
-                        for (int j = 0; j + 1 < r; j += 2) {
-                            s0 -= As[as_idx(16 * b + r, 16 * b + j)] * x[j];
-                            s1 -= As[as_idx(16 * b + r, 16 * b + j + 1)] * x[j + 1];
-                        }
-                        if (r & 1) s0 -= As[as_idx(16 * b + r, 16 * b + r - 1)] * x[r - 1];
-                        x[r] = (r < cc) ? 0.f : s0 + s1;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) M[(16 * b + r) * kLd + 16 * b + cc] = x[r];
-                }
+                solve_diag(As, M, t);  // threads 0..63: the four 16 x 16 diagonal blocks
                 wg_sync(1, kThreadsP);
-                solve_level_Y<1>(As, M, Ys, t);
+                solve_level_Y<1, kThreadsP>(As, M, Ys, t);
                 wg_sync(1, kThreadsP);
-                solve_level_T<1>(M, Ys, t);
+                solve_level_T<1, kThreadsP>(M, Ys, t);
                 wg_sync(1, kThreadsP);
-                solve_level_Y<2>(As, M, Ys, t);
+                solve_level_Y<2, kThreadsP>(As, M, Ys, t);
                 wg_sync(1, kThreadsP);
-                solve_level_T<2>(M, Ys, t);
+                solve_level_T<2, kThreadsP>(M, Ys, t);
                 wg_sync(1, kThreadsP);
-                solve_level_Y<3>(As, M, Ys, t);
+                solve_level_Y<3, kThreadsP>(As, M, Ys, t);
                 wg_sync(1, kThreadsP);
-                solve_level_T<3>(M, Ys, t);
+                solve_level_T<3, kThreadsP>(M, Ys, t);
                 wg_sync(1, kThreadsP);
                 // B operands of MMA_W / MMA_U: row n = t/4, columns s in [16 q, 16 q + 16), s <= n
                 // (written over As, which is no longer read)
@@ -802,37 +673,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;  // resolved once per process (a driver entry point)
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)ptr;
-    }
-    return fn;
-}
-
-// [T_total, H, 128] bf16 viewed as (d, head, token); box 64 x 1 x 64, 128-byte swizzle
-bool make_map(CUtensorMap* map, const void* base, int64_t T_total, int H) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)std::max<int64_t>(T_total, 1)};
-    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
-    cuuint32_t box[3] = {64, 1, 64};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)

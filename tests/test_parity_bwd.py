@@ -83,3 +83,23 @@ def test_backward_workload_full_size_sampled_heads():
                        dST=x["dST"][b:b + 1, h:h + 1])
         got = [sl(t) for t in mine[:5]] + [mine[5][b:b + 1, h:h + 1]]
         compare(got, r, 1e-2, f"unit ({b},{h})")
+
+
+@pytest.mark.parametrize("flags", [0, GDN_FLAG_PORTABLE], ids=["tensor-core", "portable"])
+def test_varlen_ragged_d128_bf16(flags):
+    """bf16 d=128: the shape the tensor-core backward takes (flags=0) and the CUDA-core
+    kernels (portable), on ragged sequences with empty and single-token ones, GQA 2:4."""
+    inp = make_inputs(1, 0, 2, 4, 128, 128, dtype="bf16", seed=11, s0_std=0.2, backward=True,
+                      lengths=[3, 64, 0, 129, 1, 200], device=DEV)
+    compare(run(inp, flags), ref(inp), TOL[inp["q"].dtype], f"flags={flags}")
+
+
+def test_tensor_core_and_portable_backward_agree():
+    """The two backward implementations on the same bf16 input agree with each other
+    at least as closely as each agrees with the oracle."""
+    inp = make_inputs(2, 300, 1, 2, 128, 128, dtype="bf16", seed=12, s0_std=0.1, backward=True,
+                      device=DEV)
+    a, b, r = run(inp), run(inp, GDN_FLAG_PORTABLE), ref(inp)
+    compare(a, r, TOL[inp["q"].dtype], "tensor-core")
+    compare(b, r, TOL[inp["q"].dtype], "portable")
+    compare(a, [t.double().cpu() for t in b], TOL[inp["q"].dtype], "tc vs portable")
