@@ -81,14 +81,6 @@ struct TcBwdArgs {
     float* dkw;      // [T_total][Hv][dk] per-value-head dk
 };
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Reduce-scatter over a warp: lane L ends with the warp-sums of indices L*(N/32) .. +N/32-1
 // in v[0 .. N/32-1].
 template <int N>

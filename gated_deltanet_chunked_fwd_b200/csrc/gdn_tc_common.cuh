@@ -22,6 +22,17 @@ constexpr int kLdY = 20;  // row stride (floats) of the level scratch
 
 __device__ __forceinline__ int nchunks_of(int64_t len) { return (int)((len + kChunk - 1) / kChunk); }
 
+// Per-(chunk, value head) images in the workspace (bf16 T of the WY step, one 8 KB
+// 128-byte-swizzled 64 x 64 tile each) are addressed by a slot: chunk c of sequence n, which
+// starts at token bos, has slot floor(bos / 64) + n + c.  Slots of different chunks never
+// coincide (a sequence's chunks end at most one slot past floor(end / 64) + n, and the next
+// sequence starts at floor(end / 64) + n + 1), and every slot is below img_slots().
+constexpr uint32_t kTImgBytes = 8192;
+__host__ __device__ __forceinline__ int64_t img_slot(int64_t bos, int n, int c) {
+    return bos / kChunk + n + c;
+}
+inline int64_t img_slots(const Problem& p) { return p.T_total / kChunk + p.N + 1; }
+
 __device__ __forceinline__ uint4 pack8(const float* v) {
     uint4 w;
     w.x = pack_bf16(v[0], v[1]);

@@ -1,14 +1,15 @@
 // gdn_tc_fwd.cu -- fused tensor-core forward of the chunked gated delta rule
 // for bf16 tensors with dk = dv = 128 on sm_100a.
 //
-// One launch does the whole forward.  Each CTA owns one (sequence, value head,
-// segment of chunks) and walks its chunks in order, keeping the fp32 state in
-// TMEM; per chunk of C = 64 tokens (notation of gdn_internal.cuh):
+// Two launches do the whole forward.  The first (gdn_tc_wy.cu) forms, for every
+// (chunk, value head) at once, the state-independent WY / UT inverse
+// T = (I + A)^-1, A = strictly-lower(diag(beta) (K K^T o E)), as a bf16 image in the
+// workspace.  The second (this file) is the fused state chain: each CTA owns one
+// (sequence, value head, segment of chunks) and walks its chunks in order, keeping
+// the fp32 state in TMEM; per chunk of C = 64 tokens (notation of gdn_internal.cuh):
 //   gates      gamma = cumsum g, Gam, E = exp(gamma_r - gamma_s)       CUDA cores
-//   MMA1       [Q;K] K^T -> Q K^T and K K^T  (M=128 rows: 64 q + 64 k)  tensor core
-//   WY / UT    A = strictly-lower(diag(beta) K K^T o E),
-//              T = (I + A)^-1 (16x16 diagonal blocks by substitution,
-//              block merges by level)                                   CUDA cores, fp32
+//   MMA1       [Q;K] K^T -> Q K^T (rows 0-63 of the M=128 product)      tensor core
+//   Bw, Bu     T diag(beta Gam), T diag(beta) from the T image          CUDA cores
 //   MMA_W/U    W^T = K^T (T diag(beta Gam))^T,  Ut^T = V^T (T diag(beta))^T
 //   MMA_HW     U^T = Ut^T - H^T W^T  (accumulated onto Ut^T, A negated)
 //   MMA_HQ/UP  O^T = Gam * (H^T Q^T) + U^T P^T,  P = lower-incl(Q K^T o E)
@@ -16,7 +17,8 @@
 // All matrices are oriented so that a 128-wide head dimension is the MMA's M
 // (TMEM lane = dv or dk index), so every MMA is M = 128 with N = 64 or 128.
 // Operands live in shared memory as 128-byte-swizzled tiles; q / k / v tiles
-// come in by TMA (double-buffered: chunk c+1 loads while chunk c computes).
+// come in by TMA and the T image by a bulk copy (double-buffered: chunk c+1 loads
+// while chunk c computes).
 //
 // Long sequences are split into segments that run on different SMs
 // (gate-driven context parallelism, dothoosh.com FlashQLA article, first
@@ -47,8 +49,8 @@ using namespace tc;
 namespace {
 
 // Two groups of warps run a two-stage software pipeline over the chunks of a segment:
-//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T / K K^T,
-//                                       P and A, T = (I + A)^-1, W^T and Ut^T, W^T -> smem
+//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T, P,
+//                                       Bw / Bu from the T image, W^T and Ut^T, W^T -> smem
 //   group S (threads 256-383, 4 warps)  the state chain of chunk k-1..k: U^T = Ut^T - H^T W^T,
 //                                       H^T <- Gam_n H^T + U^T Kd, outputs, bf16 copy of H
 // Each group has one tcgen05 issuer (threads 0 and 256) and its own commit
@@ -61,7 +63,7 @@ constexpr int kThreadsS = 128;
 constexpr int kTmemCols = 512;
 // TMEM column map (lane = row of the M = 128 MMA)
 constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk     [0, 128)
-constexpr uint32_t kColR1 = 128;  // Q K^T / K K^T, then W^T (warpgroup P)   [128, 192)
+constexpr uint32_t kColR1 = 128;  // Q K^T (lanes 0-63), then W^T (group P)   [128, 192)
 constexpr uint32_t kColR2 = 192;  // 2 x (Ut^T -> U^T), by chunk parity      [192, 320)
 constexpr uint32_t kColHQ = 320;  // H^T Q^T                                 [320, 384)
 constexpr uint32_t kColUP = 384;  // U^T P^T                                 [384, 448)
@@ -71,22 +73,17 @@ constexpr uint32_t kColHb = 448;  // bf16 H^T, A operand (K pairs per column) [4
 // shared memory carve-up (bytes from a 1024-aligned base)
 constexpr uint32_t kStageQK = 0;       // 2 x 32 KB: [dk atom][q rows 0-63 | k rows 64-127][128 B]
 constexpr uint32_t kStageV = 65536;    // 2 x 16 KB: [dv atom][64 rows][128 B]
-constexpr uint32_t kHb = 98304;        // 32 KB  bf16 H^T: [dk atom][128 dv rows][128 B]
-constexpr uint32_t kPt = 131072;       // 2 x 8 KB  P: [64 n rows][64 s], by chunk parity
-constexpr uint32_t kBw = 147456;       // 8 KB   T diag(beta Gam): [n][s]
-constexpr uint32_t kBu = 155648;       // 8 KB   T diag(beta): [n][s]
-constexpr uint32_t kWt = 163840;       // 16 KB  W^T: [128 dk rows][64 tokens]
-constexpr uint32_t kUb = 180224;       // 16 KB  U^T: [128 dv rows][64 tokens]
-constexpr uint32_t kAs = kBw;         // fp32 [64][64] A, float4-XOR-swizzled (Bw/Bu are written
-                                       // only after the solve has read A for the last time)
-constexpr uint32_t kM = 196608;        // fp32 [64][68] T (lower triangle; diagonal blocks hold zeros above)
-constexpr uint32_t kYs = kM + 64 * kLd * 4;  // fp32 [3][16][20] solve scratch
-constexpr uint32_t kVec = 218112;      // 3 x 2 KB of per-token vectors, by chunk index mod 3
+constexpr uint32_t kPt = 98304;        // 2 x 8 KB  P: [64 n rows][64 s], by chunk parity
+constexpr uint32_t kBw = 114688;       // 8 KB   T diag(beta Gam): [n][s]
+constexpr uint32_t kBu = 122880;       // 8 KB   T diag(beta): [n][s]
+constexpr uint32_t kWt = 131072;       // 16 KB  W^T: [128 dk rows][64 tokens]
+constexpr uint32_t kTimg = 147456;     // 2 x 8 KB  bf16 T images [n][s], by chunk parity
+constexpr uint32_t kVec = 163840;      // 3 x 2 KB of per-token vectors, by chunk index mod 3
 constexpr uint32_t kVecStride = 512;   // floats per buffer
 constexpr uint32_t kRed = kVec + 3 * kVecStride * 4;  // 16 floats
 constexpr uint32_t kBar = kRed + 64;   // 9 mbarriers + TMEM base
 constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
-static_assert(kYs + 3 * 16 * kLdY * 4 <= kVec, "solve scratch overlaps the vectors");
+static_assert(kTimg + 2 * kTImgBytes <= kVec, "T images overlap the vectors");
 
 struct TcArgs {
     Problem p;
@@ -94,6 +91,7 @@ struct TcArgs {
     int fixed_segs; // segments per sequence when cu_seqlens is absent
     int auto_warm;  // 1: gate-driven warm-up for segments that do not start a sequence
     float log_eps;  // warm-up stops once the summed log decay is <= log_eps
+    const uint8_t* timg;  // T images of the WY step, by (image slot, value head)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -247,12 +245,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t0 = (int)(bos + (int64_t)c * kChunk);
         uint8_t* qk = sm + kStageQK + stage * 32768;
         uint8_t* vv = sm + kStageV + stage * 16384;
-        mbar_arrive_expect_tx(&bar_tma[stage], 49152);
+        mbar_arrive_expect_tx(&bar_tma[stage], 49152 + kTImgBytes);
         for (int a = 0; a < 2; ++a) {
             tma_load_3d(qk + a * 16384, &tm_q, &bar_tma[stage], 64 * a, hk, t0);
             tma_load_3d(qk + a * 16384 + 8192, &tm_k, &bar_tma[stage], 64 * a, hk, t0);
             tma_load_3d(vv + a * 8192, &tm_v, &bar_tma[stage], 64 * a, h, t0);
         }
+        bulk_load(sm + kTimg + stage * kTImgBytes,
+                  args.timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kTImgBytes, kTImgBytes,
+                  &bar_tma[stage]);
     };
 
     // ---- initial state (warpgroup S): H^T (lane = dv index m) from S0 or zero
@@ -376,95 +377,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
 
-            // P (rows 0..63, into Pt[stage]) and A (rows 64..127, into As);
-            // this thread: TMEM lane `row`, columns [32 hf, 32 hf + 32)
-            {
-                float v[32];
-                tmem_ld32(tl + kColR1 + 32 * hf, v);
-                const int r = row & 63;
-                const int s0 = 32 * hf;
-                const float ar = va[r];
-                float E[32];
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
-                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) E[4 * c4 + e] = fac ? ar * bb[e] : exp2f(ar - bb[e]);
-                }
-                if (row < 64) {
-                    if (emit) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int s = s0 + e;
-                            v[e] = (s <= r && r < lc) ? v[e] * E[e] : 0.f;
-                        }
-                        store_row32(sm + kPt + stage * 8192, r, 4 * hf, v);
-                    }
-                } else {
-                    const float br = vbeta[r];
-                    float* As = (float*)(sm + kAs);
+            // P (TMEM lanes 0..63: warps 0, 1, 4, 5, columns [32 hf, 32 hf + 32)) and, meanwhile,
+            // the B operands of MMA_W / MMA_U from the T image (warps 2, 3, 6, 7):
+            // Bw = T diag(beta Gam), Bu = T diag(beta), in the image's swizzled layout
+            if ((warp & 3) < 2) {
+                if (emit) {
+                    float v[32];
+                    tmem_ld32(tl + kColR1 + 32 * hf, v);
+                    const int r = row;
+                    const int s0 = 32 * hf;
+                    const float ar = va[r];
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
-                        float4 w;
-                        const int sb = s0 + 4 * c4;
-                        w.x = (sb + 0 < r && r < lc) ? br * v[4 * c4 + 0] * E[4 * c4 + 0] : 0.f;
-                        w.y = (sb + 1 < r && r < lc) ? br * v[4 * c4 + 1] * E[4 * c4 + 1] : 0.f;
-                        w.z = (sb + 2 < r && r < lc) ? br * v[4 * c4 + 2] * E[4 * c4 + 2] : 0.f;
-                        w.w = (sb + 3 < r && r < lc) ? br * v[4 * c4 + 3] * E[4 * c4 + 3] : 0.f;
-                        *reinterpret_cast<float4*>(As + as_idx(r, sb)) = w;
-                    }
-                }
-            }
-            tc_fence_before();
-            wg_sync(1, kThreadsP);
-
-            // T = (I + A)^-1 in fp32: diagonal 16x16 blocks by substitution, then 3 merge levels
-            {
-                const float* As = (const float*)(sm + kAs);
-                float* M = (float*)(sm + kM);
-                float* Ys = (float*)(sm + kYs);
-                solve_diag(As, M, t);  // threads 0..63: the four 16 x 16 diagonal blocks
-                wg_sync(1, kThreadsP);
-                solve_level_Y<1, kThreadsP>(As, M, Ys, t);
-                wg_sync(1, kThreadsP);
-                solve_level_T<1, kThreadsP>(M, Ys, t);
-                wg_sync(1, kThreadsP);
-                solve_level_Y<2, kThreadsP>(As, M, Ys, t);
-                wg_sync(1, kThreadsP);
-                solve_level_T<2, kThreadsP>(M, Ys, t);
-                wg_sync(1, kThreadsP);
-                solve_level_Y<3, kThreadsP>(As, M, Ys, t);
-                wg_sync(1, kThreadsP);
-                solve_level_T<3, kThreadsP>(M, Ys, t);
-                wg_sync(1, kThreadsP);
-                // B operands of MMA_W / MMA_U: row n = t/4, columns s in [16 q, 16 q + 16), s <= n
-                // (written over As, which is no longer read)
-                const int nrow = t >> 2, q = t & 3;
-                float vw[16], vu[16];
+                        const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
+                        const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int sb = 16 * q + 4 * c4;
-                    const float4 tt = *reinterpret_cast<const float4*>(M + nrow * kLd + sb);
-                    const float4 g4 = *reinterpret_cast<const float4*>(vbG + sb);
-                    const float4 b4 = *reinterpret_cast<const float4*>(vbeta + sb);
-                    const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-                    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                        for (int e = 0; e < 4; ++e) {
+                            const int s = s0 + 4 * c4 + e;
+                            const float E = fac ? ar * bb[e] : exp2f(ar - bb[e]);
+                            v[4 * c4 + e] = (s <= r && r < lc) ? v[4 * c4 + e] * E : 0.f;
+                        }
+                    }
+                    store_row32(sm + kPt + stage * 8192, r, 4 * hf, v);
+                }
+            } else {
+                const int li = ((warp >> 2) << 6) | ((warp & 1) << 5) | lane;  // 0..127
+                const int nr = li >> 1, c0 = 4 * (li & 1);
+                const uint8_t* timg_s = sm + kTimg + stage * kTImgBytes;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int chunk = c0 + cc;
+                    const uint32_t off = sw128_off(nr, chunk);
+                    uint4 u = *reinterpret_cast<const uint4*>(timg_s + off);
+                    const __nv_bfloat162* t2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+                    float tv[8], vw[8], vu[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float tv_e = (sb + e <= nrow) ? tv[e] : 0.f;
-                        vw[4 * c4 + e] = tv_e * gv[e];
-                        vu[4 * c4 + e] = tv_e * bv[e];
+                        const float2 f = __bfloat1622float2(t2[e]);
+                        tv[2 * e] = f.x;
+                        tv[2 * e + 1] = f.y;
                     }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        vw[e] = tv[e] * vbG[8 * chunk + e];
+                        vu[e] = tv[e] * vbeta[8 * chunk + e];
+                    }
+                    *reinterpret_cast<uint4*>(sm + kBw + off) = pack8(vw);
+                    *reinterpret_cast<uint4*>(sm + kBu + off) = pack8(vu);
                 }
-                wg_sync(1, kThreadsP);  // As overlaps Bw / Bu
-                *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q)) = pack8(vw);
-                *reinterpret_cast<uint4*>(sm + kBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
-                *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q)) = pack8(vu);
-                *reinterpret_cast<uint4*>(sm + kBu + sw128_off(nrow, 2 * q + 1)) = pack8(vu + 8);
             }
-            fence_proxy_async();
+            fence_proxy_async();  // Pt, Bw, Bu are read by the tensor core
+            tc_fence_before();
             wg_sync(1, kThreadsP);
 
             if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1);  MMA_U: Ut^T = V^T Bu^T (R2[stage])
@@ -730,13 +693,17 @@ bool tc_fwd_supported(const Problem& p) {
     return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128;
 }
 
-size_t tc_fwd_workspace(const Problem&) { return 0; }
-int tc_fwd_launches(const Problem&) { return 1; }
+// workspace: the T images of the WY step
+size_t tc_fwd_workspace(const Problem& p) { return wy_tc_workspace(p); }
+int tc_fwd_launches(const Problem& p) { return (p.num_chunks > 0 ? 1 : 0) + 1; }
 
-gdn_status launch_fwd_tc(const FwdPlan& plan, char*, cudaStream_t s) {
+gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
     const Problem& p = plan.p;
+    gdn_status st = launch_wy_tc(p, (uint8_t*)ws, s);
+    if (st) return st;
     TcArgs a;
     a.p = p;
+    a.timg = (const uint8_t*)ws;
     const std::vector<int> nck = chunk_counts(p, plan.cu_host);
     const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count());
     a.L = sc.L;

@@ -80,8 +80,11 @@ def test_misaligned_tensor_is_rejected(field, offset):
 
 
 def test_workspace_checks():
-    # the tensor-core path (bf16, 128 x 128) needs no workspace; the portable one does
-    assert ws_size(fwd_args()) == (OK, 0)
+    # the tensor-core path (bf16, 128 x 128) keeps one 8 KB T image per (image slot, value
+    # head), slots = T_total // 64 + N + 1; the portable path keeps fp32 W, U, gamma, states
+    st, need_tc = ws_size(fwd_args())
+    assert st == OK and need_tc == (256 // 64 + 1 + 1) * 4 * 8192
+    assert call_fwd(fwd_args(), ws=0) == WORKSPACE
     a = fwd_args(flags=_abi.GDN_FLAG_PORTABLE)
     st, need = ws_size(a)
     assert st == OK and need > 0 and need % 256 == 0
