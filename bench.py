@@ -372,7 +372,7 @@ def run_ours(args, world, rank, local):
                        "global_batch": world, "seq_len": T, "heads": Hv, "head_dim": dk,
                        "parallelism": f"replicas x{world} (no collective)",
                        "l2": "flushed before every timed step (2x L2 write, outside the events)",
-                       "path": "tensor-core fused" if launches == 1 else "cuda-core 4-kernel"},
+                       "path": "tensor-core (WY kernel + fused state chain)" if launches <= 2 else "cuda-core 4-kernel"},
             "tflops": {"dense": tflops_dense, "triangular": tflops_tri, "peak_bf16": bf16,
                        "frac_dense": tflops_dense / bf16},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",

@@ -11,7 +11,7 @@
 //   MMA1       [Q;K] K^T -> Q K^T (rows 0-63 of the M=128 product)      tensor core
 //   Bw, Bu     T diag(beta Gam), T diag(beta) from the T image          CUDA cores
 //   MMA_W/U    W^T = K^T (T diag(beta Gam))^T,  Ut^T = V^T (T diag(beta))^T
-//   MMA_HW     U^T = Ut^T - H^T W^T  (accumulated onto Ut^T, A negated)
+//   MMA_HW     U^T = Ut^T - H^T W^T  (accumulated onto Ut^T, B = -W^T)
 //   MMA_HQ/UP  O^T = Gam * (H^T Q^T) + U^T P^T,  P = lower-incl(Q K^T o E)
 //   MMA_H      H^T <- Gam_n H^T + (U^T diag(exp(gamma_n - gamma))) K
 // All matrices are oriented so that a 128-wide head dimension is the MMA's M
@@ -52,7 +52,7 @@ namespace {
 //   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T, P,
 //                                       Bw / Bu from the T image, W^T and Ut^T, W^T -> smem
 //   group S (threads 256-383, 4 warps)  the state chain of chunk k-1..k: U^T = Ut^T - H^T W^T,
-//                                       H^T <- Gam_n H^T + U^T Kd, outputs, bf16 copy of H
+//                                       H^T <- Gam_n H^T + (U^T diag(decay)) K, outputs, bf16 H
 // Each group has one tcgen05 issuer (threads 0 and 256) and its own commit
 // barrier; they hand chunks over through mbarriers (full / empty pairs).  Warp w
 // reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so group P's two warps per lane
@@ -78,9 +78,9 @@ constexpr uint32_t kBw = 114688;       // 8 KB   T diag(beta Gam): [n][s]
 constexpr uint32_t kBu = 122880;       // 8 KB   T diag(beta): [n][s]
 constexpr uint32_t kWt = 131072;       // 16 KB  W^T: [128 dk rows][64 tokens]
 constexpr uint32_t kTimg = 147456;     // 2 x 8 KB  bf16 T images [n][s], by chunk parity
-constexpr uint32_t kVec = 163840;      // 3 x 2 KB of per-token vectors, by chunk index mod 3
+constexpr uint32_t kVec = 163840;      // 4 x 2 KB of per-token vectors, by chunk index mod 4
 constexpr uint32_t kVecStride = 512;   // floats per buffer
-constexpr uint32_t kRed = kVec + 3 * kVecStride * 4;  // 16 floats
+constexpr uint32_t kRed = kVec + 4 * kVecStride * 4;  // 16 floats
 constexpr uint32_t kBar = kRed + 64;   // 9 mbarriers + TMEM base
 constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
 static_assert(kTimg + 2 * kTImgBytes <= kVec, "T images overlap the vectors");
@@ -92,6 +92,7 @@ struct TcArgs {
     int auto_warm;  // 1: gate-driven warm-up for segments that do not start a sequence
     float log_eps;  // warm-up stops once the summed log decay is <= log_eps
     const uint8_t* timg;  // T images of the WY step, by (image slot, value head)
+    const float2* summ;   // per (image slot, value head): summed log decay, norm-condition flag
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -100,7 +101,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Problem& p = args.p;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* vred = (float*)(sm + kRed);
     uint64_t* bars = (uint64_t*)(sm + kBar);
     uint64_t* bar_tma = bars;          // [2] stage full (TMA transaction bytes)
     uint64_t* bar_mma_p = bars + 2;    // warpgroup P's MMA completions
@@ -108,7 +108,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bar_wt_full = bars + 4;  // W^T of chunk k in smem, Ut^T of chunk k in TMEM
     uint64_t* bar_wt_empty = bars + 5; // MMA_HW of chunk k has read W^T
     uint64_t* bar_s_done = bars + 6;   // [2] group S finished chunk k (parity buffers free)
-    uint64_t* bar_gates = bars + 8;    // group P wrote the per-token vectors of chunk k
     uint32_t* tmem_slot = (uint32_t*)(bars + 9);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -168,58 +167,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c0 = min(nck, seg * args.L);
     const int c1 = min(nck, (seg + 1) * args.L);
 
-    // ---- warm-up start (gate-driven); exact start from S0 when seg == 0
-    int cstart = 0;
-    if (seg > 0 && args.auto_warm) {
-        float cum = 0.f;
-        int w = c0;
-        int bad = 0;
-        while (w > 0 && cum > args.log_eps) {
-            --w;
-            const int64_t t0 = bos + (int64_t)w * kChunk;
-            const int lw = (int)min((int64_t)kChunk, len - (int64_t)w * kChunk);
-            // summed log decay of chunk w, and the contraction condition beta |k|^2 <= 2
-            const int r = tid >> 2, q = tid & 3;
-            float nrm = 0.f, gsum = 0.f;
-            int viol = 0;
-            if (r < lw) {
-                const uint4* kr = (const uint4*)((const __nv_bfloat16*)p.k +
-                                                 ((t0 + r) * p.Hk + hk) * dk + q * 32);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint4 u = kr[c];
-                    const __nv_bfloat162* b2 = (const __nv_bfloat162*)&u;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float2 f = __bfloat1622float2(b2[e]);
-                        nrm += f.x * f.x + f.y * f.y;
-                    }
-                }
-            }
-            nrm += __shfl_xor_sync(0xffffffffu, nrm, 1);
-            nrm += __shfl_xor_sync(0xffffffffu, nrm, 2);
-            if (q == 0 && r < lw) {
-                const float b = p.beta[(t0 + r) * Hv + h];
-                gsum = p.g[(t0 + r) * Hv + h];
-                if (!(b >= 0.f && b * nrm <= 2.f)) viol = 1;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
-            viol = __syncthreads_or(viol);
-            if (lane == 0) vred[warp] = gsum;
-            __syncthreads();
-            float tot = 0.f;
-#pragma unroll
-            for (int i = 0; i < kThreads / 32; ++i) tot += vred[i];
-            cum += tot;
-            __syncthreads();
-            bad |= viol;
-        }
-        cstart = (cum > args.log_eps || bad) ? 0 : w;
-    }
-    const bool exact = (cstart == 0);
-    const int nk = c1 - cstart;  // chunks this CTA walks (warm-up + own)
-
     // ---- set-up: barriers, TMEM
     if (tid == 0) {
         for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
@@ -239,6 +186,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lane quarter
     const uint32_t sbase = smem_u32(sm);
 
+    // ---- initial state (warpgroup S): H^T (lane = dv index m) from S0 or zero
+    auto load_state = [&](bool from_s0) {
+        const int m = tid - kThreadsP;
+        const float* s0 = (from_s0 && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
+        float v[64];
+        uint32_t w[32];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e] = s0 ? s0[(int64_t)(64 * a + e) * dv + m] : 0.f;
+            tmem_st64(tl + kColH + 64 * a, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+            tmem_st32u(tl + kColHb + 32 * a, w);
+        }
+    };
+    // A segment that starts its sequence (or any segment when the warm-up is off) starts
+    // exactly from S0; that does not depend on the WY step, so it runs before waiting for it.
+    const bool known_exact = (seg == 0) || !args.auto_warm;
+    if (known_exact && tid >= kThreadsP) load_state(true);
+    // The WY step (the previous launch) must be complete before its images and summaries are read.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // ---- warm-up start (gate-driven); exact start from S0 when seg == 0.  The WY step left,
+    // per chunk, its summed log decay and whether some token breaks 0 <= beta |k|^2 <= 2.
+    int cstart = 0;
+    if (!known_exact) {
+        float cum = 0.f;
+        int w = c0;
+        bool bad = false;
+        while (w > 0 && cum > args.log_eps) {
+            --w;
+            const float2 cs = args.summ[img_slot(bos, n, w) * Hv + h];
+            cum += cs.x;
+            bad |= cs.y != 0.f;
+        }
+        cstart = (cum > args.log_eps || bad) ? 0 : w;
+    }
+    const bool exact = (cstart == 0);
+    const int nk = c1 - cstart;  // chunks this CTA walks (warm-up + own)
+    if (!known_exact && tid >= kThreadsP) load_state(exact);
     auto issue_tma = [&](int k) {
         const int c = cstart + k;
         const int stage = k & 1;
@@ -256,22 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   &bar_tma[stage]);
     };
 
-    // ---- initial state (warpgroup S): H^T (lane = dv index m) from S0 or zero
-    if (tid >= kThreadsP) {
-        const int m = tid - kThreadsP;
-        const float* s0 = (exact && p.S0) ? p.S0 + ((int64_t)n * Hv + h) * dk * dv : nullptr;
-        float v[64];
-        uint32_t w[32];
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) v[e] = s0 ? s0[(int64_t)(64 * a + e) * dv + m] : 0.f;
-            tmem_st64(tl + kColH + 64 * a, v);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-            tmem_st32u(tl + kColHb + 32 * a, w);
-        }
-    } else if (tid == 0) {
+    if (tid == 0) {
         if (nk > 0) issue_tma(0);
         if (nk > 1) issue_tma(1);
     }
@@ -292,16 +265,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hf = t >> 7;                       // which 32-column half of a TMEM row
         const int row = ((warp & 3) << 5) | lane;    // TMEM lane (= MMA row) this thread reads
         uint32_t ph = 0;  // parity of bar_mma_p
-        float nxt_b = 0.f, nxt_g = 0.f;
-        auto load_gates = [&](int k) {
-            const int c = cstart + k;
-            const int64_t t0 = bos + (int64_t)c * kChunk;
-            const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-            nxt_b = t < lc ? p.beta[(t0 + t) * Hv + h] : 0.f;
-            nxt_g = t < lc ? p.g[(t0 + t) * Hv + h] : 0.f;  // padding: g = 0
+        // Gates run one chunk ahead in warp 2 (lane l: rows 2l, 2l+1), so chunk k+1's vectors
+        // are in shared memory before chunk k is handed to group S.  g / beta of the chunk after
+        // that are prefetched into registers.
+        float gx0 = 0.f, gx1 = 0.f, bx0 = 0.f, bx1 = 0.f;
+        auto load_gates = [&](int kk) {
+            const int cc = cstart + kk;
+            const int64_t t0 = bos + (int64_t)cc * kChunk;
+            const int lcc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
+            const int r0 = 2 * lane;
+            gx0 = r0 < lcc ? p.g[(t0 + r0) * Hv + h] : 0.f;  // padding: g = 0, beta = 0
+            gx1 = r0 + 1 < lcc ? p.g[(t0 + r0 + 1) * Hv + h] : 0.f;
+            bx0 = r0 < lcc ? p.beta[(t0 + r0) * Hv + h] : 0.f;
+            bx1 = r0 + 1 < lcc ? p.beta[(t0 + r0 + 1) * Hv + h] : 0.f;
         };
-        if (t < 64 && nk > 0) load_gates(0);
-        const float LOG2E = 1.4426950408889634f;
+        // vectors of chunk kk (buffer kk mod 4): beta, gamma = cumsum g, Gam = exp(gamma),
+        // beta Gam, decay to the chunk end exp(gamma_n - gamma), the E factors a, b, and the
+        // flag that says whether E_rs = a_r b_s (every |gamma - gamma_31| < 80) or exp2(a_r - b_s)
+        auto gates = [&](int kk) {
+            float* vec = (float*)(sm + kVec) + (kk & 3) * kVecStride;
+            float incl = gx0 + gx1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const float g1 = incl, g0 = incl - gx1;
+            const float gm = __shfl_sync(0xffffffffu, g1, 15);  // gamma_31
+            const float gl = __shfl_sync(0xffffffffu, g1, 31);  // gamma_63 (= gamma of the last token)
+            const bool fac = __all_sync(0xffffffffu, fabsf(g0 - gm) < 80.f && fabsf(g1 - gm) < 80.f);
+            const float LOG2E = 1.4426950408889634f;
+            const float e0 = expf(g0), e1 = expf(g1);
+            const int r0 = 2 * lane;
+            *reinterpret_cast<float2*>(vec + r0) = make_float2(bx0, bx1);
+            *reinterpret_cast<float2*>(vec + 64 + r0) = make_float2(g0, g1);
+            *reinterpret_cast<float2*>(vec + 128 + r0) = make_float2(e0, e1);
+            *reinterpret_cast<float2*>(vec + 192 + r0) = make_float2(bx0 * e0, bx1 * e1);
+            *reinterpret_cast<float2*>(vec + 256 + r0) = make_float2(expf(gl - g0), expf(gl - g1));
+            *reinterpret_cast<float2*>(vec + 320 + r0) =
+                fac ? make_float2(expf(g0 - gm), expf(g1 - gm)) : make_float2(g0 * LOG2E, g1 * LOG2E);
+            *reinterpret_cast<float2*>(vec + 384 + r0) =
+                fac ? make_float2(expf(gm - g0), expf(gm - g1)) : make_float2(g0 * LOG2E, g1 * LOG2E);
+            if (lane == 0) vec[448] = fac ? 1.f : 0.f;
+        };
+        if (warp == 2 && nk > 0) {
+            load_gates(0);
+            gates(0);
+            if (nk > 1) load_gates(1);
+        }
 
         for (int k = 0; k < nk; ++k) {
             const int c = cstart + k;
@@ -310,14 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t sV = sbase + kStageV + stage * 16384;
-            float* vec = (float*)(sm + kVec) + (k % 3) * kVecStride;
-            float* vbeta = vec;
-            float* vgam = vec + 64;
-            float* vGam = vec + 128;
-            float* vbG = vec + 192;
-            float* vdec = vec + 256;
-            float* va = vec + 320;
-            float* vb = vec + 384;
+            const float* vec = (const float*)(sm + kVec) + (k & 3) * kVecStride;
+            const float* vbeta = vec;
+            const float* vbG = vec + 192;
+            const float* va = vec + 320;
+            const float* vb = vec + 384;
 
             // buffers of parity `stage` are free once warpgroup S finished chunk k-2
             if (k >= 2) {
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = wg_and(1, kThreadsP, mbar_wait(&bar_tma[stage], (k >> 1) & 1));
             if (!ok) break;
-            if (t == 0) {  // MMA1: [Q;K] K^T -> Q K^T (lanes 0-63), K K^T (lanes 64-127)
+            if (t == 0) {  // MMA1: [Q;K] K^T -> Q K^T (lanes 0-63; lanes 64-127 are unused)
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -336,46 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(bar_mma_p);
             }
-
-            // gates (threads 0..63): gamma = cumsum g; overlaps MMA1
-            float gr = 0.f, gm = 0.f;
-            if (t < 64) {
-                float x = nxt_g;
-                const float b = nxt_b;
-                if (k + 1 < nk) load_gates(k + 1);
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, o);
-                    if (lane >= o) x += y;
-                }
-                vbeta[t] = b;
-                vgam[t] = x;
+            if (warp == 2 && k + 1 < nk) {  // the next chunk's gates, while MMA1 runs
+                gates(k + 1);
+                if (k + 2 < nk) load_gates(k + 2);
             }
-            wg_sync(1, kThreadsP);
-            if (t < 64) {
-                gr = vgam[t] + (t >= 32 ? vgam[31] : 0.f);
-                gm = vgam[31];
-                const float gl = vgam[63] + vgam[31];
-                const float eg = expf(gr);
-                vGam[t] = eg;
-                vbG[t] = vbeta[t] * eg;
-                vdec[t] = expf(gl - gr);
-            }
-            // E_rs = exp(gamma_r - gamma_s) = a_r * b_s with a_r = exp(gamma_r - gamma_31),
-            // b_s = exp(gamma_31 - gamma_s) while every |gamma - gamma_31| < 80 (both factors
-            // far inside the fp32 range); otherwise one exp2 per entry.
-            const bool fac = !wg_or(1, kThreadsP, t < 64 && !(fabsf(gr - gm) < 80.f));
-            if (t < 64) {
-                va[t] = fac ? expf(gr - gm) : gr * LOG2E;
-                vb[t] = fac ? expf(gm - gr) : gr * LOG2E;
-            }
-            wg_sync(1, kThreadsP);
-            if (t == 0) mbar_arrive(bar_gates);
-
             ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
             ph ^= 1;
             if (!ok) break;
             tc_fence_after();
+            const bool fac = vec[448] != 0.f;
 
             // P (TMEM lanes 0..63: warps 0, 1, 4, 5, columns [32 hf, 32 hf + 32)) and, meanwhile,
             // the B operands of MMA_W / MMA_U from the T image (warps 2, 3, 6, 7):
@@ -457,23 +434,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; ++e) v[e] = -v[e];  // MMA_HW accumulates -H^T W^T
                 store_row32(sm + kWt, row, 4 * hf, v);
             }
-            {  // K rows <- exp(gamma_n - gamma_s) * K rows (B operand of MMA_H; MMA1 / MMA_W are done)
-                const int srow = t >> 2, q = t & 3;
-                uint8_t* krow = sm + kStageQK + stage * 32768 + (q >> 1) * 16384 + (64 + srow) * 128;
-                const float d = vdec[srow];
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int c8 = 4 * (q & 1) + ((i4 + srow) & 3);  // rotated: rows spread over banks
-                    uint4 u = *reinterpret_cast<uint4*>(krow + 16 * c8);
-                    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float2 f = __bfloat1622float2(b2[e]);
-                        b2[e] = __floats2bfloat162_rn(f.x * d, f.y * d);
-                    }
-                    *reinterpret_cast<uint4*>(krow + 16 * c8) = u;
-                }
-            }
             fence_proxy_async();
             tc_fence_before();
             wg_sync(1, kThreadsP);
@@ -491,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int cc = cstart + kk;
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
-            const float* vGam = (const float*)(sm + kVec) + (kk % 3) * kVecStride + 128;
+            const float* vGam = (const float*)(sm + kVec) + (kk & 3) * kVecStride + 128;
             __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -548,17 +508,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             if (m == 0) mbar_arrive(bar_wt_empty);
 
-            {  // U^T (lane = dv index, fp32) -> bf16 pairs in the first 32 columns of the same buffer
+            {  // U^T (lane = dv index, fp32) -> bf16 pairs in the same buffer: U^T in columns 0-31
+               // (A of MMA_UP), U^T diag(exp(gamma_n - gamma)) in columns 32-63 (A of MMA_H)
+                const float* vdec = (const float*)(sm + kVec) + (k & 3) * kVecStride + 256;
                 float v[64];
                 uint32_t w[32];
                 tmem_ld64(tl + colR2, v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
                 tmem_st32u(tl + colR2, w);
+#pragma unroll
+                for (int e4 = 0; e4 < 16; ++e4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(vdec + 4 * e4);
+                    w[2 * e4] = pack_bf16(v[4 * e4] * d4.x, v[4 * e4 + 1] * d4.y);
+                    w[2 * e4 + 1] = pack_bf16(v[4 * e4 + 2] * d4.z, v[4 * e4 + 3] * d4.w);
+                }
+                tmem_st32u(tl + colR2 + 32, w);
             }
             tc_fence_before();
             wg_sync(2, kThreadsS);
-            if (m == 0) {  // MMA_HQ: H^T Q^T;  MMA_UP: U^T P^T;  MMA_H: H^T += U^T Kd
+            if (m == 0) {  // MMA_HQ: H^T Q^T;  MMA_UP: U^T P^T;  MMA_H: H^T += (U^T diag(decay)) K
                 tc_fence_after();
                 if (emit) {
 #pragma unroll
@@ -575,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    mma_bf16_ts(tmem + kColH, tmem + colR2 + 8 * j,
+                    mma_bf16_ts(tmem + kColH, tmem + colR2 + 32 + 8 * j,
                                 desc_sw128(sQK + 8192 + j * 2048, 16384, 1024), id_bmn_n128, 1);
                 mma_commit(bar_mma_s);
             }
@@ -586,13 +555,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m == 0 && k + 2 < nk) issue_tma(k + 2);  // stage `stage` is no longer read
 
             // bf16 copy of the new state (A operand of the next chunk's MMAs); pre-scale by its Gam_n
+            // (chunk k+1's vectors were written before chunk k was handed over)
             const bool more = k + 1 < nk;
-            if (more) {
-                ok = wg_and(2, kThreadsS, mbar_wait(bar_gates, (k + 1) & 1));
-                if (!ok) break;
-            }
             {
-                const float Gn = more ? ((const float*)(sm + kVec))[((k + 1) % 3) * kVecStride + 128 + 63] : 1.f;
+                const float Gn = more ? ((const float*)(sm + kVec))[((k + 1) & 3) * kVecStride + 128 + 63] : 1.f;
                 float v[64];
                 uint32_t w[32];
 #pragma unroll
@@ -699,11 +665,11 @@ int tc_fwd_launches(const Problem& p) { return (p.num_chunks > 0 ? 1 : 0) + 1; }
 
 gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
     const Problem& p = plan.p;
-    gdn_status st = launch_wy_tc(p, (uint8_t*)ws, s);
-    if (st) return st;
+    // all host-side preparation first, so that the two launches follow each other directly
     TcArgs a;
     a.p = p;
     a.timg = (const uint8_t*)ws;
+    a.summ = (const float2*)(ws + wy_tc_summary_offset(p));
     const std::vector<int> nck = chunk_counts(p, plan.cu_host);
     const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count());
     a.L = sc.L;
@@ -718,7 +684,23 @@ gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
                              (int)kSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
-    gdn_fwd_tc_kernel<<<(unsigned)sc.ctas, kThreads, kSmemBytes, s>>>(mq, mk, mv, a);
+    const gdn_status st = launch_wy_tc(p, (uint8_t*)ws, s);
+    if (st) return st;
+    // Programmatic dependent launch: the fused kernel may start while the WY kernel drains; it
+    // sets up and loads S0 for exact segments, then waits (griddepcontrol.wait) for the WY
+    // kernel's outputs.  Only when the WY kernel is the previous launch in the stream, so that
+    // nothing earlier (for instance the producer of S0) can overlap.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sc.ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.num_chunks > 0 ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, gdn_fwd_tc_kernel, mq, mk, mv, a) != cudaSuccess) return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

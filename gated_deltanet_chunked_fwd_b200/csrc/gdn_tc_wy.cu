@@ -16,7 +16,8 @@
 // fast chunk: 128 threads and about 39 KB of shared memory per CTA, five CTAs per SM.  The
 // Gram block K K^T is formed with warp-level mma.sync (bf16 in, fp32 out): its fragments
 // stay in registers, where the gate scaling turns them into A without a TMEM round trip.
-// The inverse is the blocked fp32 solve of gdn_tc_common.cuh.
+// The inverse is blocked: the four 16 x 16 diagonal blocks by fp32 substitution, then three
+// merge levels on the tensor cores (warp mma.sync in tf32).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -35,11 +36,12 @@ constexpr int kWyThreads = 128;
 constexpr int kWyMinBlocks = 5;  // CTAs per SM the shared memory and registers are sized for
 // shared memory (bytes from a 128-aligned base)
 constexpr uint32_t wK = 0;                                 // 16 KB bf16 K [dk half][64 rows][128 B];
-                                                           // then fp32 A [64][64] (as_idx layout)
-constexpr uint32_t wM = 16384;                             // fp32 [64][kLd] T
-constexpr uint32_t wYs = wM + 64 * kLd * 4;                // fp32 [3][16][kLdY] solve scratch
-constexpr uint32_t wVec = wYs + 3 * 16 * kLdY * 4;         // beta, gamma, a, b: 4 x 64 fp32
-constexpr uint32_t wSmemBytes = wVec + 4 * 64 * 4 + 128;   // + alignment slack
+                                                           // then fp32 A [64][kLd]
+constexpr uint32_t wM = 64 * kLd * 4;                      // fp32 [64][kLd] T
+constexpr uint32_t wYs = wM + 64 * kLd * 4;                // fp32 [4 warps][16][9] merge scratch
+constexpr uint32_t wVec = wYs + 3 * 16 * kLdY * 4;         // beta, gamma, a, b, |k|^2: 5 x 64 fp32
+constexpr uint32_t wSmemBytes = wVec + 5 * 64 * 4 + 128;   // + alignment slack
+static_assert(4 * 16 * 9 * 4 <= 3 * 16 * kLdY * 4, "merge scratch fits");
 static_assert(wSmemBytes * kWyMinBlocks + kWyMinBlocks * 1024 <= 228 * 1024, "five CTAs per SM");
 
 // 4 8x8 b16 matrices from shared memory (lane groups of 8 give the row addresses of matrix 0..3)
@@ -56,6 +58,101 @@ __device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t 
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// fp32 -> tf32 (round to nearest, ties away), as the 32-bit pattern mma.sync reads
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D += A B for one 16 x 8 x 8 tile in tf32 (A row-major, B column-major, D fp32)
+__device__ __forceinline__ void mma_tf32(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D += A B with fp32 operands rounded to tf32.  In the merges below this adds a relative error
+// of about 1e-6 (|T - T_exact| / |T| over random chunks of the workloads' distributions), some
+// thirty times below the bf16 rounding that the T image gets afterwards.
+__device__ __forceinline__ void mma_tf32_rn(float* d, const float* a, const float* b) {
+    const uint32_t ar[4] = {to_tf32(a[0]), to_tf32(a[1]), to_tf32(a[2]), to_tf32(a[3])};
+    const uint32_t br[2] = {to_tf32(b[0]), to_tf32(b[1])};
+    mma_tf32(d, ar, br);
+}
+
+// The four 16 x 16 diagonal blocks of T (threads 0..63: block t / 16, column t % 16): unit
+// lower-triangular inverse by forward substitution, written with zeros above the diagonal.
+// A and T are [64][kLd] row-major, so every A element is read at a compile-time offset from
+// the block origin.
+__device__ __forceinline__ void diag_inverse(const float* As, float* M, int t) {
+    if (t < 64) {
+        const int b = t >> 4, cc = t & 15;
+        const float* a = As + 16 * b * (kLd + 1);
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+            for (int j = 0; j + 1 < r; j += 2) {
+                s0 -= a[r * kLd + j] * x[j];
+                s1 -= a[r * kLd + j + 1] * x[j + 1];
+            }
+            if (r & 1) s0 -= a[r * kLd + r - 1] * x[r - 1];
+            x[r] = (r < cc) ? 0.f : s0 + s1;
+        }
+        float* m = M + 16 * b * (kLd + 1) + cc;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) m[r * kLd] = x[r];
+    }
+}
+
+// Level D (1..3) of the blocked inverse on the tensor cores: for the blocks (i, j0 = i - D),
+//   Y = sum_{k = j0}^{i-1} A_ik T_k,j0,   T_i,j0 = -T_ii Y      (16 x 16 blocks)
+// A work unit is one 8-column half of one block (one m16n8 tile); warp w takes units w, w + 4.
+// Y goes from the accumulator layout to the B-operand layout through a per-warp 16 x 9 scratch.
+template <int D>
+__device__ __forceinline__ void merge_level(const float* As, float* M, float* ysw, int warp, int lane) {
+    constexpr int kUnits = 2 * (4 - D);
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int u = warp; u < kUnits; u += 4) {
+        const int i = D + (u >> 1), j0 = i - D, col = 16 * j0 + 8 * (u & 1);
+        const int r0 = 16 * i + g, r1 = r0 + 8;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kb = 0; kb < D; ++kb) {
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                const int kc = 16 * (j0 + kb) + 8 * ks;
+                const float a[4] = {As[r0 * kLd + kc + t], As[r1 * kLd + kc + t],
+                                    As[r0 * kLd + kc + t + 4], As[r1 * kLd + kc + t + 4]};
+                const float b[2] = {M[(kc + t) * kLd + col + g], M[(kc + t + 4) * kLd + col + g]};
+                mma_tf32_rn(y, a, b);
+            }
+        }
+        ysw[g * 9 + 2 * t] = y[0];
+        ysw[g * 9 + 2 * t + 1] = y[1];
+        ysw[(g + 8) * 9 + 2 * t] = y[2];
+        ysw[(g + 8) * 9 + 2 * t + 1] = y[3];
+        __syncwarp();
+        float r[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const int kc = 16 * i + 8 * ks;
+            const float a[4] = {M[r0 * kLd + kc + t], M[r1 * kLd + kc + t], M[r0 * kLd + kc + t + 4],
+                                M[r1 * kLd + kc + t + 4]};
+            const float b[2] = {ysw[(8 * ks + t) * 9 + g], ysw[(8 * ks + t + 4) * 9 + g]};
+            mma_tf32_rn(r, a, b);
+        }
+        __syncwarp();  // the scratch is rewritten by this warp's next unit
+        *reinterpret_cast<float2*>(M + r0 * kLd + col + 2 * t) = make_float2(-r[0], -r[1]);
+        *reinterpret_cast<float2*>(M + r1 * kLd + col + 2 * t) = make_float2(-r[2], -r[3]);
+    }
 }
 
 // Image slot x -> (sequence n, chunk c of it, its first token and length); false when the
@@ -84,9 +181,12 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
 }
 
 __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
-    gdn_wy_tc_kernel(const Problem p, uint8_t* __restrict__ timg) {
+    gdn_wy_tc_kernel(const Problem p, uint8_t* __restrict__ timg, float2* __restrict__ summ) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    // the forward's state-chain kernel may be scheduled as soon as every CTA of this grid has
+    // started (it waits for this grid's completion before reading the images)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y, hk = h / p.group, Hv = p.Hv;
     int n = 0, c = 0;
@@ -116,6 +216,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     float* vgam = vbeta + 64;
     float* va = vbeta + 128;
     float* vb = vbeta + 192;
+    float* vnrm = vbeta + 256;
     float gr = 0.f;
     if (tid < 64) {
         float x = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;
@@ -140,12 +241,22 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         vb[tid] = fac ? expf(gm - gr) : gr * LOG2E;
     }
 
-    // ---- K K^T, lower block triangle: warp w owns rows 16w..16w+15, column tiles 0..2w+1
+    // ---- K K^T, lower block triangle: 20 tiles of 16 rows (m-tile) x 8 columns (n-tile), five
+    // per warp.  m-tiles 0 and 3 (2 + 8 tiles) are shared by warps 0 and 1, m-tiles 1 and 2
+    // (4 + 6 tiles) by warps 2 and 3; a warp's tiles are one run of n-tiles in m-tile mA and
+    // possibly a second run in m-tile mB.
     const int g8 = lane >> 2, t4 = lane & 3;
-    const int ntiles = 2 * warp + 2;
-    float acc[8][4];
+    int mA, jA, nA, mB, jB;
+    switch (warp) {
+        case 0: mA = 0; jA = 0; nA = 2; mB = 3; jB = 0; break;   // (0: 0-1), (3: 0-2)
+        case 1: mA = 3; jA = 3; nA = 5; mB = 3; jB = 8; break;   // (3: 3-7)
+        case 2: mA = 1; jA = 0; nA = 4; mB = 2; jB = 0; break;   // (1: 0-3), (2: 0)
+        default: mA = 2; jA = 1; nA = 5; mB = 2; jB = 6; break;  // (2: 1-5)
+    }
+    const bool twoA = nA < 5;  // warp-uniform: a second m-tile run exists
+    float acc[5][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    for (int i = 0; i < 5; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     __syncthreads();  // K tile, vectors
     {
         const uint32_t sK = smem_u32(sm + wK);
@@ -153,59 +264,70 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         for (int kk = 0; kk < 8; kk += 2) {  // pairs of 16-wide k steps
             const uint32_t half = sK + (kk >> 2) * 8192;
             const int ch = 2 * (kk & 3);
-            uint32_t a0[4], a1[4];
-            const int arow = 16 * warp + (lane & 15);
-            ldsm_x4(a0, half + sw128_off(arow, ch + (lane >> 4)));
-            ldsm_x4(a1, half + sw128_off(arow, ch + 2 + (lane >> 4)));
+            uint32_t aA0[4], aA1[4], aB0[4], aB1[4];
+            ldsm_x4(aA0, half + sw128_off(16 * mA + (lane & 15), ch + (lane >> 4)));
+            ldsm_x4(aA1, half + sw128_off(16 * mA + (lane & 15), ch + 2 + (lane >> 4)));
+            if (twoA) {
+                ldsm_x4(aB0, half + sw128_off(16 * mB + (lane & 15), ch + (lane >> 4)));
+                ldsm_x4(aB1, half + sw128_off(16 * mB + (lane & 15), ch + 2 + (lane >> 4)));
+            }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (j < ntiles) {  // warp-uniform
-                    uint32_t b[4];
-                    ldsm_x4(b, half + sw128_off(8 * j + (lane & 7), ch + (lane >> 3)));
-                    mma_16816(acc[j], a0, b[0], b[1]);
-                    mma_16816(acc[j], a1, b[2], b[3]);
+            for (int i = 0; i < 5; ++i) {
+                const bool inA = i < nA;  // warp-uniform
+                const int j = inA ? jA + i : jB + (i - nA);
+                uint32_t b[4];
+                ldsm_x4(b, half + sw128_off(8 * j + (lane & 7), ch + (lane >> 3)));
+                if (inA) {
+                    mma_16816(acc[i], aA0, b[0], b[1]);
+                    mma_16816(acc[i], aA1, b[2], b[3]);
+                } else {
+                    mma_16816(acc[i], aB0, b[0], b[1]);
+                    mma_16816(acc[i], aB1, b[2], b[3]);
                 }
             }
         }
     }
     __syncthreads();  // every warp is done with the K tile: A overwrites it
 
-    // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> shared memory (fp32)
+    // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> shared memory (fp32); the diagonal of
+    // K K^T gives |k_r|^2 for the chunk summary
     float* As = (float*)(sm + wK);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j < ntiles) {
+    for (int i = 0; i < 5; ++i) {
+        const bool inA = i < nA;
+        const int m = inA ? mA : mB, j = inA ? jA + i : jB + (i - nA);
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int r = 16 * warp + g8 + 8 * hr, s = 8 * j + 2 * t4;
-                const float ar = va[r], br = vbeta[r];
-                float2 w;
-                const float e0 = fac ? ar * vb[s] : exp2f(ar - vb[s]);
-                const float e1 = fac ? ar * vb[s + 1] : exp2f(ar - vb[s + 1]);
-                w.x = (s < r && r < lc) ? br * acc[j][2 * hr] * e0 : 0.f;
-                w.y = (s + 1 < r && r < lc) ? br * acc[j][2 * hr + 1] * e1 : 0.f;
-                *reinterpret_cast<float2*>(As + as_idx(r, s)) = w;
-            }
+        for (int hr = 0; hr < 2; ++hr) {
+            const int r = 16 * m + g8 + 8 * hr, s = 8 * j + 2 * t4;
+            const float ar = va[r], br = vbeta[r];
+            const float2 b2 = *reinterpret_cast<const float2*>(vb + s);
+            const float e0 = fac ? ar * b2.x : exp2f(ar - b2.x);
+            const float e1 = fac ? ar * b2.y : exp2f(ar - b2.y);
+            float2 w;
+            w.x = (s < r && r < lc) ? br * acc[i][2 * hr] * e0 : 0.f;
+            w.y = (s + 1 < r && r < lc) ? br * acc[i][2 * hr + 1] * e1 : 0.f;
+            *reinterpret_cast<float2*>(As + r * kLd + s) = w;
+            if (s == r) vnrm[r] = acc[i][2 * hr];
+            if (s + 1 == r) vnrm[r] = acc[i][2 * hr + 1];
         }
     }
-    __syncthreads();
+    // Chunk summary for the forward's gate-driven split: the summed log decay of the chunk and
+    // whether some token breaks 0 <= beta |k|^2 <= 2 (the condition under which each token's
+    // state map has norm <= exp(g)).
+    const bool viol = __syncthreads_or(tid < lc && !(vbeta[tid] >= 0.f && vbeta[tid] * vnrm[tid] <= 2.f));
+    if (tid == 63) summ[img_slot(bos, n, c) * Hv + h] = make_float2(gr, viol ? 1.f : 0.f);
 
     // ---- T = (I + A)^-1: diagonal 16 x 16 blocks, then three merge levels
     float* M = (float*)(sm + wM);
     float* Ys = (float*)(sm + wYs);
-    solve_diag(As, M, tid);
+    diag_inverse(As, M, tid);
     __syncthreads();
-    solve_level_Y<1, kWyThreads>(As, M, Ys, tid);
+    float* ysw = Ys + warp * 16 * 9;
+    merge_level<1>(As, M, ysw, warp, lane);
     __syncthreads();
-    solve_level_T<1, kWyThreads>(M, Ys, tid);
+    merge_level<2>(As, M, ysw, warp, lane);
     __syncthreads();
-    solve_level_Y<2, kWyThreads>(As, M, Ys, tid);
-    __syncthreads();
-    solve_level_T<2, kWyThreads>(M, Ys, tid);
-    __syncthreads();
-    solve_level_Y<3, kWyThreads>(As, M, Ys, tid);
-    __syncthreads();
-    solve_level_T<3, kWyThreads>(M, Ys, tid);
+    merge_level<3>(As, M, ysw, warp, lane);
     __syncthreads();
 
     // ---- bf16 image: thread = (row nr, half of the columns); zeros above the diagonal
@@ -227,7 +349,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
 
 }  // namespace
 
-gdn_status launch_wy_tc(const Problem& p, uint8_t* timg, cudaStream_t s) {
+gdn_status launch_wy_tc(const Problem& p, uint8_t* ws, cudaStream_t s) {
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
@@ -235,12 +357,14 @@ gdn_status launch_wy_tc(const Problem& p, uint8_t* timg, cudaStream_t s) {
                              (int)wSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     const dim3 grid((unsigned)slots, (unsigned)p.Hv);
-    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(p, timg);
+    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(p, ws, (float2*)(ws + wy_tc_summary_offset(p)));
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// workspace: the T images, then one float2 summary per (image slot, value head)
+size_t wy_tc_summary_offset(const Problem& p) { return (size_t)img_slots(p) * p.Hv * kTImgBytes; }
 size_t wy_tc_workspace(const Problem& p) {
-    return p.num_chunks > 0 ? (size_t)img_slots(p) * p.Hv * kTImgBytes : 0;
+    return p.num_chunks > 0 ? align_up(wy_tc_summary_offset(p), 256) + (size_t)img_slots(p) * p.Hv * 8 : 0;
 }
 
 }  // namespace gdn
