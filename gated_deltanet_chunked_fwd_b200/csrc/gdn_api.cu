@@ -139,10 +139,12 @@ gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan) {
     b.dS0 = a->dS0;
     const int64_t nc = p.num_chunks;
     plan->use_tc = !(a->flags & GDN_FLAG_PORTABLE) && tc_bwd_supported(p);
+    plan->cu_host = a->cu_seqlens ? a->cu_seqlens_host : nullptr;
+    plan->split_mode = (a->flags & GDN_FLAG_SPLIT_OFF) ? 1 : (a->flags & GDN_FLAG_SPLIT_FORCE) ? 2 : 0;
     if (plan->use_tc) {
         size_t o1, o2, o3, o4;
         plan->total = align_up(tc_bwd_workspace(p, &o1, &o2, &o3, &o4), kAlign);
-        plan->launches = p.T_total > 0 ? 2 : 1;
+        plan->launches = tc_bwd_launches(p);
         return GDN_OK;
     }
     size_t off = 0;

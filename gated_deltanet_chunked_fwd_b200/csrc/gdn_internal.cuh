@@ -89,12 +89,18 @@ size_t tc_fwd_workspace(const Problem& p);
 gdn_status launch_wy_tc(const Problem& p, uint8_t* ws, cudaStream_t s);
 size_t wy_tc_workspace(const Problem& p);
 size_t wy_tc_summary_offset(const Problem& p);
+// WY + fused kernel in replay mode: bf16 H^T entry-state image (32 KB) of every chunk, by
+// (image slot, value head), into himg; `ws` holds the WY outputs (wy_tc_workspace bytes)
+gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, char* ws, uint8_t* himg,
+                            cudaStream_t s);
 int tc_fwd_launches(const Problem& p);
 bool tc_fwd_supported(const Problem& p);
 
 struct BwdPlan {
     BwdProblem b;
     bool use_tc;  // tensor-core backward
+    const int32_t* cu_host;  // host copy of cu_seqlens (or nullptr)
+    int split_mode;          // 0 auto, 1 off, 2 force
     size_t off_table, off_W, off_U, off_gam, off_Hc, off_dHc, off_dU, off_dqw, off_dkw, total;
     int launches;
 };
@@ -104,6 +110,7 @@ gdn_status launch_bwd_reduce(const BwdProblem& b, const float* dqw, const float*
 bool tc_bwd_supported(const Problem& p);
 size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, size_t* off_dqw,
                         size_t* off_dkw);
+int tc_bwd_launches(const Problem& p);
 gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s);
 
 // shared SIMT pieces (also used by the backward's forward recompute)

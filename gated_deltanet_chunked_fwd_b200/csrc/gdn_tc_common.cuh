@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
+#include <vector>
 
 #include "gdn_internal.cuh"
 #include "gdn_sm100.cuh"
@@ -170,6 +172,60 @@ __device__ __forceinline__ void solve_diag(const float* As, float* M, int t) {
 }
 
 // ------------------------------------------------------------------- host side
+// Multi-SM split of the chunk chains (host side): chunks per sequence, and the segment length L
+// that minimises the estimated makespan (waves of CTAs x chunk steps per CTA, a warm-up chunk
+// counted as 1.5 steps).  split_mode: 0 auto, 1 off (one segment per sequence), 2 force (L = 2).
+inline int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// Segments of L chunks: count and estimated makespan in chunk-steps.
+struct SplitChoice {
+    int L;
+    int64_t ctas;
+};
+
+inline SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int split_mode, int nsm) {
+    int maxc = 1;
+    for (int c : nchunks) maxc = std::max(maxc, c);
+    auto count = [&](int L) {
+        int64_t s = 0;
+        for (int c : nchunks) s += std::max(1, (c + L - 1) / L);
+        return s * Hv;
+    };
+    if (split_mode == 1) return {maxc, count(maxc)};
+    if (split_mode == 2) {
+        const int L = std::max(1, std::min(maxc, 2));
+        return {L, count(L)};
+    }
+    int bestL = maxc;
+    double best = 1e300;
+    for (int L = 1; L <= maxc; ++L) {
+        const int64_t S = count(L);
+        const double waves = std::ceil((double)S / nsm);
+        const double est = waves * (L + (L < maxc ? 1.5 : 0.0));
+        if (est < best - 1e-9 || (std::fabs(est - best) < 1e-9 && L > bestL)) {
+            best = est;
+            bestL = L;
+        }
+    }
+    return {bestL, count(bestL)};
+}
+
+inline std::vector<int> chunk_counts(const Problem& p, const int32_t* cu_host) {
+    std::vector<int> v;
+    if (!p.cu) {
+        v.assign(p.N, (p.T + kChunk - 1) / kChunk);
+    } else {
+        v.resize(p.N);
+        for (int n = 0; n < p.N; ++n) v[n] = (cu_host[n + 1] - cu_host[n] + kChunk - 1) / kChunk;
+    }
+    return v;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,

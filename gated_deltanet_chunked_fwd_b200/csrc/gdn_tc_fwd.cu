@@ -93,6 +93,8 @@ struct TcArgs {
     float log_eps;  // warm-up stops once the summed log decay is <= log_eps
     const uint8_t* timg;  // T images of the WY step, by (image slot, value head)
     const float2* summ;   // per (image slot, value head): summed log decay, norm-condition flag
+    uint8_t* himg;        // replay mode (backward): bf16 H^T entry-state image per own chunk, by
+                          // (image slot, value head); no outputs.  nullptr: the forward
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < nk; ++k) {
             const int c = cstart + k;
             const int stage = k & 1;
-            const bool emit = c >= c0;
+            const bool emit = c >= c0 && !args.himg;
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t sV = sbase + kStageV + stage * 16384;
@@ -473,8 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < nk && ok; ++k) {
             const int c = cstart + k;
             const int stage = k & 1;
-            const bool emit = c >= c0;
-            const bool emit_prev = k > 0 && (c - 1) >= c0;
+            const bool emit = c >= c0 && !args.himg;
+            const bool emit_prev = k > 0 && (c - 1) >= c0 && !args.himg;
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t colR2 = kColR2 + 64 * stage;
 
@@ -502,6 +504,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(bar_mma_s);
             }
             if (emit_prev) epilogue(k - 1);  // overlaps MMA_HW of this chunk
+            if (args.himg && c >= c0) {
+                // replay mode: the chunk's entry state, as the bf16 H^T image [dk half][128 dv
+                // rows][128 B] (128-byte swizzled) that the backward loads; the bf16 copy in TMEM
+                // holds it (dk pairs per column)
+                uint8_t* img = args.himg + (img_slot(bos, n, c) * Hv + h) * (int64_t)32768;
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    float w[32];
+                    tmem_ld32(tl + kColHb + 32 * a, w);
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc)
+                        *reinterpret_cast<uint4*>(img + a * 16384 + sw128_off(m, cc)) =
+                            make_uint4(__float_as_uint(w[4 * cc]), __float_as_uint(w[4 * cc + 1]),
+                                       __float_as_uint(w[4 * cc + 2]), __float_as_uint(w[4 * cc + 3]));
+                }
+            }
             ok = wg_and(2, kThreadsS, mbar_wait(bar_mma_s, ph));
             ph ^= 1;
             if (!ok) break;
@@ -578,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             wg_sync(2, kThreadsS);
             if (m == 0) mbar_arrive(&bar_s_done[stage]);
         }
-        if (ok && nk > 0 && cstart + nk - 1 >= c0) epilogue(nk - 1);
+        if (ok && nk > 0 && cstart + nk - 1 >= c0 && !args.himg) epilogue(nk - 1);
         if (ok && p.ST && seg == segs_n - 1) {
             // final state S_T = H (stored [dk][dv]): thread m writes column m
             float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + m;
@@ -602,57 +620,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------- host side
-int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
-// Segments of L chunks: count and estimated makespan in chunk-steps.
-struct SplitChoice {
-    int L;
-    int64_t ctas;
-};
-
-SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int split_mode, int nsm) {
-    int maxc = 1;
-    for (int c : nchunks) maxc = std::max(maxc, c);
-    auto count = [&](int L) {
-        int64_t s = 0;
-        for (int c : nchunks) s += std::max(1, (c + L - 1) / L);
-        return s * Hv;
-    };
-    if (split_mode == 1) return {maxc, count(maxc)};
-    if (split_mode == 2) {
-        const int L = std::max(1, std::min(maxc, 2));
-        return {L, count(L)};
-    }
-    int bestL = maxc;
-    double best = 1e300;
-    for (int L = 1; L <= maxc; ++L) {
-        const int64_t S = count(L);
-        const double waves = std::ceil((double)S / nsm);
-        const double est = waves * (L + (L < maxc ? 1.5 : 0.0));
-        if (est < best - 1e-9 || (std::fabs(est - best) < 1e-9 && L > bestL)) {
-            best = est;
-            bestL = L;
-        }
-    }
-    return {bestL, count(bestL)};
-}
-
-std::vector<int> chunk_counts(const Problem& p, const int32_t* cu_host) {
-    std::vector<int> v;
-    if (!p.cu) {
-        v.assign(p.N, (p.T + kChunk - 1) / kChunk);
-    } else {
-        v.resize(p.N);
-        for (int n = 0; n < p.N; ++n) v[n] = (cu_host[n + 1] - cu_host[n] + kChunk - 1) / kChunk;
-    }
-    return v;
-}
-
 }  // namespace
 
 bool tc_fwd_supported(const Problem& p) {
@@ -663,18 +630,20 @@ bool tc_fwd_supported(const Problem& p) {
 size_t tc_fwd_workspace(const Problem& p) { return wy_tc_workspace(p); }
 int tc_fwd_launches(const Problem& p) { return (p.num_chunks > 0 ? 1 : 0) + 1; }
 
-gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
-    const Problem& p = plan.p;
+// The WY kernel, then the fused kernel (forward, or replay of the states when himg != nullptr)
+gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int split_mode, char* ws,
+                              uint8_t* himg, cudaStream_t s) {
     // all host-side preparation first, so that the two launches follow each other directly
     TcArgs a;
     a.p = p;
     a.timg = (const uint8_t*)ws;
     a.summ = (const float2*)(ws + wy_tc_summary_offset(p));
-    const std::vector<int> nck = chunk_counts(p, plan.cu_host);
-    const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count());
+    a.himg = himg;
+    const std::vector<int> nck = chunk_counts(p, cu_host);
+    const SplitChoice sc = choose_split(nck, p.Hv, split_mode, sm_count());
     a.L = sc.L;
     a.fixed_segs = p.cu ? 0 : std::max(1, (nck.empty() ? 1 : (nck[0] + sc.L - 1) / sc.L));
-    a.auto_warm = plan.split_mode == 1 ? 0 : 1;
+    a.auto_warm = split_mode == 1 ? 0 : 1;
     a.log_eps = (float)(-30.0 * std::log(2.0));
     CUtensorMap mq, mk, mv;
     const int64_t Tt = std::max<int64_t>(p.T_total, 1);
@@ -702,6 +671,18 @@ gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
     cfg.numAttrs = p.num_chunks > 0 ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, gdn_fwd_tc_kernel, mq, mk, mv, a) != cudaSuccess) return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
+    return launch_fwd_tc_impl(plan.p, plan.cu_host, plan.split_mode, ws, nullptr, s);
+}
+
+gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, char* ws, uint8_t* himg,
+                            cudaStream_t s) {
+    Problem q = p;  // states only: no o, no S_T
+    q.o = nullptr;
+    q.ST = nullptr;
+    return launch_fwd_tc_impl(q, cu_host, 0, ws, himg, s);
 }
 
 }  // namespace gdn

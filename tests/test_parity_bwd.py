@@ -6,7 +6,8 @@ import pytest
 import torch
 
 import oracle
-from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_PORTABLE, gdn_chunk_bwd
+from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE,
+                                             GDN_FLAG_SPLIT_OFF, gdn_chunk_bwd)
 from gated_deltanet_chunked_fwd_b200.inputs import make_inputs, make_workload
 from tests._helpers import TOL, cpu, rel_l2
 
@@ -103,3 +104,20 @@ def test_tensor_core_and_portable_backward_agree():
     compare(a, r, TOL[inp["q"].dtype], "tensor-core")
     compare(b, r, TOL[inp["q"].dtype], "portable")
     compare(a, [t.double().cpu() for t in b], TOL[inp["q"].dtype], "tc vs portable")
+
+
+@pytest.mark.parametrize("flags", [GDN_FLAG_SPLIT_OFF, GDN_FLAG_SPLIT_FORCE], ids=["split-off", "split-force"])
+def test_tensor_core_split_modes(flags):
+    """The tensor-core backward with one segment per sequence (no warm-ups) and with
+    two-chunk segments (reverse warm-ups at every segment end), ragged varlen, GQA 2:4."""
+    inp = make_inputs(1, 0, 2, 4, 128, 128, dtype="bf16", seed=13, s0_std=0.2, backward=True,
+                      lengths=[3, 64, 0, 300, 1, 200], device=DEV)
+    compare(run(inp, flags), ref(inp), TOL[inp["q"].dtype], f"flags={flags}")
+
+
+def test_tensor_core_slow_decay_exact_fallback():
+    """Slow decay (g = -softplus(N(-6, 1)), |sum g| over a chunk ~ 0.16): reverse warm-ups never
+    reach the 2^-30 bound, so every segment runs from dS_T at the sequence end."""
+    inp = make_inputs(2, 700, 1, 2, 128, 128, dtype="bf16", seed=14, s0_std=0.1, g_mu=-6.0,
+                      backward=True, device=DEV)
+    compare(run(inp), ref(inp), TOL[inp["q"].dtype], "slow decay")
