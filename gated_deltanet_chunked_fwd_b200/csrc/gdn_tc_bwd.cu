@@ -6,7 +6,8 @@
 // kernel in replay mode (the bf16 entry state H^T of every chunk, as a ready-to-use
 // 128-byte-swizzled shared-memory image), this reverse kernel, and the reduction of dq / dk over
 // grouped value heads.  The reverse kernel runs one CTA per (sequence, value head, segment of
-// chunks), 128 threads (thread i <-> TMEM lane i <-> MMA row i).  A segment walks its chunks
+// chunks), 256 threads: the two warps of each TMEM lane quarter share its lanes (thread <-> MMA
+// row) and split each row's columns, or tokens, in halves.  A segment walks its chunks
 // backwards with the state adjoint dH (fp32, TMEM).  Its exit adjoint comes from a reverse
 // warm-up: the adjoint map of a chunk, dH -> (Gam_n I - W^T Kd) dH, is the transpose of the
 // chunk's state map and has the same norm bound exp(sum g) while 0 <= beta |k|^2 <= 2, so a
@@ -45,7 +46,7 @@ using namespace tc;
 
 namespace {
 
-constexpr int kNT = 128;
+constexpr int kNT = 256;
 constexpr int kTmemColsB = 512;
 // TMEM columns (lane = MMA row)
 constexpr uint32_t cH = 0;     // dH^T fp32                                      [0, 128)
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kNT, 1)
     float* va = vbeta + 256;
     float* vb = vbeta + 320;
     float* vgam = vbeta + 384;
-    float* red = (float*)(sm + bRed);        // [4][64]
+    float* red = (float*)(sm + bRed);        // [8 warps][32] partial sums
     float* acc_g = red + 256;                // dgamma accumulator [64]
     float* acc_b = red + 320;                // dbeta accumulator [64]
     float* acc_s = red + 384;                // scalars
@@ -220,9 +221,12 @@ __global__ void __launch_bounds__(kNT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lane quarter
     const uint32_t sb = smem_u32(sm);
-    const int m = tid;  // TMEM lane / head-dimension index owned by this thread
+    // thread <-> TMEM lane m (an MMA row: a head-dimension index); the two warps of a lane
+    // quarter split each row's columns (or tokens) in halves, hh = 0 / 1
+    const int m = ((warp & 3) << 5) | lane;
+    const int hh = warp >> 2;
     uint32_t ph_ld = 0, ph_mma = 0;
     bool ok = true;
 
@@ -310,11 +314,8 @@ __global__ void __launch_bounds__(kNT, 1)
         const float* dst = b.dST ? b.dST + ((int64_t)n * Hv + h) * dk * dv : nullptr;
         float v[64];
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) v[e] = (dst && exact_end) ? dst[(int64_t)(64 * a + e) * dv + m] : 0.f;
-            tmem_st64(tl + cH + 64 * a, v);
-        }
+        for (int e = 0; e < 64; ++e) v[e] = (dst && exact_end) ? dst[(int64_t)(64 * hh + e) * dv + m] : 0.f;
+        tmem_st64(tl + cH + 64 * hh, v);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -327,16 +328,13 @@ __global__ void __launch_bounds__(kNT, 1)
         {
             float v[64];
             uint32_t w[32];
+            tmem_ld64(tl + cH + 64 * hh, v);
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                tmem_ld64(tl + cH + 64 * a, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-                tmem_st32u(tl + cHb + 32 * a, w);
-                if (emit) {
-                    store_row32(sm + bDHt + a * 16384, m, 0, v);
-                    store_row32(sm + bDHt + a * 16384, m, 4, v + 32);
-                }
+            for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+            tmem_st32u(tl + cHb + 32 * hh, w);
+            if (emit) {
+                store_row32(sm + bDHt + hh * 16384, m, 0, v);
+                store_row32(sm + bDHt + hh * 16384, m, 4, v + 32);
             }
         }
         if (tid < 64) {
@@ -355,27 +353,31 @@ __global__ void __launch_bounds__(kNT, 1)
         mma1();
         if (!(ok = mma_sync_wait())) break;
         // P (rows 0..63) -> smem; Bw, Bu from the T image
-        if (tid < 64) {
-            const int r = tid;
-            float v[64];
-            tmem_ld64(tl + cR1, v);
-#pragma unroll
-            for (int s = 0; s < 64; ++s) v[s] = (s <= r && r < lc) ? v[s] * Efac(fac, r, s) : 0.f;
-            store_row32(sm + bP, r, 0, v);
-            store_row32(sm + bP, r, 4, v + 32);
-        }
-        {
-            const int nrow = tid >> 1, hf = tid & 1;
-            float vw[32], vu[32];
+        if (m < 64) {  // P row m, this thread's half of the columns
+            const int r = m;
+            float v[32];
+            tmem_ld32(tl + cR1 + 32 * hh, v);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const int s = 32 * hf + e;
+                const int s = 32 * hh + e;
+                v[e] = (s <= r && r < lc) ? v[e] * Efac(fac, r, s) : 0.f;
+            }
+            store_row32(sm + bP, r, 4 * hh, v);
+        }
+        {  // row nrow, columns [16 q, 16 q + 16)
+            const int nrow = tid >> 2, q = tid & 3;
+            float vw[16], vu[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int s = 16 * q + e;
                 const float t = bf(sm + bT, nrow, s);
                 vw[e] = t * vbG[s];
                 vu[e] = t * vbeta[s];
             }
-            store_row32(sm + bBw, nrow, 4 * hf, vw);
-            store_row32(sm + bBu, nrow, 4 * hf, vu);
+            *reinterpret_cast<uint4*>(sm + bBw + sw128_off(nrow, 2 * q)) = pack8(vw);
+            *reinterpret_cast<uint4*>(sm + bBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
+            *reinterpret_cast<uint4*>(sm + bBu + sw128_off(nrow, 2 * q)) = pack8(vu);
+            *reinterpret_cast<uint4*>(sm + bBu + sw128_off(nrow, 2 * q + 1)) = pack8(vu + 8);
         }
         fence_proxy_async();
         tc_fence_before();
@@ -404,20 +406,19 @@ __global__ void __launch_bounds__(kNT, 1)
         {  // -W^T -> Wt;  Q rows * Gam -> Qg (over Bw/Bu);  dU^T -> bf16 (R5 cols 0..31);
            // <dH_c, H_c>, then dH^T <- Gam_n dH^T
             float v[64];
-            tmem_ld64(tl + cR2, v);
+            tmem_ld32(tl + cR2 + 32 * hh, v);
 #pragma unroll
-            for (int e = 0; e < 64; ++e) v[e] = -v[e];
-            store_row32(sm + bWt, m, 0, v);
-            store_row32(sm + bWt, m, 4, v + 32);
+            for (int e = 0; e < 32; ++e) v[e] = -v[e];
+            store_row32(sm + bWt, m, 4 * hh, v);
             {
                 // rows past the sequence end hold the next sequence's q and dO: zero them here
-                const int r = m >> 1, a = m & 1;
+                const int r = tid >> 2, a = (tid >> 1) & 1, part = tid & 1;
                 const float gmul = r < lc ? vGam[r] : 0.f;
                 const uint4* src = reinterpret_cast<const uint4*>(sm + bQK + a * 16384 + r * 128);
                 uint4* dst = reinterpret_cast<uint4*>(sm + bBw + a * 8192 + r * 128);
 #pragma unroll
-                for (int i8 = 0; i8 < 8; ++i8) {
-                    const int c8 = (i8 + r) & 7;
+                for (int i4 = 0; i4 < 4; ++i4) {
+                    const int c8 = (4 * part + i4 + r) & 7;
                     uint4 u = src[c8];
                     __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
@@ -428,25 +429,28 @@ __global__ void __launch_bounds__(kNT, 1)
                     dst[c8] = u;  // same swizzle position: row r keeps its chunk permutation
                 }
             }
-            float w64[64];
-            tmem_ld64x2(tl + cR4, v, tl + cR5, w64);
-            uint32_t w[32];
+            {  // dU^T = dO^T P + (dH^T K^T) diag(dec) -> bf16 pairs in R5 columns 0..31; the other
+               // half reads fp32 columns this half overwrites, hence the barrier
+                float w32[32];
+                tmem_ld32x2(tl + cR4 + 32 * hh, v, tl + cR5 + 32 * hh, w32);
+                uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                w[e] = pack_bf16(v[2 * e] + vdec[2 * e] * w64[2 * e], v[2 * e + 1] + vdec[2 * e + 1] * w64[2 * e + 1]);
-            tmem_st32u(tl + cR5, w);
+                for (int e = 0; e < 16; ++e) {
+                    const int s = 32 * hh + 2 * e;
+                    w[e] = pack_bf16(v[2 * e] + vdec[s] * w32[2 * e], v[2 * e + 1] + vdec[s + 1] * w32[2 * e + 1]);
+                }
+                __syncthreads();
+                tmem_st16u(tl + cR5 + 16 * hh, w);
+            }
             float dhh = 0.f;
             const float Gn = vGam[63];
+            tmem_ld64(tl + cH + 64 * hh, v);
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                tmem_ld64(tl + cH + 64 * a, v);
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    if (emit) dhh += v[e] * bf(sm + bHt + a * 16384, m, e);
-                    v[e] *= Gn;
-                }
-                tmem_st64(tl + cH + 64 * a, v);
+            for (int e = 0; e < 64; ++e) {
+                if (emit) dhh += v[e] * bf(sm + bHt + hh * 16384, m, e);
+                v[e] *= Gn;
             }
+            tmem_st64(tl + cH + 64 * hh, v);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) dhh += __shfl_xor_sync(0xffffffffu, dhh, o);
             if (lane == 0) atomicAdd(&acc_s[0], dhh);
@@ -480,33 +484,35 @@ __global__ void __launch_bounds__(kNT, 1)
         if (!(ok = mma_sync_wait())) break;
         if (emit) {  // the chunk's gradients (own chunks only)
             {  // U^T -> Ut;  TdU: dv out, rows 64..127 of the dO tile, -TdU^T -> Wt, dbeta part
-                float v[64];
-                tmem_ld64(tl + cR3, v);
-                store_row32(sm + bUt, m, 0, v);
-                store_row32(sm + bUt, m, 4, v + 32);
-                tmem_ld64(tl + cR2, v);
+                // this thread: row m of U^T and of TdU^T, tokens r in [32 hh, 32 hh + 32)
+                float v[32];
+                tmem_ld32(tl + cR3 + 32 * hh, v);
+                store_row32(sm + bUt, m, 4 * hh, v);
+                tmem_ld32(tl + cR2 + 32 * hh, v);
                 __nv_bfloat16* dvp = (__nv_bfloat16*)b.dv + (t0 * Hv + h) * dv + m;
-                float bvals[64];
+                float bvals[32];
     #pragma unroll
-                for (int r = 0; r < 64; ++r) {
-                    if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn(vbeta[r] * v[r]);
-                    bvals[r] = v[r] * bf(sm + bV + (m >> 6) * 8192, r, m & 63);  // TdU[r][m] v[r][m]
+                for (int e = 0; e < 32; ++e) {
+                    const int r = 32 * hh + e;
+                    if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn(vbeta[r] * v[e]);
+                    bvals[e] = v[e] * bf(sm + bV + (m >> 6) * 8192, r, m & 63);  // TdU[r][m] v[r][m]
                     // TdU row r of the stacked [dO ; TdU] tile: element (64 + r, m)
                     *reinterpret_cast<__nv_bfloat16*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
-                                                      (m & 7) * 2) = __float2bfloat16_rn(v[r]);
+                                                      (m & 7) * 2) = __float2bfloat16_rn(v[e]);
                 }
     #pragma unroll
-                for (int e = 0; e < 64; ++e) v[e] = -v[e];
-                store_row32(sm + bWt, m, 0, v);
-                store_row32(sm + bWt, m, 4, v + 32);
-                warp_reduce_scatter<64>(bvals, lane);
-                red[warp * 64 + 2 * lane] = bvals[0];
-                red[warp * 64 + 2 * lane + 1] = bvals[1];
+                for (int e = 0; e < 32; ++e) v[e] = -v[e];
+                store_row32(sm + bWt, m, 4 * hh, v);
+                warp_reduce_scatter<32>(bvals, lane);  // lane l: token 32 hh + l, summed over this warp's m
+                red[warp * 32 + lane] = bvals[0];
             }
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
-            if (tid < 64) acc_b[tid] += red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
+            if (tid < 64) {
+                const int q4 = (tid >> 5) * 4, l = tid & 31;
+                acc_b[tid] += red[q4 * 32 + l] + red[(q4 + 1) * 32 + l] + red[(q4 + 2) * 32 + l] + red[(q4 + 3) * 32 + l];
+            }
             if (tid == 0) {
                 tc_fence_after();
     #pragma unroll
@@ -531,66 +537,71 @@ __global__ void __launch_bounds__(kNT, 1)
                                 desc_sw128(sb + bUt + j * 2048, 8192, 1024), id_mm64, j > 0);
             }
             if (!(ok = mma_sync_wait())) break;
-            {  // dP (lanes 0..63) and dA (lanes 64..127) rows: dgamma / dbeta terms, dP o E, G
-                const int r = tid & 63;
-                float d[64], x[64];
-                tmem_ld64x2(tl + cR3, d, tl + cR1, x);
+            {  // dP (lanes 0..63) and dA (lanes 64..127) rows, columns s in [32 hh, 32 hh + 32):
+               // dgamma / dbeta terms, dP o E, G
+                const int r = m & 63;
+                float d[32], x[32];
+                tmem_ld32x2(tl + cR3 + 32 * hh, d, tl + cR1 + 32 * hh, x);
                 float rowsum = 0.f, bsum = 0.f;
-                if (tid < 64) {
+                if (m < 64) {
     #pragma unroll
-                    for (int s = 0; s < 64; ++s) {
+                    for (int e = 0; e < 32; ++e) {
+                        const int s = 32 * hh + e;
                         const bool in = (s <= r && r < lc);
                         const float E = Efac(fac, r, s);
-                        const float P = in ? x[s] * E : 0.f;
-                        const float dP = in ? d[s] : 0.f;
+                        const float P = in ? x[e] * E : 0.f;
+                        const float dP = in ? d[e] : 0.f;
                         rowsum += dP * P;
-                        x[s] = dP * P;      // column-sum term
-                        d[s] = dP * E;      // dP o E
+                        x[e] = dP * P;      // column-sum term
+                        d[e] = dP * E;      // dP o E
                     }
-                    store_row32(sm + bP, r, 0, d);
-                    store_row32(sm + bP, r, 4, d + 32);
+                    store_row32(sm + bP, r, 4 * hh, d);
                 } else {
                     float* G = (float*)(sm + bV);
                     const float br = vbeta[r];
     #pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
+                    for (int c4 = 0; c4 < 8; ++c4) {
                         float4 gw;
                         float* gp = &gw.x;
     #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s = 4 * c4 + e;
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const int e = 4 * c4 + e4, s = 32 * hh + e;
                             const bool in = (s < r && r < lc);
                             const float E = Efac(fac, r, s);
-                            const float dA = in ? -d[s] : 0.f;
-                            const float KE = x[s] * E;
+                            const float dA = in ? -d[e] : 0.f;
+                            const float KE = x[e] * E;
                             const float A = br * KE;
                             rowsum += dA * A;
                             bsum += dA * KE;
-                            x[s] = dA * A;
-                            gp[e] = dA * E * br;
+                            x[e] = dA * A;
+                            gp[e4] = dA * E * br;
                         }
-                        *reinterpret_cast<float4*>(G + as_idx(r, 4 * c4)) = gw;
+                        *reinterpret_cast<float4*>(G + as_idx(r, 32 * hh + 4 * c4)) = gw;
                     }
                 }
-                warp_reduce_scatter<64>(x, lane);
-                red[warp * 64 + 2 * lane] = x[0];
-                red[warp * 64 + 2 * lane + 1] = x[1];
+                warp_reduce_scatter<32>(x, lane);  // lane l: column 32 hh + l, summed over this warp's rows
+                red[warp * 32 + lane] = x[0];
+                // dgamma_r += rowsum (own row) - colsum (all rows) for both dP o P and dA o A
+                atomicAdd(&acc_g[r], rowsum);
+                if (m >= 64) atomicAdd(&acc_b[r], bsum);
                 __syncthreads();
-                // dgamma_r += rowsum (own row)  -  colsum (all rows) for both dP o P and dA o A
-                if (tid < 64) acc_g[tid] += rowsum - (red[tid] + red[64 + tid]);
-                __syncthreads();
-                if (tid >= 64) acc_g[r] += rowsum - (red[128 + r] + red[192 + r]);
-                if (tid >= 64) acc_b[r] += bsum;
+                if (tid < 64) {
+                    const int q4 = (tid >> 5) * 4, l = tid & 31;
+                    acc_g[tid] -= red[q4 * 32 + l] + red[(q4 + 1) * 32 + l] + red[(q4 + 2) * 32 + l] +
+                                  red[(q4 + 3) * 32 + l];
+                }
             }
             __syncthreads();
-            if (tid < 64) {  // S = G + G^T, row s = tid
-                const int s = tid;
+            if (tid < 128) {  // S = G + G^T, row s = tid % 64, columns [32 (tid / 64), + 32)
+                const int s = tid & 63, hs = tid >> 6;
                 const float* G = (const float*)(sm + bV);
-                float v[64];
+                float v[32];
     #pragma unroll
-                for (int j = 0; j < 64; ++j) v[j] = G[as_idx(s, j)] + G[as_idx(j, s)];
-                store_row32(sm + bT, s, 0, v);
-                store_row32(sm + bT, s, 4, v + 32);
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = 32 * hs + jj;
+                    v[jj] = G[as_idx(s, j)] + G[as_idx(j, s)];
+                }
+                store_row32(sm + bT, s, 4 * hs, v);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -611,65 +622,83 @@ __global__ void __launch_bounds__(kNT, 1)
                                 desc_sw128(sb + bT + j * 32, 16, 1024), id_mk64, 1);
             }
             if (!(ok = mma_sync_wait())) break;
-            {  // epilogue: thread i = dk index
+            {  // epilogue: thread i = dk index (TMEM lane), tokens [32 hh, 32 hh + 32)
                 const int i = m;
-                float gv[64], bv[64];
+                float gv[32], bv[32];
                 float kdk = 0.f;
                 const uint8_t* qtile = sm + bQK + (i >> 6) * 16384;
+                // without grouped heads dq / dk go out directly (bf16); else per value head (fp32)
+                // for the reduction over the group
+                const bool direct = p.group == 1;
                 float* dqp = args.dqw + (t0 * Hv + h) * dk + i;
                 float* dkp = args.dkw + (t0 * Hv + h) * dk + i;
-    #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                __nv_bfloat16* dqb = (__nv_bfloat16*)b.dq + (t0 * Hv + h) * dk + i;
+                __nv_bfloat16* dkb = (__nv_bfloat16*)b.dk + (t0 * Hv + h) * dk + i;
+                {
                     float a32[32], b32[32];
-                    tmem_ld32x2(tl + cR4 + 32 * hf, a32, tl + cR3 + 32 * hf, b32);  // H dO^T, K^T dPE^T
+                    tmem_ld32x2(tl + cR4 + 32 * hh, a32, tl + cR3 + 32 * hh, b32);  // H dO^T, K^T dPE^T
     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int r = 32 * hf + e;
+                        const int r = 32 * hh + e;
                         const float qs = vGam[r] * a32[e];  // dQs^T[i][r]
-                        if (r < lc) dqp[(int64_t)r * Hv * dk] = qs + b32[e];
-                        gv[r] = bf(qtile, r, i & 63) * qs;
+                        if (r < lc) {
+                            if (direct) dqb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(qs + b32[e]);
+                            else dqp[(int64_t)r * Hv * dk] = qs + b32[e];
+                        }
+                        gv[e] = bf(qtile, r, i & 63) * qs;
                     }
                 }
-    #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                {
                     float a32[32], b32[32], c32[32];
-                    tmem_ld32x2(tl + cR1 + 32 * hf, a32, tl + cR2 + 32 * hf, b32);  // dk main, dKd^T
-                    tmem_ld32(tl + cR5 + 32 * hf, c32);                              // TdW^T
+                    tmem_ld32x2(tl + cR1 + 32 * hh, a32, tl + cR2 + 32 * hh, b32);  // dk main, dKd^T
+                    tmem_ld32(tl + cR5 + 32 * hh, c32);                              // TdW^T
     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int s = 32 * hf + e;
+                        const int s = 32 * hh + e;
                         const float kv = bf(qtile, 64 + s, i & 63);
                         const float dkv = a32[e] + vdec[s] * b32[e] + vbG[s] * c32[e];
-                        if (s < lc) dkp[(int64_t)s * Hv * dk] = dkv;
+                        if (s < lc) {
+                            if (direct) dkb[(int64_t)s * Hv * dk] = __float2bfloat16_rn(dkv);
+                            else dkp[(int64_t)s * Hv * dk] = dkv;
+                        }
                         const float kdterm = vdec[s] * kv * b32[e];
-                        gv[s] += vbG[s] * c32[e] * kv - kdterm;
-                        bv[s] = vGam[s] * c32[e] * kv;
+                        gv[e] += vbG[s] * c32[e] * kv - kdterm;
+                        bv[e] = vGam[s] * c32[e] * kv;
                         kdk += kdterm;
                     }
                 }
-                warp_reduce_scatter<64>(gv, lane);
-                warp_reduce_scatter<64>(bv, lane);
+                warp_reduce_scatter<32>(gv, lane);  // lane l: token 32 hh + l, summed over this warp's i
+                warp_reduce_scatter<32>(bv, lane);
     #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) kdk += __shfl_xor_sync(0xffffffffu, kdk, o);
-                red[warp * 64 + 2 * lane] = gv[0];
-                red[warp * 64 + 2 * lane + 1] = gv[1];
+                red[warp * 32 + lane] = gv[0];
                 if (lane == 0) atomicAdd(&acc_s[1], kdk);
                 __syncthreads();
-                if (tid < 64) acc_g[tid] += red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
+                const int q4 = (tid >> 5) * 4, l = tid & 31;
+                if (tid < 64)
+                    acc_g[tid] += red[q4 * 32 + l] + red[(q4 + 1) * 32 + l] + red[(q4 + 2) * 32 + l] +
+                                  red[(q4 + 3) * 32 + l];
                 __syncthreads();
-                red[warp * 64 + 2 * lane] = bv[0];
-                red[warp * 64 + 2 * lane + 1] = bv[1];
+                red[warp * 32 + lane] = bv[0];
                 __syncthreads();
-                if (tid < 64) acc_b[tid] += red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
+                if (tid < 64)
+                    acc_b[tid] += red[q4 * 32 + l] + red[(q4 + 1) * 32 + l] + red[(q4 + 2) * 32 + l] +
+                                  red[(q4 + 3) * 32 + l];
                 __syncthreads();
             }
-            if (tid == 0) {  // last-row terms, then dg = reverse in-chunk cumsum of dgamma
-                acc_g[lc - 1] += acc_s[1] + vGam[63] * acc_s[0];
-                float run = 0.f;
-                for (int r = lc - 1; r >= 0; --r) {
-                    run += acc_g[r];
-                    b.dg[(t0 + r) * Hv + h] = run;
+            if (warp == 0) {  // last-row terms, then dg = reverse in-chunk cumsum of dgamma
+                const float extra = acc_s[1] + vGam[63] * acc_s[0];
+                const int r0 = 2 * lane;  // this lane's rows r0, r0 + 1
+                const float x0 = r0 < lc ? acc_g[r0] + (r0 == lc - 1 ? extra : 0.f) : 0.f;
+                const float x1 = r0 + 1 < lc ? acc_g[r0 + 1] + (r0 + 1 == lc - 1 ? extra : 0.f) : 0.f;
+                float suf = x0 + x1;  // sum over the rows of lanes >= this one
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_down_sync(0xffffffffu, suf, o);
+                    if (lane + o < 32) suf += y;
                 }
+                if (r0 < lc) b.dg[(t0 + r0) * Hv + h] = suf;
+                if (r0 + 1 < lc) b.dg[(t0 + r0 + 1) * Hv + h] = suf - x0;
             }
             if (tid < lc) b.dbeta[(t0 + tid) * Hv + h] = acc_b[tid];
         }
@@ -680,12 +709,9 @@ __global__ void __launch_bounds__(kNT, 1)
     if (ok && b.dS0 && seg == 0) {
         float* dst = b.dS0 + ((int64_t)n * Hv + h) * dk * dv + m;
         float v[64];
+        tmem_ld64(tl + cH + 64 * hh, v);
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-            tmem_ld64(tl + cH + 64 * a, v);
-#pragma unroll
-            for (int e = 0; e < 64; ++e) dst[(int64_t)(64 * a + e) * dv] = v[e];
-        }
+        for (int e = 0; e < 64; ++e) dst[(int64_t)(64 * hh + e) * dv] = v[e];
     }
     if (!ok && tid == 0) report(p.status, GDN_ERR_TIMEOUT);
     tc_fence_before();
@@ -700,8 +726,8 @@ __global__ void __launch_bounds__(kNT, 1)
 
 bool tc_bwd_supported(const Problem& p) { return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128; }
 
-// workspace: the WY outputs (T images, gate summaries), the replayed H^T images, then fp32 dq
-// and dk per value head (summed over grouped heads by the reduction)
+// workspace: the WY outputs (T images, gate summaries), the replayed H^T images, then (with
+// grouped heads) fp32 dq and dk per value head, summed over each group by the reduction
 size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, size_t* off_dqw,
                         size_t* off_dkw) {
     size_t off = 0;
@@ -709,14 +735,15 @@ size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, si
     off = align_up(off + wy_tc_workspace(p), 256);
     *off_himg = off;
     off = align_up(off + (p.num_chunks > 0 ? (size_t)img_slots(p) * p.Hv * kHImg : 0), 256);
+    const size_t per = p.group > 1 ? sizeof(float) * (size_t)p.T_total * p.Hv * p.dk : 0;
     *off_dqw = off;
-    off = align_up(off + sizeof(float) * (size_t)p.T_total * p.Hv * p.dk, 256);
+    off = align_up(off + per, 256);
     *off_dkw = off;
-    off = align_up(off + sizeof(float) * (size_t)p.T_total * p.Hv * p.dk, 256);
+    off = align_up(off + per, 256);
     return off;
 }
 
-int tc_bwd_launches(const Problem& p) { return p.num_chunks > 0 ? 4 : 1; }
+int tc_bwd_launches(const Problem& p) { return p.num_chunks > 0 ? (p.group == 1 ? 3 : 4) : 1; }
 
 gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     const BwdProblem& bp = plan.b;
@@ -731,7 +758,8 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     a.dqw = (float*)(ws + oq);
     a.dkw = (float*)(ws + ok_);
     const std::vector<int> nck = chunk_counts(p, plan.cu_host);
-    const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count());
+    // a reverse warm-up chunk runs only the dH chain: about a third of a full chunk
+    const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count(), 0.3);
     a.L = sc.L;
     a.fixed_segs = p.cu ? 0 : std::max(1, (nck.empty() ? 1 : (nck[0] + sc.L - 1) / sc.L));
     a.auto_warm = plan.split_mode == 1 ? 0 : 1;
@@ -751,7 +779,7 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     }
     gdn_bwd_tc_kernel<<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    if (p.T_total > 0) return launch_bwd_reduce(bp, a.dqw, a.dkw, s);
+    if (p.T_total > 0 && p.group > 1) return launch_bwd_reduce(bp, a.dqw, a.dkw, s);
     return GDN_OK;
 }
 

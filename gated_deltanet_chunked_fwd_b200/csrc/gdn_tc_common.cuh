@@ -174,7 +174,7 @@ __device__ __forceinline__ void solve_diag(const float* As, float* M, int t) {
 // ------------------------------------------------------------------- host side
 // Multi-SM split of the chunk chains (host side): chunks per sequence, and the segment length L
 // that minimises the estimated makespan (waves of CTAs x chunk steps per CTA, a warm-up chunk
-// counted as 1.5 steps).  split_mode: 0 auto, 1 off (one segment per sequence), 2 force (L = 2).
+// counted as warm_cost steps).  split_mode: 0 auto, 1 off (one segment per sequence), 2 force (L = 2).
 inline int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -188,7 +188,8 @@ struct SplitChoice {
     int64_t ctas;
 };
 
-inline SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int split_mode, int nsm) {
+inline SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int split_mode, int nsm,
+                                double warm_cost = 1.5) {
     int maxc = 1;
     for (int c : nchunks) maxc = std::max(maxc, c);
     auto count = [&](int L) {
@@ -206,7 +207,7 @@ inline SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int spl
     for (int L = 1; L <= maxc; ++L) {
         const int64_t S = count(L);
         const double waves = std::ceil((double)S / nsm);
-        const double est = waves * (L + (L < maxc ? 1.5 : 0.0));
+        const double est = waves * (L + (L < maxc ? warm_cost : 0.0));
         if (est < best - 1e-9 || (std::fabs(est - best) < 1e-9 && L > bestL)) {
             best = est;
             bestL = L;
