@@ -57,26 +57,30 @@ def bwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
     return T_total * (elt * (Hk * 4 * dk + Hv * 3 * dv) + Hv * 16) + 2 * N * Hv * dk * dv * 4
 
 
-def kernel_sha16():
-    """Fingerprint of the fused forward kernel's source (matches profiles/traffic.json)."""
+FWD_SOURCES = ("gdn_tc_wy.cu", "gdn_tc_fwd.cu", "gdn_tc_common.cuh", "gdn_sm100.cuh",
+               "gdn_internal.cuh")
+
+
+def source_sha16(files=FWD_SOURCES):
+    """Fingerprint of the tensor-core forward's sources (matches profiles/traffic.json)."""
     import hashlib
 
     h = hashlib.sha256()
-    for f in ("gdn_tc_fwd.cu", "gdn_tc_common.cuh", "gdn_sm100.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "gated_deltanet_chunked_fwd_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def traffic_per_launch():
-    """DRAM bytes (read + write) of one fused-forward launch from the committed ncu capture,
-    or None when the kernel source changed since that capture."""
+def traffic_per_call():
+    """DRAM bytes (read + write) of one forward call (the WY kernel and the fused kernel) from
+    the committed ncu capture, or None when the sources changed since that capture."""
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(tp):
         return None
     with open(tp) as f:
         rec = json.load(f).get("fwd_bf16_T4096_H16_d128", {})
-    return rec.get("bytes_per_launch") if rec.get("kernel_sha16") == kernel_sha16() else None
+    return rec.get("bytes_per_call") if rec.get("source_sha16") == source_sha16() else None
 
 
 def measured_peaks():
@@ -317,19 +321,19 @@ def run_ours(args, world, rank, local):
     ms_e2e = max_over_ranks(sum(time_steps(e2e_step, args.steps, flush, stream)) / args.steps, world)
     e2e_value = tokens * world / (ms_e2e * 1e-3)
 
-    # ---- roofline of the dominant kernel (the whole forward when it is one launch)
+    # ---- roofline of the forward call (the WY kernel + the fused state-chain kernel)
     hbm, bf16, src = measured_peaks()
     byts = fwd_bytes(tokens, Hk, Hv, dk, dv, N)
     dense, tri = flops_per_token_head(dk, dv)
     achieved = byts / (ms_step * 1e-3) / 1e9
     tflops_dense = dense * tokens * Hv / (ms_step * 1e-3) / 1e12
     tflops_tri = tri * tokens * Hv / (ms_step * 1e-3) / 1e12
-    traffic = traffic_per_launch() if launches == 1 else None
+    traffic = traffic_per_call() if launches == 2 else None
 
     # ---- backward on its own workload (one step per measurement)
     bwd = None
     if not args.no_bwd:
-        bi = make_workload(4, seed=rank, device=dev)
+        bi = make_workload(4, seed=rank, device=dev, B=args.bwd_batch)
         qs = [bi[n] for n in ("q", "k", "v", "beta", "g", "do")]
         wsb = torch.empty(max(gdn.gdn_chunk_bwd_workspace_size(*qs[:5]), 1), dtype=torch.uint8,
                           device=dev)
@@ -344,10 +348,17 @@ def run_ours(args, world, rank, local):
         bt = bi["q"].shape[0] * bi["q"].shape[1]
         bd, btri = flops_per_token_head(dk, dv, backward=True)
         bb = bwd_bytes(bt, Hk, Hv, dk, dv, bi["q"].shape[0])
-        bwd = {"workload": "gdn_bwd bf16 B=4 T=8192 H=16 dk=dv=128 C=64", "tokens_per_s": bt * world / (bms * 1e-3),
+        t_roof = max(bd * bt * Hv / (bf16 * 1e12), bb / (hbm * 1e9))  # seconds
+        bwd = {"workload": f"gdn_bwd bf16 B={args.bwd_batch} T=8192 H=16 dk=dv=128 C=64",
+               "tokens_per_s": bt * world / (bms * 1e-3),
                "ms": bms, "tflops_dense": bd * bt * Hv / (bms * 1e-3) / 1e12,
                "tflops_tri": btri * bt * Hv / (bms * 1e-3) / 1e12,
                "hbm_gbs": bb / (bms * 1e-3) / 1e9,
+               "roofline": {"bound": "tensor" if bd * bt * Hv / (bf16 * 1e12) >= bb / (hbm * 1e9) else "hbm",
+                            "t_roof_ms": t_roof * 1e3, "frac": t_roof / (bms * 1e-3),
+                            "peak_tflops": bf16, "peak_gbs": hbm, "peak_source": src},
+               "path": "WY kernel + fused kernel (state replay) + reverse kernel"
+                       + (" + dq/dk group reduction" if Hv != Hk else ""),
                "launches": gdn.launch_count(*qs[:5], backward=True)}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
@@ -378,7 +389,7 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
                          "peak_source": src, "algorithmic_bytes": byts,
-                         "kernel": "whole forward (all launches of one call)"},
+                         "kernel": "whole forward call: gdn_wy_tc_kernel + gdn_fwd_tc_kernel"},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches * args.steps,
@@ -397,6 +408,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--bwd-batch", type=int, default=4,
+                    help="sequences in the backward workload (4 = the backward workload; fewer for a small profile)")
     args = ap.parse_args()
     if args.impl == "reference":
         # the oracle arm runs on rank 0's host cores only; no process group
