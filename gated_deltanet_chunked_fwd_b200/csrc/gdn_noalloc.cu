@@ -4,9 +4,8 @@
 // Some callers have no way to call cudaMalloc: code that runs inside a framework
 // plugin or an inference server whose memory is pooled and frozen after start-up,
 // or a runtime that forbids allocation on the request path.  For them this entry
-// point runs the CUDA-core forward (the portable kernels, the ones that need
-// scratch memory) with its scratch in a fixed, file-scope device array instead of
-// a workspace argument.  The array is part of the library image: every GPU that
+// point runs the CUDA-core forward (the portable kernels) with its scratch in a
+// fixed, file-scope device array instead of a workspace argument.  The array is part of the library image: every GPU that
 // loads libgdn.so holds it until the process exits.
 #include <mutex>
 
@@ -51,7 +50,7 @@ extern "C" {
 gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, void* stream) {
     if (!args) return GDN_ERR_INVALID_ARG;
     gdn_fwd_args a = *args;
-    a.flags |= GDN_FLAG_PORTABLE;  // the CUDA-core kernels: the path that uses scratch memory
+    a.flags |= GDN_FLAG_PORTABLE;  // the CUDA-core kernels
     FwdPlan plan;
     gdn_status st = plan_fwd(&a, &plan);
     if (st) return st;

@@ -138,7 +138,10 @@ typedef struct gdn_bwd_args {
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these arguments (the
  * pointers may be NULL here; only sizes, dtype and cu_seqlens_host are read).
- * Returns GDN_OK and sets *bytes, or an argument error. */
+ * Returns GDN_OK and sets *bytes, or an argument error.  The tensor-core path
+ * (bf16, dk = dv = 128) keeps one 8 KB bf16 T = (I + A)^-1 image and one 8-byte
+ * gate summary per (chunk slot, value head), with floor(T_total / 64) + N + 1
+ * chunk slots; the CUDA-core path keeps fp32 W, U, gamma and chunk states. */
 GDN_API gdn_status gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args, size_t* bytes);
 
 /* Forward: o and (optionally) S_T from q, k, v, beta, g and (optionally) S0.
@@ -148,7 +151,9 @@ GDN_API gdn_status gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args, size_t
 GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size_t workspace_bytes,
                          void* stream);
 
-/* Bytes of device workspace gdn_chunk_bwd needs. */
+/* Bytes of device workspace gdn_chunk_bwd needs: on the tensor-core path the
+ * forward's images and summaries, a 32 KB bf16 entry-state image per (chunk
+ * slot, value head), and with grouped heads fp32 dq / dk per value head. */
 GDN_API gdn_status gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args, size_t* bytes);
 
 /* Backward: dq, dk, dv, dbeta, dg and (optionally) dS0 of the forward above
@@ -166,7 +171,7 @@ GDN_API const char* gdn_status_string(int status);
  * is an interface convenience of this library.)
  *
  * It computes exactly what gdn_chunk_fwd computes, always with the CUDA-core
- * kernels (the path that needs scratch memory), and keeps that scratch in a
+ * kernels (as with GDN_FLAG_PORTABLE), and keeps their scratch in a
  * fixed device array of GDN_NOALLOC_SCRATCH_BYTES that is part of libgdn.so:
  * every GPU that loads the library holds it until the process exits.  It calls
  * no cudaMalloc / cudaFree.  Problems whose scratch would exceed the array are
