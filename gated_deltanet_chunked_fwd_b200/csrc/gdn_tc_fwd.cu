@@ -12,7 +12,8 @@
 //   Bw, Bu     T diag(beta Gam), T diag(beta) from the T image          CUDA cores
 //   MMA_W/U    W^T = K^T (T diag(beta Gam))^T,  Ut^T = V^T (T diag(beta))^T
 //   MMA_HW     U^T = Ut^T - H^T W^T  (accumulated onto Ut^T, B = -W^T)
-//   MMA_HQ/UP  O^T = Gam * (H^T Q^T) + U^T P^T,  P = lower-incl(Q K^T o E)
+//   MMA_O      O^T = H^T (diag(Gam) Q)^T + U^T P^T,  P = lower-incl(Q K^T o E)
+//              (Q scaled by Gam in shared memory once Q K^T has read it)
 //   MMA_H      H^T <- Gam_n H^T + (U^T diag(exp(gamma_n - gamma))) K
 // All matrices are oriented so that a 128-wide head dimension is the MMA's M
 // (TMEM lane = dv or dk index), so every MMA is M = 128 with N = 64 or 128.
@@ -65,8 +66,8 @@ constexpr int kTmemCols = 512;
 constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk     [0, 128)
 constexpr uint32_t kColR1 = 128;  // Q K^T (lanes 0-63), then W^T (group P)   [128, 192)
 constexpr uint32_t kColR2 = 192;  // 2 x (Ut^T -> U^T), by chunk parity      [192, 320)
-constexpr uint32_t kColHQ = 320;  // H^T Q^T                                 [320, 384)
-constexpr uint32_t kColUP = 384;  // U^T P^T                                 [384, 448)
+constexpr uint32_t kColO = 320;   // O^T = H^T (diag(Gam) Q)^T + U^T P^T      [320, 384)
+                                  // (columns [384, 448) are free)
 constexpr uint32_t kColHb = 448;  // bf16 H^T, A operand (K pairs per column) [448, 512)
 // U^T in bf16 (A operand of MMA_UP / MMA_H) overwrites the first 32 columns of its R2 buffer.
 
@@ -80,7 +81,8 @@ constexpr uint32_t kWt = 131072;       // 16 KB  W^T: [128 dk rows][64 tokens]
 constexpr uint32_t kTimg = 147456;     // 2 x 8 KB  bf16 T images [n][s], by chunk parity
 constexpr uint32_t kVec = 163840;      // 4 x 2 KB of per-token vectors, by chunk index mod 4
 constexpr uint32_t kVecStride = 512;   // floats per buffer
-constexpr uint32_t kRed = kVec + 4 * kVecStride * 4;  // 16 floats
+constexpr uint32_t kOst = kVec + 4 * kVecStride * 4;  // 16 KB bf16 o tile [dv atom][64 tokens][128 B]
+constexpr uint32_t kRed = kOst + 16384;                // 16 floats
 constexpr uint32_t kBar = kRed + 64;   // 9 mbarriers + TMEM base
 constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
 static_assert(kTimg + 2 * kTImgBytes <= kVec, "T images overlap the vectors");
@@ -99,7 +101,8 @@ struct TcArgs {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const TcArgs args) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                      const TcArgs args) {
     const Problem& p = args.p;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -176,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        if (!args.himg) prefetch_tensormap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -366,15 +370,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int r = row;
                     const int s0 = 32 * hf;
                     const float ar = va[r];
+                    if (fac) {  // block-uniform: E_rs = a_r b_s
 #pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
-                        const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
+                            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s = s0 + 4 * c4 + e;
-                            const float E = fac ? ar * bb[e] : exp2f(ar - bb[e]);
-                            v[4 * c4 + e] = (s <= r && r < lc) ? v[4 * c4 + e] * E : 0.f;
+                            for (int e = 0; e < 4; ++e) {
+                                const int s = s0 + 4 * c4 + e;
+                                v[4 * c4 + e] = (s <= r && r < lc) ? v[4 * c4 + e] * (ar * bb[e]) : 0.f;
+                            }
+                        }
+                    } else {  // E_rs = exp2(a_r - b_s) with a = b = gamma log2(e)
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
+                            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int s = s0 + 4 * c4 + e;
+                                v[4 * c4 + e] = (s <= r && r < lc) ? v[4 * c4 + e] * exp2f(ar - bb[e]) : 0.f;
+                            }
                         }
                     }
                     store_row32(sm + kPt + stage * 8192, r, 4 * hf, v);
@@ -383,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int li = ((warp >> 2) << 6) | ((warp & 1) << 5) | lane;  // 0..127
                 const int nr = li >> 1, c0 = 4 * (li & 1);
                 const uint8_t* timg_s = sm + kTimg + stage * kTImgBytes;
-#pragma unroll
+#pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     const int chunk = c0 + cc;
                     const uint32_t off = sw128_off(nr, chunk);
@@ -396,10 +412,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tv[2 * e] = f.x;
                         tv[2 * e + 1] = f.y;
                     }
+                    const float4 g0 = *reinterpret_cast<const float4*>(vbG + 8 * chunk);
+                    const float4 g1 = *reinterpret_cast<const float4*>(vbG + 8 * chunk + 4);
+                    const float4 b0 = *reinterpret_cast<const float4*>(vbeta + 8 * chunk);
+                    const float4 b1 = *reinterpret_cast<const float4*>(vbeta + 8 * chunk + 4);
+                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const float bb8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        vw[e] = tv[e] * vbG[8 * chunk + e];
-                        vu[e] = tv[e] * vbeta[8 * chunk + e];
+                        vw[e] = tv[e] * gg[e];
+                        vu[e] = tv[e] * bb8[e];
                     }
                     *reinterpret_cast<uint4*>(sm + kBw + off) = pack8(vw);
                     *reinterpret_cast<uint4*>(sm + kBu + off) = pack8(vu);
@@ -436,6 +458,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; ++e) v[e] = -v[e];  // MMA_HW accumulates -H^T W^T
                 store_row32(sm + kWt, row, 4 * hf, v);
             }
+            if (emit) {  // Q rows <- Gam_n Q rows, in place (MMA1 has read Q): B operand of MMA_O,
+                         // so that H^T (diag(Gam) Q)^T and U^T P^T accumulate into one buffer
+                const int srow = t >> 2, q = t & 3;
+                uint8_t* qrow = sm + kStageQK + stage * 32768 + (q >> 1) * 16384 + srow * 128;
+                const float gmul = vec[128 + srow];
+#pragma unroll
+                for (int i4 = 0; i4 < 4; ++i4) {
+                    const int c8 = 4 * (q & 1) + ((i4 + srow) & 3);  // rotated: rows spread over banks
+                    uint4 u = *reinterpret_cast<uint4*>(qrow + 16 * c8);
+                    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(b2[e]);
+                        b2[e] = __floats2bfloat162_rn(f.x * gmul, f.y * gmul);
+                    }
+                    *reinterpret_cast<uint4*>(qrow + 16 * c8) = u;
+                }
+            }
             fence_proxy_async();
             tc_fence_before();
             wg_sync(1, kThreadsP);
@@ -444,30 +484,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ======================= group S: the state chain =======================
         // Per chunk k: MMA_HW, then (overlapping it) the outputs of chunk k-1; U^T -> bf16 in
-        // TMEM; MMA_HQ / MMA_UP / MMA_H (A operands from TMEM); then one pass over H that
+        // TMEM; MMA_O / MMA_H (A operands from TMEM); then one pass over H that
         // writes its bf16 copy and pre-scales it by the next chunk's Gam_n (MMA_H of chunk
         // k+1 accumulates onto it).
         const int m = tid - kThreadsP;
         uint32_t ph = 0;  // parity of bar_mma_s
-        auto epilogue = [&](int kk) {  // o[t0+n][h][m] = Gam_n (H^T Q^T)[m][n] + (U^T P^T)[m][n]
+        // o[t0+n][h][m] = O^T[m][n].  A whole chunk goes through a
+        // shared-memory tile and one TMA store per 64-column half: lanes m, m^1 swap one value so
+        // that each thread writes bf16 pairs (columns m & ~1, m | 1) of one token.  A chunk cut
+        // short by its sequence's end is stored element by element, masked to its tokens.
+        auto epilogue = [&](int kk) {
             const int cc = cstart + kk;
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
-            const float* vGam = (const float*)(sm + kVec) + (kk & 3) * kVecStride + 128;
-            __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+            if (lc == kChunk) {
+                if (m == 0) bulk_wait_read0();  // the previous chunk's store has read the tile
+                wg_sync(2, kThreadsS);
+                const bool odd = m & 1;
+                const int c = m & ~1, cin = c & 63;
+                uint8_t* tile = sm + kOst + (c >> 6) * 8192;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    float ov[32];
+                    tmem_ld32(tl + kColO + 32 * hf, ov);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float hq[32], up[32];
-                tmem_ld32x2(tl + kColHQ + 32 * hf, hq, tl + kColUP + 32 * hf, up);
+                    for (int e = 0; e < 32; e += 2) {
+                        const int nn = 32 * hf + e;
+                        const float x0 = ov[e], x1 = ov[e + 1];
+                        const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
+                        const uint32_t w = odd ? pack_bf16(recv, x1) : pack_bf16(x0, recv);
+                        const int row = nn + (odd ? 1 : 0);
+                        *reinterpret_cast<uint32_t*>(tile + sw128_off(row, cin >> 3) + (cin & 7) * 2) = w;
+                    }
+                }
+                fence_proxy_async();  // the tile is read by the TMA store
+                wg_sync(2, kThreadsS);
+                if (m == 0) {
+                    tma_store_3d(&tm_o, sm + kOst, 0, h, (int)t0);
+                    tma_store_3d(&tm_o, sm + kOst + 8192, 64, h, (int)t0);
+                    bulk_commit();
+                }
+            } else {
+                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 g4 = *reinterpret_cast<const float4*>(vGam + 32 * hf + 4 * e4);
-                    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+                for (int hf = 0; hf < 2; ++hf) {
+                    float ov[32];
+                    tmem_ld32(tl + kColO + 32 * hf, ov);
 #pragma unroll
-                    for (int e1 = 0; e1 < 4; ++e1) {
-                        const int e = 4 * e4 + e1, nn = 32 * hf + e;
-                        if (nn < lc)
-                            op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(gv[e1] * hq[e] + up[e]);
+                    for (int e = 0; e < 32; ++e) {
+                        const int nn = 32 * hf + e;
+                        if (nn < lc) op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(ov[e]);
                     }
                 }
             }
@@ -545,20 +611,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             wg_sync(2, kThreadsS);
-            if (m == 0) {  // MMA_HQ: H^T Q^T;  MMA_UP: U^T P^T;  MMA_H: H^T += (U^T diag(decay)) K
+            if (m == 0) {  // MMA_O: O^T = H^T (diag(Gam) Q)^T + U^T P^T;  MMA_H: H^T += (U^T diag(decay)) K
                 tc_fence_after();
                 if (emit) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                        mma_bf16_ts(tmem + kColHQ, tmem + kColHb + 8 * j, desc_sw128(sQK + koff, 16, 1024),
+                        mma_bf16_ts(tmem + kColO, tmem + kColHb + 8 * j, desc_sw128(sQK + koff, 16, 1024),
                                     id_n64, j > 0);
                     }
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        mma_bf16_ts(tmem + kColUP, tmem + colR2 + 8 * j,
-                                    desc_sw128(sbase + kPt + stage * 8192 + j * 32, 16, 1024), id_n64,
-                                    j > 0);
+                        mma_bf16_ts(tmem + kColO, tmem + colR2 + 8 * j,
+                                    desc_sw128(sbase + kPt + stage * 8192 + j * 32, 16, 1024), id_n64, 1);
                 }
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
@@ -579,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float Gn = more ? ((const float*)(sm + kVec))[((k + 1) & 3) * kVecStride + 128 + 63] : 1.f;
                 float v[64];
                 uint32_t w[32];
-#pragma unroll
+#pragma unroll 1
                 for (int a = 0; a < 2; ++a) {
                     tmem_ld64(tl + kColH + 64 * a, v);
 #pragma unroll
@@ -597,6 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m == 0) mbar_arrive(&bar_s_done[stage]);
         }
         if (ok && nk > 0 && cstart + nk - 1 >= c0 && !args.himg) epilogue(nk - 1);
+        if (m == 0) bulk_wait0();  // every output tile has been written
         if (ok && p.ST && seg == segs_n - 1) {
             // final state S_T = H (stored [dk][dv]): thread m writes column m
             float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + m;
@@ -645,10 +711,12 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
     a.fixed_segs = p.cu ? 0 : std::max(1, (nck.empty() ? 1 : (nck[0] + sc.L - 1) / sc.L));
     a.auto_warm = split_mode == 1 ? 0 : 1;
     a.log_eps = (float)(-30.0 * std::log(2.0));
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const int64_t Tt = std::max<int64_t>(p.T_total, 1);
     if (!make_map(&mq, p.q, Tt, p.Hk) || !make_map(&mk, p.k, Tt, p.Hk) || !make_map(&mv, p.v, Tt, p.Hv))
         return GDN_ERR_CUDA;
+    // o (replay mode writes no o: the map is then never used)
+    if (!make_map(&mo, p.o ? p.o : p.v, Tt, p.Hv)) return GDN_ERR_CUDA;
     if (cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
@@ -669,7 +737,7 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = p.num_chunks > 0 ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, gdn_fwd_tc_kernel, mq, mk, mv, a) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, gdn_fwd_tc_kernel, mq, mk, mv, mo, a) != cudaSuccess) return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -301,8 +301,14 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
             const int r = 16 * m + g8 + 8 * hr, s = 8 * j + 2 * t4;
             const float ar = va[r], br = vbeta[r];
             const float2 b2 = *reinterpret_cast<const float2*>(vb + s);
-            const float e0 = fac ? ar * b2.x : exp2f(ar - b2.x);
-            const float e1 = fac ? ar * b2.y : exp2f(ar - b2.y);
+            float e0, e1;
+            if (fac) {  // block-uniform
+                e0 = ar * b2.x;
+                e1 = ar * b2.y;
+            } else {
+                e0 = exp2f(ar - b2.x);
+                e1 = exp2f(ar - b2.y);
+            }
             float2 w;
             w.x = (s < r && r < lc) ? br * acc[i][2 * hr] * e0 : 0.f;
             w.y = (s + 1 < r && r < lc) ? br * acc[i][2 * hr + 1] * e1 : 0.f;
