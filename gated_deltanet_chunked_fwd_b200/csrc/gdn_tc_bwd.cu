@@ -278,8 +278,29 @@ __global__ void __launch_bounds__(kNT, 1)
         __syncthreads();
         return fac;
     };
-    auto Efac = [&](bool fac, int r, int s) -> float {
-        return fac ? va[r] * vb[s] : exp2f(va[r] - vb[s]);
+    // E_rs for the 32 columns s0 .. s0 + 31 of row r: a_r b_s when every |gamma - gamma_31| < 80
+    // (block-uniform), else exp2(a_r - b_s) with a = b = gamma log2(e)
+    auto fill_E = [&](bool fac, int r, int s0, float* E) {
+        const float ar = va[r];
+        if (fac) {
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
+                E[4 * c4] = ar * b4.x;
+                E[4 * c4 + 1] = ar * b4.y;
+                E[4 * c4 + 2] = ar * b4.z;
+                E[4 * c4 + 3] = ar * b4.w;
+            }
+        } else {
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(vb + s0 + 4 * c4);
+                E[4 * c4] = exp2f(ar - b4.x);
+                E[4 * c4 + 1] = exp2f(ar - b4.y);
+                E[4 * c4 + 2] = exp2f(ar - b4.z);
+                E[4 * c4 + 3] = exp2f(ar - b4.w);
+            }
+        }
     };
     auto mma1 = [&]() {  // [Q;K] K^T -> R1
         if (tid == 0) {
@@ -355,12 +376,13 @@ __global__ void __launch_bounds__(kNT, 1)
         // P (rows 0..63) -> smem; Bw, Bu from the T image
         if (m < 64) {  // P row m, this thread's half of the columns
             const int r = m;
-            float v[32];
+            float v[32], E[32];
             tmem_ld32(tl + cR1 + 32 * hh, v);
+            fill_E(fac, r, 32 * hh, E);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int s = 32 * hh + e;
-                v[e] = (s <= r && r < lc) ? v[e] * Efac(fac, r, s) : 0.f;
+                v[e] = (s <= r && r < lc) ? v[e] * E[e] : 0.f;
             }
             store_row32(sm + bP, r, 4 * hh, v);
         }
@@ -494,7 +516,8 @@ __global__ void __launch_bounds__(kNT, 1)
     #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int r = 32 * hh + e;
-                    if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn(vbeta[r] * v[e]);
+                    const float4 bt4 = *reinterpret_cast<const float4*>(vbeta + 32 * hh + (e & ~3));
+                    if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn((&bt4.x)[e & 3] * v[e]);
                     bvals[e] = v[e] * bf(sm + bV + (m >> 6) * 8192, r, m & 63);  // TdU[r][m] v[r][m]
                     // TdU row r of the stacked [dO ; TdU] tile: element (64 + r, m)
                     *reinterpret_cast<__nv_bfloat16*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
@@ -540,15 +563,16 @@ __global__ void __launch_bounds__(kNT, 1)
             {  // dP (lanes 0..63) and dA (lanes 64..127) rows, columns s in [32 hh, 32 hh + 32):
                // dgamma / dbeta terms, dP o E, G
                 const int r = m & 63;
-                float d[32], x[32];
+                float d[32], x[32], Ev[32];
                 tmem_ld32x2(tl + cR3 + 32 * hh, d, tl + cR1 + 32 * hh, x);
+                fill_E(fac, r, 32 * hh, Ev);
                 float rowsum = 0.f, bsum = 0.f;
                 if (m < 64) {
     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int s = 32 * hh + e;
                         const bool in = (s <= r && r < lc);
-                        const float E = Efac(fac, r, s);
+                        const float E = Ev[e];
                         const float P = in ? x[e] * E : 0.f;
                         const float dP = in ? d[e] : 0.f;
                         rowsum += dP * P;
@@ -567,7 +591,7 @@ __global__ void __launch_bounds__(kNT, 1)
                         for (int e4 = 0; e4 < 4; ++e4) {
                             const int e = 4 * c4 + e4, s = 32 * hh + e;
                             const bool in = (s < r && r < lc);
-                            const float E = Efac(fac, r, s);
+                            const float E = Ev[e];
                             const float dA = in ? -d[e] : 0.f;
                             const float KE = x[e] * E;
                             const float A = br * KE;
@@ -640,7 +664,9 @@ __global__ void __launch_bounds__(kNT, 1)
     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int r = 32 * hh + e;
-                        const float qs = vGam[r] * a32[e];  // dQs^T[i][r]
+                        const float4 g4 = *reinterpret_cast<const float4*>(vGam + 32 * hh + (e & ~3));
+                        const float gme = (&g4.x)[e & 3];
+                        const float qs = gme * a32[e];  // dQs^T[i][r]
                         if (r < lc) {
                             if (direct) dqb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(qs + b32[e]);
                             else dqp[(int64_t)r * Hv * dk] = qs + b32[e];
@@ -656,14 +682,19 @@ __global__ void __launch_bounds__(kNT, 1)
                     for (int e = 0; e < 32; ++e) {
                         const int s = 32 * hh + e;
                         const float kv = bf(qtile, 64 + s, i & 63);
-                        const float dkv = a32[e] + vdec[s] * b32[e] + vbG[s] * c32[e];
+                        const int s4 = 32 * hh + (e & ~3);
+                        const float4 dc4 = *reinterpret_cast<const float4*>(vdec + s4);
+                        const float4 bg4 = *reinterpret_cast<const float4*>(vbG + s4);
+                        const float4 gm4 = *reinterpret_cast<const float4*>(vGam + s4);
+                        const float dec_s = (&dc4.x)[e & 3], bG_s = (&bg4.x)[e & 3], Gam_s = (&gm4.x)[e & 3];
+                        const float dkv = a32[e] + dec_s * b32[e] + bG_s * c32[e];
                         if (s < lc) {
                             if (direct) dkb[(int64_t)s * Hv * dk] = __float2bfloat16_rn(dkv);
                             else dkp[(int64_t)s * Hv * dk] = dkv;
                         }
-                        const float kdterm = vdec[s] * kv * b32[e];
-                        gv[e] += vbG[s] * c32[e] * kv - kdterm;
-                        bv[e] = vGam[s] * c32[e] * kv;
+                        const float kdterm = dec_s * kv * b32[e];
+                        gv[e] += bG_s * c32[e] * kv - kdterm;
+                        bv[e] = Gam_s * c32[e] * kv;
                         kdk += kdterm;
                     }
                 }
