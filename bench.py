@@ -144,16 +144,22 @@ class Clocks:
                 "samples": len(rows)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU (torchrun environment); NCCL on GPUs, gloo when there is none."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
 
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout,
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -165,11 +171,19 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest per-rank value (a step time): the job is as slow as its slowest rank."""
     if world <= 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job units per second: every rank runs its own replica on its own batch (weak
+    scaling, no collective on the data path), and the step takes ``ms``, the max over ranks."""
+    return units_per_rank * world / (ms * 1e-3)
 
 
 # ----------------------------------------------------------------- oracle arm
@@ -290,7 +304,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     ms_step = max_over_ranks(sum(ms) / len(ms), world)
     tokens = B * T
-    value = tokens * world / (ms_step * 1e-3)
+    value = job_throughput(tokens, world, ms_step)
 
     # ---- e2e: pinned host inputs, H2D + call + D2H of o and S_T, inside the timed region
     host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("beta", beta),
@@ -319,7 +333,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     ms_e2e = max_over_ranks(sum(time_steps(e2e_step, args.steps, flush, stream)) / args.steps, world)
-    e2e_value = tokens * world / (ms_e2e * 1e-3)
+    e2e_value = job_throughput(tokens, world, ms_e2e)
 
     # ---- roofline of the forward call (the WY kernel + the fused state-chain kernel)
     hbm, bf16, src = measured_peaks()
@@ -350,7 +364,7 @@ def run_ours(args, world, rank, local):
         bb = bwd_bytes(bt, Hk, Hv, dk, dv, bi["q"].shape[0])
         t_roof = max(bd * bt * Hv / (bf16 * 1e12), bb / (hbm * 1e9))  # seconds
         bwd = {"workload": f"gdn_bwd bf16 B={args.bwd_batch} T=8192 H=16 dk=dv=128 C=64",
-               "tokens_per_s": bt * world / (bms * 1e-3),
+               "tokens_per_s": job_throughput(bt, world, bms),
                "ms": bms, "tflops_dense": bd * bt * Hv / (bms * 1e-3) / 1e12,
                "tflops_tri": btri * bt * Hv / (bms * 1e-3) / 1e12,
                "hbm_gbs": bb / (bms * 1e-3) / 1e9,
