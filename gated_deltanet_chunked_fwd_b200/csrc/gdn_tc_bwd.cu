@@ -246,12 +246,22 @@ __global__ void __launch_bounds__(kNT, 1)
         return r;
     };
     // gates of chunk c: beta, gamma (cumsum), Gam, beta Gam, decay to the chunk end, E factors
+    // g and beta of the next chunk in the walk, loaded one chunk ahead (threads 0..63)
+    float nxt_g = 0.f, nxt_b = 0.f;
+    auto prefetch_gates = [&](int c) {
+        if (tid < 64 && c >= c0) {
+            const int64_t t0 = bos + (int64_t)c * kChunk;
+            const int lcc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+            nxt_g = tid < lcc ? p.g[(t0 + tid) * Hv + h] : 0.f;  // padding: g = 0, beta = 0
+            nxt_b = tid < lcc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
+        }
+    };
     auto gates = [&](int c, int lc) -> bool {
-        const int64_t t0 = bos + (int64_t)c * kChunk;
         float gr = 0.f, gm = 0.f;
         if (tid < 64) {
-            float x = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;
-            const float bt = tid < lc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
+            float x = nxt_g;
+            const float bt = nxt_b;
+            prefetch_gates(c - 1);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -341,6 +351,7 @@ __global__ void __launch_bounds__(kNT, 1)
         __syncthreads();
         tc_fence_after();
     }
+    prefetch_gates(cend - 1);
     for (int c = cend - 1; c >= c0 && ok; --c) {
         const bool emit = c < c1;  // own chunk (else: reverse warm-up, the dH chain only)
         const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
@@ -390,11 +401,18 @@ __global__ void __launch_bounds__(kNT, 1)
             const int nrow = tid >> 2, q = tid & 3;
             float vw[16], vu[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int s = 16 * q + e;
-                const float t = bf(sm + bT, nrow, s);
-                vw[e] = t * vbG[s];
-                vu[e] = t * vbeta[s];
+            for (int hc = 0; hc < 2; ++hc) {
+                const uint4 u = *reinterpret_cast<const uint4*>(sm + bT + sw128_off(nrow, 2 * q + hc));
+                const __nv_bfloat162* t2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const float2 f = __bfloat1622float2(t2[e2]);
+                    const int e = 8 * hc + 2 * e2, s = 16 * q + e;
+                    vw[e] = f.x * vbG[s];
+                    vw[e + 1] = f.y * vbG[s + 1];
+                    vu[e] = f.x * vbeta[s];
+                    vu[e + 1] = f.y * vbeta[s + 1];
+                }
             }
             *reinterpret_cast<uint4*>(sm + bBw + sw128_off(nrow, 2 * q)) = pack8(vw);
             *reinterpret_cast<uint4*>(sm + bBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
@@ -467,11 +485,20 @@ __global__ void __launch_bounds__(kNT, 1)
             float dhh = 0.f;
             const float Gn = vGam[63];
             tmem_ld64(tl + cH + 64 * hh, v);
+            if (emit) {  // <dH_c, H_c> over this thread's row m, columns [64 hh, 64 hh + 64)
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                if (emit) dhh += v[e] * bf(sm + bHt + hh * 16384, m, e);
-                v[e] *= Gn;
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(sm + bHt + hh * 16384 + sw128_off(m, c8));
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        dhh += v[8 * c8 + 2 * e] * f.x + v[8 * c8 + 2 * e + 1] * f.y;
+                    }
+                }
             }
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e] *= Gn;
             tmem_st64(tl + cH + 64 * hh, v);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) dhh += __shfl_xor_sync(0xffffffffu, dhh, o);
