@@ -173,6 +173,41 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         : "memory");
 }
 
+// 8 consecutive 32-bit TMEM columns of this warp's 32 lanes -> 8 registers per thread; waits.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+}
+
+// five 8-column loads (five accumulators) with one wait
+__device__ __forceinline__ void tmem_ld8x5(uint32_t t0, float* v0, uint32_t t1, float* v1, uint32_t t2,
+                                           float* v2, uint32_t t3, float* v3, uint32_t t4, float* v4) {
+    uint32_t* a = reinterpret_cast<uint32_t*>(v0);
+    uint32_t* b = reinterpret_cast<uint32_t*>(v1);
+    uint32_t* c = reinterpret_cast<uint32_t*>(v2);
+    uint32_t* d = reinterpret_cast<uint32_t*>(v3);
+    uint32_t* e = reinterpret_cast<uint32_t*>(v4);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%40];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%41];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16,%17,%18,%19,%20,%21,%22,%23}, [%42];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24,%25,%26,%27,%28,%29,%30,%31}, [%43];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%32,%33,%34,%35,%36,%37,%38,%39}, [%44];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+          "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+          "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3]), "=r"(c[4]), "=r"(c[5]), "=r"(c[6]), "=r"(c[7]),
+          "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]), "=r"(d[7]),
+          "=r"(e[0]), "=r"(e[1]), "=r"(e[2]), "=r"(e[3]), "=r"(e[4]), "=r"(e[5]), "=r"(e[6]), "=r"(e[7])
+        : "r"(t0), "r"(t1), "r"(t2), "r"(t3), "r"(t4)
+        : "memory");
+}
+
 // 32 consecutive 32-bit TMEM columns of this warp's 32 lanes -> 32 registers per
 // thread (thread i of the warp gets lane 32*(warp%4) + i).  Waits for completion.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {

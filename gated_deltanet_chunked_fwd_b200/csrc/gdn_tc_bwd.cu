@@ -673,9 +673,9 @@ __global__ void __launch_bounds__(kNT, 1)
                                 desc_sw128(sb + bT + j * 32, 16, 1024), id_mk64, 1);
             }
             if (!(ok = mma_sync_wait())) break;
-            {  // epilogue: thread i = dk index (TMEM lane), tokens [32 hh, 32 hh + 32)
+            {  // epilogue: thread i = dk index (TMEM lane), tokens [32 hh, 32 hh + 32) in four
+               // groups of eight (a rolled loop: a short body keeps the instruction stream small)
                 const int i = m;
-                float gv[32], bv[32];
                 float kdk = 0.f;
                 const uint8_t* qtile = sm + bQK + (i >> 6) * 16384;
                 // without grouped heads dq / dk go out directly (bf16); else per value head (fp32)
@@ -685,63 +685,69 @@ __global__ void __launch_bounds__(kNT, 1)
                 float* dkp = args.dkw + (t0 * Hv + h) * dk + i;
                 __nv_bfloat16* dqb = (__nv_bfloat16*)b.dq + (t0 * Hv + h) * dk + i;
                 __nv_bfloat16* dkb = (__nv_bfloat16*)b.dk + (t0 * Hv + h) * dk + i;
-                {
-                    float a32[32], b32[32];
-                    tmem_ld32x2(tl + cR4 + 32 * hh, a32, tl + cR3 + 32 * hh, b32);  // H dO^T, K^T dPE^T
-    #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int r = 32 * hh + e;
-                        const float4 g4 = *reinterpret_cast<const float4*>(vGam + 32 * hh + (e & ~3));
-                        const float gme = (&g4.x)[e & 3];
-                        const float qs = gme * a32[e];  // dQs^T[i][r]
-                        if (r < lc) {
-                            if (direct) dqb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(qs + b32[e]);
-                            else dqp[(int64_t)r * Hv * dk] = qs + b32[e];
-                        }
-                        gv[e] = bf(qtile, r, i & 63) * qs;
+                float* red2 = (float*)(sm + bBw);  // [8 warps][32]: the Gam-scaled Q is no longer read
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    const int tb = 32 * hh + 8 * g;  // first token of the group
+                    float hdo[8], kpe[8], dkm[8], dkd[8], tdw[8];
+                    // H dO^T, K^T dPE^T, dk main, dKd^T, TdW^T for the group's 8 tokens
+                    tmem_ld8x5(tl + cR4 + tb, hdo, tl + cR3 + tb, kpe, tl + cR1 + tb, dkm, tl + cR2 + tb, dkd,
+                               tl + cR5 + tb, tdw);
+                    float gam8[8], dec8[8], bg8[8];
+#pragma unroll
+                    for (int h4 = 0; h4 < 2; ++h4) {
+                        const float4 x1 = *reinterpret_cast<const float4*>(vGam + tb + 4 * h4);
+                        const float4 x2 = *reinterpret_cast<const float4*>(vdec + tb + 4 * h4);
+                        const float4 x3 = *reinterpret_cast<const float4*>(vbG + tb + 4 * h4);
+                        gam8[4 * h4] = x1.x; gam8[4 * h4 + 1] = x1.y; gam8[4 * h4 + 2] = x1.z; gam8[4 * h4 + 3] = x1.w;
+                        dec8[4 * h4] = x2.x; dec8[4 * h4 + 1] = x2.y; dec8[4 * h4 + 2] = x2.z; dec8[4 * h4 + 3] = x2.w;
+                        bg8[4 * h4] = x3.x; bg8[4 * h4 + 1] = x3.y; bg8[4 * h4 + 2] = x3.z; bg8[4 * h4 + 3] = x3.w;
                     }
-                }
-                {
-                    float a32[32], b32[32], c32[32];
-                    tmem_ld32x2(tl + cR1 + 32 * hh, a32, tl + cR2 + 32 * hh, b32);  // dk main, dKd^T
-                    tmem_ld32(tl + cR5 + 32 * hh, c32);                              // TdW^T
-    #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int s = 32 * hh + e;
-                        const float kv = bf(qtile, 64 + s, i & 63);
-                        const int s4 = 32 * hh + (e & ~3);
-                        const float4 dc4 = *reinterpret_cast<const float4*>(vdec + s4);
-                        const float4 bg4 = *reinterpret_cast<const float4*>(vbG + s4);
-                        const float4 gm4 = *reinterpret_cast<const float4*>(vGam + s4);
-                        const float dec_s = (&dc4.x)[e & 3], bG_s = (&bg4.x)[e & 3], Gam_s = (&gm4.x)[e & 3];
-                        const float dkv = a32[e] + dec_s * b32[e] + bG_s * c32[e];
-                        if (s < lc) {
-                            if (direct) dkb[(int64_t)s * Hv * dk] = __float2bfloat16_rn(dkv);
-                            else dkp[(int64_t)s * Hv * dk] = dkv;
+                    float gv[8], bv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int r = tb + e;
+                        const float qs = gam8[e] * hdo[e];  // dQs^T[i][r]
+                        const float dqv = qs + kpe[e];
+                        const float kv = bf(qtile, 64 + r, i & 63);
+                        const float dkv = dkm[e] + dec8[e] * dkd[e] + bg8[e] * tdw[e];
+                        if (r < lc) {
+                            if (direct) {
+                                dqb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(dqv);
+                                dkb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(dkv);
+                            } else {
+                                dqp[(int64_t)r * Hv * dk] = dqv;
+                                dkp[(int64_t)r * Hv * dk] = dkv;
+                            }
                         }
-                        const float kdterm = dec_s * kv * b32[e];
-                        gv[e] += bG_s * c32[e] * kv - kdterm;
-                        bv[e] = Gam_s * c32[e] * kv;
+                        const float kdterm = dec8[e] * kv * dkd[e];
+                        gv[e] = bf(qtile, r, i & 63) * qs + bg8[e] * tdw[e] * kv - kdterm;
+                        bv[e] = gam8[e] * tdw[e] * kv;
                         kdk += kdterm;
                     }
+                    // sums over this warp's 32 i for each of the 8 tokens: lane l ends with token l / 4
+                    warp_reduce_scatter<8>(gv, lane);
+                    warp_reduce_scatter<8>(bv, lane);
+                    gv[0] += __shfl_xor_sync(0xffffffffu, gv[0], 2);
+                    gv[0] += __shfl_xor_sync(0xffffffffu, gv[0], 1);
+                    bv[0] += __shfl_xor_sync(0xffffffffu, bv[0], 2);
+                    bv[0] += __shfl_xor_sync(0xffffffffu, bv[0], 1);
+                    if ((lane & 3) == 0) {
+                        red[warp * 32 + 8 * g + (lane >> 2)] = gv[0];
+                        red2[warp * 32 + 8 * g + (lane >> 2)] = bv[0];
+                    }
                 }
-                warp_reduce_scatter<32>(gv, lane);  // lane l: token 32 hh + l, summed over this warp's i
-                warp_reduce_scatter<32>(bv, lane);
     #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) kdk += __shfl_xor_sync(0xffffffffu, kdk, o);
-                red[warp * 32 + lane] = gv[0];
                 if (lane == 0) atomicAdd(&acc_s[1], kdk);
                 __syncthreads();
-                const int q4 = (tid >> 5) * 4, l = tid & 31;
-                if (tid < 64)
+                if (tid < 64) {
+                    const int q4 = (tid >> 5) * 4, l = tid & 31;
                     acc_g[tid] += red[q4 * 32 + l] + red[(q4 + 1) * 32 + l] + red[(q4 + 2) * 32 + l] +
                                   red[(q4 + 3) * 32 + l];
-                __syncthreads();
-                red[warp * 32 + lane] = bv[0];
-                __syncthreads();
-                if (tid < 64)
-                    acc_b[tid] += red[q4 * 32 + l] + red[(q4 + 1) * 32 + l] + red[(q4 + 2) * 32 + l] +
-                                  red[(q4 + 3) * 32 + l];
+                    acc_b[tid] += red2[q4 * 32 + l] + red2[(q4 + 1) * 32 + l] + red2[(q4 + 2) * 32 + l] +
+                                  red2[(q4 + 3) * 32 + l];
+                }
                 __syncthreads();
             }
             if (warp == 0) {  // last-row terms, then dg = reverse in-chunk cumsum of dgamma
