@@ -184,6 +184,20 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
         : "memory");
 }
 
+// two 8-column loads with one wait
+__device__ __forceinline__ void tmem_ld8x2(uint32_t t0, float* v0, uint32_t t1, float* v1) {
+    uint32_t* a = reinterpret_cast<uint32_t*>(v0);
+    uint32_t* b = reinterpret_cast<uint32_t*>(v1);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%16];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%17];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+          "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7])
+        : "r"(t0), "r"(t1)
+        : "memory");
+}
+
 // five 8-column loads (five accumulators) with one wait
 __device__ __forceinline__ void tmem_ld8x5(uint32_t t0, float* v0, uint32_t t1, float* v1, uint32_t t2,
                                            float* v2, uint32_t t3, float* v3, uint32_t t4, float* v4) {

@@ -532,29 +532,36 @@ __global__ void __launch_bounds__(kNT, 1)
         }
         if (!(ok = mma_sync_wait())) break;
         if (emit) {  // the chunk's gradients (own chunks only)
-            {  // U^T -> Ut;  TdU: dv out, rows 64..127 of the dO tile, -TdU^T -> Wt, dbeta part
-                // this thread: row m of U^T and of TdU^T, tokens r in [32 hh, 32 hh + 32)
-                float v[32];
-                tmem_ld32(tl + cR3 + 32 * hh, v);
-                store_row32(sm + bUt, m, 4 * hh, v);
-                tmem_ld32(tl + cR2 + 32 * hh, v);
+            {  // U^T -> Ut;  TdU: dv out, rows 64..127 of the dO tile, -TdU^T -> Wt, dbeta part;
+               // this thread: row m of U^T and of TdU^T, tokens [32 hh, 32 hh + 32) in groups of 8
                 __nv_bfloat16* dvp = (__nv_bfloat16*)b.dv + (t0 * Hv + h) * dv + m;
-                float bvals[32];
-    #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int r = 32 * hh + e;
-                    const float4 bt4 = *reinterpret_cast<const float4*>(vbeta + 32 * hh + (e & ~3));
-                    if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn((&bt4.x)[e & 3] * v[e]);
-                    bvals[e] = v[e] * bf(sm + bV + (m >> 6) * 8192, r, m & 63);  // TdU[r][m] v[r][m]
-                    // TdU row r of the stacked [dO ; TdU] tile: element (64 + r, m)
-                    *reinterpret_cast<__nv_bfloat16*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
-                                                      (m & 7) * 2) = __float2bfloat16_rn(v[e]);
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    const int tb = 32 * hh + 8 * g;  // first token of the group
+                    float u8[8], t8[8];
+                    tmem_ld8x2(tl + cR3 + tb, u8, tl + cR2 + tb, t8);
+                    *reinterpret_cast<uint4*>(sm + bUt + sw128_off(m, tb >> 3)) = pack8(u8);
+                    const float4 bt0 = *reinterpret_cast<const float4*>(vbeta + tb);
+                    const float4 bt1 = *reinterpret_cast<const float4*>(vbeta + tb + 4);
+                    const float btv[8] = {bt0.x, bt0.y, bt0.z, bt0.w, bt1.x, bt1.y, bt1.z, bt1.w};
+                    float bvals[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int r = tb + e;
+                        if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn(btv[e] * t8[e]);
+                        bvals[e] = t8[e] * bf(sm + bV + (m >> 6) * 8192, r, m & 63);  // TdU[r][m] v[r][m]
+                        // TdU row r of the stacked [dO ; TdU] tile: element (64 + r, m)
+                        *reinterpret_cast<__nv_bfloat16*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
+                                                          (m & 7) * 2) = __float2bfloat16_rn(t8[e]);
+                        t8[e] = -t8[e];
+                    }
+                    *reinterpret_cast<uint4*>(sm + bWt + sw128_off(m, tb >> 3)) = pack8(t8);
+                    // sums over this warp's 32 m for each token: lane l ends with token tb + l / 4
+                    warp_reduce_scatter<8>(bvals, lane);
+                    bvals[0] += __shfl_xor_sync(0xffffffffu, bvals[0], 2);
+                    bvals[0] += __shfl_xor_sync(0xffffffffu, bvals[0], 1);
+                    if ((lane & 3) == 0) red[warp * 32 + 8 * g + (lane >> 2)] = bvals[0];
                 }
-    #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = -v[e];
-                store_row32(sm + bWt, m, 4 * hh, v);
-                warp_reduce_scatter<32>(bvals, lane);  // lane l: token 32 hh + l, summed over this warp's m
-                red[warp * 32 + lane] = bvals[0];
             }
             fence_proxy_async();
             tc_fence_before();
@@ -587,51 +594,64 @@ __global__ void __launch_bounds__(kNT, 1)
                                 desc_sw128(sb + bUt + j * 2048, 8192, 1024), id_mm64, j > 0);
             }
             if (!(ok = mma_sync_wait())) break;
-            {  // dP (lanes 0..63) and dA (lanes 64..127) rows, columns s in [32 hh, 32 hh + 32):
-               // dgamma / dbeta terms, dP o E, G
+            {  // dP (lanes 0..63) and dA (lanes 64..127) rows, columns s in [32 hh, 32 hh + 32) in
+               // four groups of eight: dgamma / dbeta terms, dP o E, G
                 const int r = m & 63;
-                float d[32], x[32], Ev[32];
-                tmem_ld32x2(tl + cR3 + 32 * hh, d, tl + cR1 + 32 * hh, x);
-                fill_E(fac, r, 32 * hh, Ev);
+                const float ar = va[r], br = vbeta[r];
+                float* G = (float*)(sm + bV);
                 float rowsum = 0.f, bsum = 0.f;
-                if (m < 64) {
-    #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int s = 32 * hh + e;
-                        const bool in = (s <= r && r < lc);
-                        const float E = Ev[e];
-                        const float P = in ? x[e] * E : 0.f;
-                        const float dP = in ? d[e] : 0.f;
-                        rowsum += dP * P;
-                        x[e] = dP * P;      // column-sum term
-                        d[e] = dP * E;      // dP o E
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    const int sb = 32 * hh + 8 * g;  // first column of the group
+                    float d[8], x[8], E[8];
+                    tmem_ld8x2(tl + cR3 + sb, d, tl + cR1 + sb, x);
+                    {
+                        const float4 b0 = *reinterpret_cast<const float4*>(vb + sb);
+                        const float4 b1 = *reinterpret_cast<const float4*>(vb + sb + 4);
+                        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                        if (fac) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) E[e] = ar * bb[e];
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) E[e] = exp2f(ar - bb[e]);
+                        }
                     }
-                    store_row32(sm + bP, r, 4 * hh, d);
-                } else {
-                    float* G = (float*)(sm + bV);
-                    const float br = vbeta[r];
-    #pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        float4 gw;
-                        float* gp = &gw.x;
-    #pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const int e = 4 * c4 + e4, s = 32 * hh + e;
+                    if (m < 64) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int s = sb + e;
+                            const bool in = (s <= r && r < lc);
+                            const float P = in ? x[e] * E[e] : 0.f;
+                            const float dP = in ? d[e] : 0.f;
+                            rowsum += dP * P;
+                            x[e] = dP * P;      // column-sum term
+                            d[e] = dP * E[e];   // dP o E
+                        }
+                        *reinterpret_cast<uint4*>(sm + bP + sw128_off(r, sb >> 3)) = pack8(d);
+                    } else {
+                        float gw[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int s = sb + e;
                             const bool in = (s < r && r < lc);
-                            const float E = Ev[e];
                             const float dA = in ? -d[e] : 0.f;
-                            const float KE = x[e] * E;
+                            const float KE = x[e] * E[e];
                             const float A = br * KE;
                             rowsum += dA * A;
                             bsum += dA * KE;
                             x[e] = dA * A;
-                            gp[e4] = dA * E * br;
+                            gw[e] = dA * E[e] * br;
                         }
-                        *reinterpret_cast<float4*>(G + as_idx(r, 32 * hh + 4 * c4)) = gw;
+                        *reinterpret_cast<float4*>(G + as_idx(r, sb)) = make_float4(gw[0], gw[1], gw[2], gw[3]);
+                        *reinterpret_cast<float4*>(G + as_idx(r, sb + 4)) = make_float4(gw[4], gw[5], gw[6], gw[7]);
                     }
+                    // column sums over this warp's rows: lane l ends with column sb + l / 4
+                    warp_reduce_scatter<8>(x, lane);
+                    x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
+                    x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
+                    if ((lane & 3) == 0) red[warp * 32 + 8 * g + (lane >> 2)] = x[0];
                 }
-                warp_reduce_scatter<32>(x, lane);  // lane l: column 32 hh + l, summed over this warp's rows
-                red[warp * 32 + lane] = x[0];
                 // dgamma_r += rowsum (own row) - colsum (all rows) for both dP o P and dA o A
                 atomicAdd(&acc_g[r], rowsum);
                 if (m >= 64) atomicAdd(&acc_b[r], bsum);
