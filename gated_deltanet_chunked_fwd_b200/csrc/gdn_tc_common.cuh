@@ -182,38 +182,46 @@ inline int sm_count() {
     return n > 0 ? n : 148;
 }
 
-// Segments of L chunks: count and estimated makespan in chunk-steps.
+// Segments of L chunks, except that the one segment of a sequence that starts exactly (it needs
+// no warm-up) takes up to `lead` chunks more: a sequence of c chunks has
+// max(1, ceil((c - lead) / L)) segments.  Count of CTAs over all sequences and value heads.
 struct SplitChoice {
     int L;
+    int lead;
     int64_t ctas;
 };
 
+inline int segments_of(int c, int L, int lead) { return std::max(1, (c - lead + L - 1) / L); }
+
+// lead_auto: the exact segment's extra chunks in auto mode (0 keeps every segment at L)
 inline SplitChoice choose_split(const std::vector<int>& nchunks, int Hv, int split_mode, int nsm,
-                                double warm_cost = 1.5) {
+                                double warm_cost = 1.5, int lead_auto = 0) {
     int maxc = 1;
     for (int c : nchunks) maxc = std::max(maxc, c);
-    auto count = [&](int L) {
+    auto count = [&](int L, int lead) {
         int64_t s = 0;
-        for (int c : nchunks) s += std::max(1, (c + L - 1) / L);
+        for (int c : nchunks) s += segments_of(c, L, lead);
         return s * Hv;
     };
-    if (split_mode == 1) return {maxc, count(maxc)};
+    if (split_mode == 1) return {maxc, 0, count(maxc, 0)};
     if (split_mode == 2) {
         const int L = std::max(1, std::min(maxc, 2));
-        return {L, count(L)};
+        return {L, 0, count(L, 0)};
     }
-    int bestL = maxc;
+    int bestL = maxc, bestLead = 0;
     double best = 1e300;
     for (int L = 1; L <= maxc; ++L) {
-        const int64_t S = count(L);
+        const int lead = L < maxc ? lead_auto : 0;
+        const int64_t S = count(L, lead);
         const double waves = std::ceil((double)S / nsm);
-        const double est = waves * (L + (L < maxc ? warm_cost : 0.0));
+        const double est = waves * (L + (L < maxc ? std::max(warm_cost, (double)lead) : 0.0));
         if (est < best - 1e-9 || (std::fabs(est - best) < 1e-9 && L > bestL)) {
             best = est;
             bestL = L;
+            bestLead = lead;
         }
     }
-    return {bestL, count(bestL)};
+    return {bestL, bestLead, count(bestL, bestLead)};
 }
 
 inline std::vector<int> chunk_counts(const Problem& p, const int32_t* cu_host) {

@@ -90,6 +90,7 @@ static_assert(kTimg + 2 * kTImgBytes <= kVec, "T images overlap the vectors");
 struct TcArgs {
     Problem p;
     int L;          // chunks per segment
+    int lead;       // extra chunks of a sequence's first segment (it needs no warm-up)
     int fixed_segs; // segments per sequence when cu_seqlens is absent
     int auto_warm;  // 1: gate-driven warm-up for segments that do not start a sequence
     float log_eps;  // warm-up stops once the summed log decay is <= log_eps
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m < p.N) {
                 b_m = p.cu[m];
                 l_m = max((int64_t)0, (int64_t)p.cu[m + 1] - b_m);
-                s_m = max(1, (nchunks_of(l_m) + args.L - 1) / args.L);
+                s_m = max(1, (nchunks_of(l_m) - args.lead + args.L - 1) / args.L);
             }
             int incl = s_m;
 #pragma unroll
@@ -169,8 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int hk = h / p.group;
     const int nck = nchunks_of(len);
-    const int c0 = min(nck, seg * args.L);
-    const int c1 = min(nck, (seg + 1) * args.L);
+    // segment seg owns chunks [c0, c1): the first one [0, lead + L), then L each
+    const int c0 = seg == 0 ? 0 : min(nck, args.lead + seg * args.L);
+    const int c1 = min(nck, args.lead + (seg + 1) * args.L);
 
     // ---- set-up: barriers, TMEM
     if (tid == 0) {
@@ -706,9 +708,12 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
     a.summ = (const float2*)(ws + wy_tc_summary_offset(p));
     a.himg = himg;
     const std::vector<int> nck = chunk_counts(p, cu_host);
-    const SplitChoice sc = choose_split(nck, p.Hv, split_mode, sm_count());
+    // the first segment of a sequence starts exactly, so it takes one chunk more than the others
+    // (a warm-up is at least one chunk)
+    const SplitChoice sc = choose_split(nck, p.Hv, split_mode, sm_count(), 1.5, 1);
     a.L = sc.L;
-    a.fixed_segs = p.cu ? 0 : std::max(1, (nck.empty() ? 1 : (nck[0] + sc.L - 1) / sc.L));
+    a.lead = sc.lead;
+    a.fixed_segs = p.cu ? 0 : (nck.empty() ? 1 : segments_of(nck[0], sc.L, sc.lead));
     a.auto_warm = split_mode == 1 ? 0 : 1;
     a.log_eps = (float)(-30.0 * std::log(2.0));
     CUtensorMap mq, mk, mv, mo;
