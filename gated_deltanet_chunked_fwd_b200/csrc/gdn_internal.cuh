@@ -84,9 +84,6 @@ gdn_status plan_fwd(const gdn_fwd_args* a, FwdPlan* plan);
 gdn_status launch_fwd_simt(const FwdPlan& plan, char* ws, cudaStream_t s);
 gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s);
 size_t tc_fwd_workspace(const Problem& p);
-// WY / UT step on its own: one bf16 T image per (chunk, value head), then per-chunk gate
-// summaries, into the workspace `ws`
-gdn_status launch_wy_tc(const Problem& p, uint8_t* ws, cudaStream_t s);
 size_t wy_tc_workspace(const Problem& p);
 size_t wy_tc_summary_offset(const Problem& p);
 // WY + fused kernel in replay mode: bf16 H^T entry-state image (32 KB) of every chunk, by

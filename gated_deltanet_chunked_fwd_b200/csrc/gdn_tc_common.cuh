@@ -19,9 +19,6 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int kLd = 68;   // row stride (floats) of the fp32 T matrix in the solve
-constexpr int kLdY = 20;  // row stride (floats) of the level scratch
-
 __device__ __forceinline__ int nchunks_of(int64_t len) { return (int)((len + kChunk - 1) / kChunk); }
 
 // Per-(chunk, value head) images in the workspace (bf16 T of the WY step, one 8 KB
@@ -83,93 +80,6 @@ __device__ __forceinline__ bool wg_or(int id, int cnt, bool pred) {
 // A (64 x 64, strictly lower) lives in As with float4 granules XOR-swizzled by row, so that a
 // warp writing 32 rows at one column, or reading 8 rows at one column, hits distinct banks.
 __device__ __forceinline__ int as_idx(int r, int s) { return r * 64 + ((((s >> 2) ^ (r & 15))) << 2) + (s & 3); }
-
-// Level-D merge of the blocked inverse (D = 1, 2, 3) over the blocks (i, i-D), i = D..3:
-//   Y = sum_{k=i-D}^{i-1} A_ik T_k,i-D   then   T_i,i-D = -T_ii Y.
-// T (in M, stride kLd) stores zeros above the diagonal of its diagonal blocks, so all sums
-// run over full blocks.  A task is one row of a block and 4 consecutive columns; the
-// j-range of Y is split over `kSplit` threads and combined with shuffles.
-template <int D, int NT>
-__device__ __forceinline__ void solve_level_Y(const float* As, const float* M, float* Ys, int t) {
-    constexpr int kTasks = (4 - D) * 64;  // (block, row, column quad)
-    constexpr int kSplit = NT / kTasks >= 4 ? 4 : (NT / kTasks >= 1 ? NT / kTasks : 1);  // 1, 2 or 4
-    constexpr int kLen = 16 * D / kSplit;
-    const int part = t % kSplit;
-#pragma unroll
-    for (int task = t / kSplit; task < kTasks; task += NT / kSplit) {
-        const int blk = task >> 6, rr = (task >> 2) & 15, quad = task & 3;
-        const int i = blk + D, j0 = i - D;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int jj = 0; jj < kLen; ++jj) {
-            const int j = part * kLen + jj;
-            const float a = As[as_idx(16 * i + rr, 16 * j0 + j)];
-            const float4 tv = *reinterpret_cast<const float4*>(M + (16 * j0 + j) * kLd + 16 * j0 + 4 * quad);
-            acc.x += a * tv.x;
-            acc.y += a * tv.y;
-            acc.z += a * tv.z;
-            acc.w += a * tv.w;
-        }
-#pragma unroll
-        for (int o = 1; o < kSplit; o <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
-        }
-        if (part == 0) *reinterpret_cast<float4*>(Ys + (blk * 16 + rr) * kLdY + 4 * quad) = acc;
-    }
-}
-
-template <int D, int NT>
-__device__ __forceinline__ void solve_level_T(float* M, const float* Ys, int t) {
-    constexpr int kTasks = (4 - D) * 64;
-#pragma unroll
-    for (int task = t; task < kTasks; task += NT) {
-        const int blk = task >> 6, rr = (task >> 2) & 15, quad = task & 3;
-        const int i = blk + D, j0 = i - D;
-        const float* trow = M + (16 * i + rr) * kLd + 16 * i;  // T_ii row rr (zeros above)
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-            const float4 tt = *reinterpret_cast<const float4*>(trow + 4 * j4);
-            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 y = *reinterpret_cast<const float4*>(Ys + (blk * 16 + 4 * j4 + e) * kLdY + 4 * quad);
-                acc.x += tv[e] * y.x;
-                acc.y += tv[e] * y.y;
-                acc.z += tv[e] * y.z;
-                acc.w += tv[e] * y.w;
-            }
-        }
-        *reinterpret_cast<float4*>(M + (16 * i + rr) * kLd + 16 * j0 + 4 * quad) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-}
-
-
-// Column cc of diagonal block b (threads 0..63): 16 x 16 unit lower-triangular inverse by
-// forward substitution, written with zeros above the diagonal.
-__device__ __forceinline__ void solve_diag(const float* As, float* M, int t) {
-    if (t < 64) {
-        const int b = t >> 4, cc = t & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
-#pragma unroll
-            for (int j = 0; j + 1 < r; j += 2) {
-                s0 -= As[as_idx(16 * b + r, 16 * b + j)] * x[j];
-                s1 -= As[as_idx(16 * b + r, 16 * b + j + 1)] * x[j + 1];
-            }
-            if (r & 1) s0 -= As[as_idx(16 * b + r, 16 * b + r - 1)] * x[r - 1];
-            x[r] = (r < cc) ? 0.f : s0 + s1;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) M[(16 * b + r) * kLd + 16 * b + cc] = x[r];
-    }
-}
 
 // ------------------------------------------------------------------- host side
 // Multi-SM split of the chunk chains (host side): chunks per sequence, and the segment length L
@@ -234,6 +144,10 @@ inline std::vector<int> chunk_counts(const Problem& p, const int32_t* cu_host) {
     }
     return v;
 }
+
+// WY / UT step on its own: one bf16 T image per (chunk, value head), then per-chunk gate
+// summaries, into the workspace `ws`; tm_k is k's tensor map (make_map below)
+gdn_status launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, cudaStream_t s);
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -13,11 +13,18 @@
 //
 // The work per chunk is small and latency-bound (a 64 x 64 x 128 Gram block and a 64 x 64
 // triangular inverse), so the kernel is built for many chunks in flight rather than for one
-// fast chunk: 128 threads and about 39 KB of shared memory per CTA, five CTAs per SM.  The
-// Gram block K K^T is formed with warp-level mma.sync (bf16 in, fp32 out): its fragments
-// stay in registers, where the gate scaling turns them into A without a TMEM round trip.
-// The inverse is blocked: the four 16 x 16 diagonal blocks by fp32 substitution, then three
-// merge levels on the tensor cores (warp mma.sync in tf32).
+// fast chunk: 128 threads, 72 registers and about 23 KB of shared memory per CTA, seven CTAs
+// per SM, so that a 4096-token, 16-head call (1024 chunks) runs as one wave.  The K tile
+// comes in by TMA.  The Gram block K K^T is formed with warp-level mma.sync (bf16 in, fp32
+// out): its fragments stay in registers, where the gate scaling turns them into A without a
+// TMEM round trip.  The inverse is blocked: the four 16 x 16 diagonal blocks by fp32
+// substitution, then three merge levels on the tensor cores (warp mma.sync in tf32).
+//
+// A and T share one fp32 64 x 64 array X: A is strictly lower and T unit lower-triangular,
+// so A sits below the diagonal and T (off its unit diagonal) above it, transposed:
+// X[r][s] = A[r][s] and X[s][r] = T[r][s] for r > s.  Every X entry that feeds a merge is
+// stored already rounded to tf32 (round to nearest, ties away), so the merges issue no
+// conversions; the diagonal blocks of A stay fp32 for the substitution.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -33,16 +40,17 @@ using namespace tc;
 namespace {
 
 constexpr int kWyThreads = 128;
-constexpr int kWyMinBlocks = 5;  // CTAs per SM the shared memory and registers are sized for
-// shared memory (bytes from a 128-aligned base)
-constexpr uint32_t wK = 0;                                 // 16 KB bf16 K [dk half][64 rows][128 B];
-                                                           // then fp32 A [64][kLd]
-constexpr uint32_t wM = 64 * kLd * 4;                      // fp32 [64][kLd] T
-constexpr uint32_t wYs = wM + 64 * kLd * 4;                // fp32 [4 warps][16][9] merge scratch
-constexpr uint32_t wVec = wYs + 3 * 16 * kLdY * 4;         // beta, gamma, a, b, |k|^2: 5 x 64 fp32
-constexpr uint32_t wSmemBytes = wVec + 5 * 64 * 4 + 128;   // + alignment slack
-static_assert(4 * 16 * 9 * 4 <= 3 * 16 * kLdY * 4, "merge scratch fits");
-static_assert(wSmemBytes * kWyMinBlocks + kWyMinBlocks * 1024 <= 228 * 1024, "five CTAs per SM");
+constexpr int kWyMinBlocks = 7;  // CTAs per SM the shared memory and registers are sized for
+constexpr int kXs = 72;          // row stride (floats) of X: conflict-free 64-bit fragment reads
+// shared memory (bytes from a 1024-aligned base: the TMA destination is 128-byte swizzled)
+constexpr uint32_t wK = 0;                          // 16 KB bf16 K [dk half][64 rows][128 B];
+                                                    // then fp32 X [64][kXs]
+constexpr uint32_t wYs = 64 * kXs * 4;              // fp32 [4 warps][16][9] merge scratch
+constexpr uint32_t wVec = wYs + 4 * 16 * 9 * 4;     // beta, gamma, a, b, |k|^2: 5 x 64 fp32
+constexpr uint32_t wBar = wVec + 5 * 64 * 4;        // mbarrier of the K tile
+constexpr uint32_t wSmemBytes = wBar + 16 + 1024;   // + alignment slack
+static_assert(wYs >= 16384, "X covers the K tile it replaces");
+static_assert(wSmemBytes * kWyMinBlocks + kWyMinBlocks * 1024 <= 228 * 1024, "CTAs per SM");
 
 // 4 8x8 b16 matrices from shared memory (lane groups of 8 give the row addresses of matrix 0..3)
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
@@ -60,98 +68,119 @@ __device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// fp32 -> tf32 (round to nearest, ties away), as the 32-bit pattern mma.sync reads
-__device__ __forceinline__ uint32_t to_tf32(float x) {
+// fp32 -> tf32 (round to nearest, ties away), kept as an fp32 value whose low 13 mantissa bits
+// are zero: mma.sync reads it as that tf32 value exactly.  In the merges this rounding adds a
+// relative error of about 1e-6 to T (|T - T_exact| / |T| over random chunks of the workloads'
+// distributions), some thirty times below the bf16 rounding that the T image gets afterwards.
+__device__ __forceinline__ float tf32r(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return __uint_as_float(r);
 }
 
-// D += A B for one 16 x 8 x 8 tile in tf32 (A row-major, B column-major, D fp32)
-__device__ __forceinline__ void mma_tf32(float* d, const uint32_t* a, const uint32_t* b) {
+// D += A B for one 16 x 8 x 8 tile in tf32 (A row-major, B column-major, D fp32); the operands
+// are tf32 values held in fp32 registers
+__device__ __forceinline__ void mma_tf32(float* d, float a0, float a1, float a2, float a3, float b0,
+                                         float b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+        : "r"(__float_as_uint(a0)), "r"(__float_as_uint(a1)), "r"(__float_as_uint(a2)),
+          "r"(__float_as_uint(a3)), "r"(__float_as_uint(b0)), "r"(__float_as_uint(b1)));
 }
 
-// D += A B with fp32 operands rounded to tf32.  In the merges below this adds a relative error
-// of about 1e-6 (|T - T_exact| / |T| over random chunks of the workloads' distributions), some
-// thirty times below the bf16 rounding that the T image gets afterwards.
-__device__ __forceinline__ void mma_tf32_rn(float* d, const float* a, const float* b) {
-    const uint32_t ar[4] = {to_tf32(a[0]), to_tf32(a[1]), to_tf32(a[2]), to_tf32(a[3])};
-    const uint32_t br[2] = {to_tf32(b[0]), to_tf32(b[1])};
-    mma_tf32(d, ar, br);
-}
+// T[r][s] given x = X[s][r] (the stored value when r > s): 1 on the diagonal, 0 above it
+__device__ __forceinline__ float t_sel(float x, int r, int s) { return r > s ? x : (r == s ? 1.f : 0.f); }
 
 // The four 16 x 16 diagonal blocks of T (threads 0..63: block t / 16, column t % 16): unit
-// lower-triangular inverse by forward substitution, written with zeros above the diagonal.
-// A and T are [64][kLd] row-major, so every A element is read at a compile-time offset from
-// the block origin.
-__device__ __forceinline__ void diag_inverse(const float* As, float* M, int t) {
-    if (t < 64) {
-        const int b = t >> 4, cc = t & 15;
-        const float* a = As + 16 * b * (kLd + 1);
-        float x[16];
+// lower-triangular inverse by forward substitution, reading each A row as 16-byte vectors.
+// Column cc of block b is T[16 b + r][16 b + cc] = x[r]; it is written to row 16 b + cc of X
+// once every thread has read its A block (the caller's barrier sits in between).
+__device__ __forceinline__ void diag_solve(const float* X, int t, float* x) {
+    const int b = t >> 4, cc = t & 15;
+    const float* a = X + 16 * b * (kXs + 1);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
+    for (int r = 0; r < 16; ++r) {
+        float row[16];
 #pragma unroll
-            for (int j = 0; j + 1 < r; j += 2) {
-                s0 -= a[r * kLd + j] * x[j];
-                s1 -= a[r * kLd + j + 1] * x[j + 1];
-            }
-            if (r & 1) s0 -= a[r * kLd + r - 1] * x[r - 1];
-            x[r] = (r < cc) ? 0.f : s0 + s1;
+        for (int q = 0; q < (r + 3) / 4; ++q) {
+            const float4 v = *reinterpret_cast<const float4*>(a + r * kXs + 4 * q);
+            row[4 * q] = v.x;
+            row[4 * q + 1] = v.y;
+            row[4 * q + 2] = v.z;
+            row[4 * q + 3] = v.w;
         }
-        float* m = M + 16 * b * (kLd + 1) + cc;
+        float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) m[r * kLd] = x[r];
+        for (int j = 0; j + 1 < r; j += 2) {
+            s0 -= row[j] * x[j];
+            s1 -= row[j + 1] * x[j + 1];
+        }
+        if (r & 1) s0 -= row[r - 1] * x[r - 1];
+        x[r] = (r < cc) ? 0.f : s0 + s1;
     }
+}
+
+__device__ __forceinline__ void diag_store(float* X, int t, const float* x) {
+    const int b = t >> 4, cc = t & 15;
+    float* m = X + (16 * b + cc) * kXs + 16 * b;  // entries left of the diagonal are no longer read
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<float4*>(m + 4 * q) =
+            make_float4(tf32r(x[4 * q]), tf32r(x[4 * q + 1]), tf32r(x[4 * q + 2]), tf32r(x[4 * q + 3]));
 }
 
 // Level D (1..3) of the blocked inverse on the tensor cores: for the blocks (i, j0 = i - D),
 //   Y = sum_{k = j0}^{i-1} A_ik T_k,j0,   T_i,j0 = -T_ii Y      (16 x 16 blocks)
 // A work unit is one 8-column half of one block (one m16n8 tile); warp w takes units w, w + 4.
+// In Y the k slots (t, t + 4) of lane (g, t) stand for the adjacent columns (2t, 2t + 1), so
+// that A and T come in as 64-bit pairs; in T_ii Y the M slots (g, g + 8) stand for the adjacent
+// rows (2g, 2g + 1), which makes both the T_ii fragment and the result 64-bit pairs in X.
 // Y goes from the accumulator layout to the B-operand layout through a per-warp 16 x 9 scratch.
 template <int D>
-__device__ __forceinline__ void merge_level(const float* As, float* M, float* ysw, int warp, int lane) {
+__device__ __forceinline__ void merge_level(float* X, float* ysw, int warp, int lane) {
     constexpr int kUnits = 2 * (4 - D);
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int u = warp; u < kUnits; u += 4) {
         const int i = D + (u >> 1), j0 = i - D, col = 16 * j0 + 8 * (u & 1);
-        const int r0 = 16 * i + g, r1 = r0 + 8;
+        const int r0 = 16 * i + g;
         float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kb = 0; kb < D; ++kb) {
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
-                const int kc = 16 * (j0 + kb) + 8 * ks;
-                const float a[4] = {As[r0 * kLd + kc + t], As[r1 * kLd + kc + t],
-                                    As[r0 * kLd + kc + t + 4], As[r1 * kLd + kc + t + 4]};
-                const float b[2] = {M[(kc + t) * kLd + col + g], M[(kc + t + 4) * kLd + col + g]};
-                mma_tf32_rn(y, a, b);
+                const int kc = 16 * (j0 + kb) + 8 * ks + 2 * t;
+                const float2 a0 = *reinterpret_cast<const float2*>(X + r0 * kXs + kc);
+                const float2 a1 = *reinterpret_cast<const float2*>(X + (r0 + 8) * kXs + kc);
+                float2 bv = *reinterpret_cast<const float2*>(X + (col + g) * kXs + kc);
+                if (kb == 0) {  // T block (j0, j0) is the diagonal one
+                    bv.x = t_sel(bv.x, kc, col + g);
+                    bv.y = t_sel(bv.y, kc + 1, col + g);
+                }
+                mma_tf32(y, a0.x, a1.x, a0.y, a1.y, bv.x, bv.y);
             }
         }
-        ysw[g * 9 + 2 * t] = y[0];
-        ysw[g * 9 + 2 * t + 1] = y[1];
-        ysw[(g + 8) * 9 + 2 * t] = y[2];
-        ysw[(g + 8) * 9 + 2 * t + 1] = y[3];
+        ysw[g * 9 + 2 * t] = tf32r(y[0]);
+        ysw[g * 9 + 2 * t + 1] = tf32r(y[1]);
+        ysw[(g + 8) * 9 + 2 * t] = tf32r(y[2]);
+        ysw[(g + 8) * 9 + 2 * t + 1] = tf32r(y[3]);
         __syncwarp();
+        const int rr = 16 * i + 2 * g;  // rows rr, rr + 1 of T_ii
         float r[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
-            const int kc = 16 * i + 8 * ks;
-            const float a[4] = {M[r0 * kLd + kc + t], M[r1 * kLd + kc + t], M[r0 * kLd + kc + t + 4],
-                                M[r1 * kLd + kc + t + 4]};
-            const float b[2] = {ysw[(8 * ks + t) * 9 + g], ysw[(8 * ks + t + 4) * 9 + g]};
-            mma_tf32_rn(r, a, b);
+            const int kc = 16 * i + 8 * ks + t;
+            const float2 p0 = *reinterpret_cast<const float2*>(X + kc * kXs + rr);
+            const float2 p1 = *reinterpret_cast<const float2*>(X + (kc + 4) * kXs + rr);
+            mma_tf32(r, t_sel(p0.x, rr, kc), t_sel(p0.y, rr + 1, kc), t_sel(p1.x, rr, kc + 4),
+                     t_sel(p1.y, rr + 1, kc + 4), ysw[(8 * ks + t) * 9 + g], ysw[(8 * ks + t + 4) * 9 + g]);
         }
         __syncwarp();  // the scratch is rewritten by this warp's next unit
-        *reinterpret_cast<float2*>(M + r0 * kLd + col + 2 * t) = make_float2(-r[0], -r[1]);
-        *reinterpret_cast<float2*>(M + r1 * kLd + col + 2 * t) = make_float2(-r[2], -r[3]);
+        // T block (i, j0), transposed into X above the diagonal
+        *reinterpret_cast<float2*>(X + (col + 2 * t) * kXs + rr) = make_float2(tf32r(-r[0]), tf32r(-r[2]));
+        *reinterpret_cast<float2*>(X + (col + 2 * t + 1) * kXs + rr) = make_float2(tf32r(-r[1]), tf32r(-r[3]));
     }
 }
 
@@ -181,9 +210,10 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
 }
 
 __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
-    gdn_wy_tc_kernel(const Problem p, uint8_t* __restrict__ timg, float2* __restrict__ summ) {
+    gdn_wy_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const Problem p, uint8_t* __restrict__ timg,
+                     float2* __restrict__ summ) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     // the forward's state-chain kernel may be scheduled as soon as every CTA of this grid has
     // started (it waits for this grid's completion before reading the images)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -194,21 +224,25 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     if (!locate_slot(p, blockIdx.x, &n, &c, &bos, &len)) return;  // CTA-uniform
     const int64_t t0 = bos + (int64_t)c * kChunk;
     const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
+    uint64_t* bar = (uint64_t*)(sm + wBar);
 
-    // ---- K tile -> shared memory, 128-byte swizzled; rows past the chunk are zero
-    {
-        const uint4* kg = reinterpret_cast<const uint4*>(p.k);
-        uint4 u[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int L = i * kWyThreads + tid, r = L >> 4, ch = L & 15;
-            u[i] = r < lc ? __ldg(kg + ((t0 + r) * p.Hk + hk) * 16 + ch) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int L = i * kWyThreads + tid, r = L >> 4, ch = L & 15;
-            *reinterpret_cast<uint4*>(sm + wK + (ch >> 3) * 8192 + sw128_off(r, ch & 7)) = u[i];
-        }
+    // ---- K tile by TMA ([dk half][64 rows][128 B], 128-byte swizzled).  Rows past the chunk
+    // (the next sequence's tokens, or zeros past the tensor's end) only reach entries of A that
+    // the mask below sets to zero.  The chunk's gates are loaded meanwhile.
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+    }
+    float x = 0.f, bt = 0.f;
+    if (tid < lc) {  // lc <= 64
+        x = p.g[(t0 + tid) * Hv + h];
+        bt = p.beta[(t0 + tid) * Hv + h];
+    }
+    __syncthreads();  // the barrier is initialised
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar, 16384);
+        tma_load_3d(sm + wK, &tm_k, bar, 0, hk, (int)t0);
+        tma_load_3d(sm + wK + 8192, &tm_k, bar, 64, hk, (int)t0);
     }
 
     // ---- gates: gamma = cumsum g (two warp scans), E_rs = a_r b_s when factorable
@@ -219,8 +253,6 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     float* vnrm = vbeta + 256;
     float gr = 0.f;
     if (tid < 64) {
-        float x = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;
-        const float bt = tid < lc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -257,7 +289,11 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     float acc[5][4];
 #pragma unroll
     for (int i = 0; i < 5; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    __syncthreads();  // K tile, vectors
+    __syncthreads();  // vectors
+    if (!__syncthreads_and(mbar_wait(bar, 0))) {  // the K tile has landed (bounded wait)
+        if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
+        return;
+    }
     {
         const uint32_t sK = smem_u32(sm + wK);
 #pragma unroll
@@ -287,34 +323,52 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
             }
         }
     }
-    __syncthreads();  // every warp is done with the K tile: A overwrites it
+    __syncthreads();  // every warp is done with the K tile: X overwrites it
 
-    // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> shared memory (fp32); the diagonal of
-    // K K^T gives |k_r|^2 for the chunk summary
-    float* As = (float*)(sm + wK);
-#pragma unroll
-    for (int i = 0; i < 5; ++i) {
-        const bool inA = i < nA;
-        const int m = inA ? mA : mB, j = inA ? jA + i : jB + (i - nA);
+    // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> X (entries on and above the diagonal
+    // that a tile covers are written as zeros and later overwritten by T).  Blocks below the
+    // diagonal block are merge operands only: stored rounded to tf32.  The diagonal of K K^T
+    // gives |k_r|^2 for the chunk summary.
+    float* X = (float*)(sm + wK);
+    {
+        float arA[2], brA[2], arB[2], brB[2];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
-            const int r = 16 * m + g8 + 8 * hr, s = 8 * j + 2 * t4;
-            const float ar = va[r], br = vbeta[r];
+            arA[hr] = va[16 * mA + g8 + 8 * hr];
+            brA[hr] = vbeta[16 * mA + g8 + 8 * hr];
+            arB[hr] = va[16 * mB + g8 + 8 * hr];
+            brB[hr] = vbeta[16 * mB + g8 + 8 * hr];
+        }
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            const bool inA = i < nA;
+            const int m = inA ? mA : mB, j = inA ? jA + i : jB + (i - nA);
+            const int s = 8 * j + 2 * t4;
+            const bool below = (j >> 1) < m;  // warp-uniform
             const float2 b2 = *reinterpret_cast<const float2*>(vb + s);
-            float e0, e1;
-            if (fac) {  // block-uniform
-                e0 = ar * b2.x;
-                e1 = ar * b2.y;
-            } else {
-                e0 = exp2f(ar - b2.x);
-                e1 = exp2f(ar - b2.y);
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = 16 * m + g8 + 8 * hr;
+                const float ar = inA ? arA[hr] : arB[hr], br = inA ? brA[hr] : brB[hr];
+                float e0, e1;
+                if (fac) {  // block-uniform
+                    e0 = ar * b2.x;
+                    e1 = ar * b2.y;
+                } else {
+                    e0 = exp2f(ar - b2.x);
+                    e1 = exp2f(ar - b2.y);
+                }
+                float2 w;
+                w.x = (s < r && r < lc) ? br * acc[i][2 * hr] * e0 : 0.f;
+                w.y = (s + 1 < r && r < lc) ? br * acc[i][2 * hr + 1] * e1 : 0.f;
+                if (below) {
+                    w.x = tf32r(w.x);
+                    w.y = tf32r(w.y);
+                }
+                *reinterpret_cast<float2*>(X + r * kXs + s) = w;
+                if (s == r) vnrm[r] = acc[i][2 * hr];
+                if (s + 1 == r) vnrm[r] = acc[i][2 * hr + 1];
             }
-            float2 w;
-            w.x = (s < r && r < lc) ? br * acc[i][2 * hr] * e0 : 0.f;
-            w.y = (s + 1 < r && r < lc) ? br * acc[i][2 * hr + 1] * e1 : 0.f;
-            *reinterpret_cast<float2*>(As + r * kLd + s) = w;
-            if (s == r) vnrm[r] = acc[i][2 * hr];
-            if (s + 1 == r) vnrm[r] = acc[i][2 * hr + 1];
         }
     }
     // Chunk summary for the forward's gate-driven split: the summed log decay of the chunk and
@@ -324,38 +378,50 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     if (tid == 63) summ[img_slot(bos, n, c) * Hv + h] = make_float2(gr, viol ? 1.f : 0.f);
 
     // ---- T = (I + A)^-1: diagonal 16 x 16 blocks, then three merge levels
-    float* M = (float*)(sm + wM);
-    float* Ys = (float*)(sm + wYs);
-    diag_inverse(As, M, tid);
+    {
+        float xs[16];
+        if (tid < 64) diag_solve(X, tid, xs);
+        __syncthreads();  // every diagonal A block has been read
+        if (tid < 64) diag_store(X, tid, xs);
+    }
     __syncthreads();
-    float* ysw = Ys + warp * 16 * 9;
-    merge_level<1>(As, M, ysw, warp, lane);
+    float* ysw = (float*)(sm + wYs) + warp * 16 * 9;
+    merge_level<1>(X, ysw, warp, lane);
     __syncthreads();
-    merge_level<2>(As, M, ysw, warp, lane);
+    merge_level<2>(X, ysw, warp, lane);
     __syncthreads();
-    merge_level<3>(As, M, ysw, warp, lane);
+    merge_level<3>(X, ysw, warp, lane);
     __syncthreads();
 
-    // ---- bf16 image: thread = (row nr, half of the columns); zeros above the diagonal
+    // ---- bf16 image: thread = rows nr4 .. nr4 + 3, columns s0 .. s0 + 7 (one 16-byte chunk of
+    // each row), from T[r][s] = X[s][r] for r > s
     {
-        const int nr = tid >> 1, hf = tid & 1;
+        const int nr4 = 4 * (tid & 15), ch = tid >> 4, s0 = 8 * ch;
         uint8_t* img = timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kTImgBytes;
+        float v[4][8];
+        if (s0 > nr4 + 3) {  // the block lies above the diagonal
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            const int chunk = 4 * hf + cc, s0 = 8 * chunk;
-            const float4 x0 = *reinterpret_cast<const float4*>(M + nr * kLd + s0);
-            const float4 x1 = *reinterpret_cast<const float4*>(M + nr * kLd + s0 + 4);
-            float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = (s0 + e <= nr) ? v[e] : 0.f;
-            *reinterpret_cast<uint4*>(img + sw128_off(nr, chunk)) = pack8(v);
+                for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float4 col = *reinterpret_cast<const float4*>(X + (s0 + e) * kXs + nr4);
+                v[0][e] = t_sel(col.x, nr4, s0 + e);
+                v[1][e] = t_sel(col.y, nr4 + 1, s0 + e);
+                v[2][e] = t_sel(col.z, nr4 + 2, s0 + e);
+                v[3][e] = t_sel(col.w, nr4 + 3, s0 + e);
+            }
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(img + sw128_off(nr4 + q, ch)) = pack8(v[q]);
     }
 }
 
 }  // namespace
 
-gdn_status launch_wy_tc(const Problem& p, uint8_t* ws, cudaStream_t s) {
+gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, cudaStream_t s) {
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
@@ -363,7 +429,8 @@ gdn_status launch_wy_tc(const Problem& p, uint8_t* ws, cudaStream_t s) {
                              (int)wSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     const dim3 grid((unsigned)slots, (unsigned)p.Hv);
-    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(p, ws, (float2*)(ws + wy_tc_summary_offset(p)));
+    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws,
+                                                          (float2*)(ws + wy_tc_summary_offset(p)));
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
