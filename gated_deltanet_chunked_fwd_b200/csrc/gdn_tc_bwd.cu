@@ -65,6 +65,8 @@ constexpr uint32_t bHt = 81920;    // 32 KB bf16 H^T [dk atom][128 dv rows][128 
 constexpr uint32_t bT = 114688;    // 8 KB  T [64 rows s][64 r]; later S = G + G^T [s][j]
 constexpr uint32_t bBw = 122880;   // 8 KB  T diag(beta Gam); later diag(Gam) Q [atom][64][128]
 constexpr uint32_t bBu = 131072;   // 8 KB  T diag(beta)      (over Bw + Bu)
+// T, Bw, Bu arrive together: one copy of the WY step's three images
+static_assert(bBw == bT + kTImgBytes && bBu == bBw + kTImgBytes, "WY images are contiguous");
 constexpr uint32_t bP = 139264;    // 8 KB  P [64 r][64 s]; later dP o E
 constexpr uint32_t bWt = 147456;   // 16 KB -W^T [128 dk rows][64 s]; later -TdU^T [128 dv rows][64 r]
 constexpr uint32_t bUt = 163840;   // 16 KB U^T [128 dv rows][64 s]
@@ -75,12 +77,11 @@ constexpr uint32_t bBar = bRed + 2048;
 constexpr uint32_t kSmemB = bBar + 64 + 1024;
 
 constexpr uint32_t kHImg = 32768;  // bytes of one saved H^T image
-constexpr uint32_t kTImg = 8192;   // bytes of one saved T image
 
 struct TcBwdArgs {
     BwdProblem b;
     const uint8_t* himg;  // H^T entry-state images, by (image slot, value head)
-    const uint8_t* timg;  // T images of the WY step, by (image slot, value head)
+    const uint8_t* timg;  // T / Bw / Bu images of the WY step, by (image slot, value head)
     const float2* summ;   // per (image slot, value head): summed log decay, norm-condition flag
     float* dqw;           // [T_total][Hv][dk] per-value-head dq
     float* dkw;           // [T_total][Hv][dk] per-value-head dk
@@ -323,11 +324,13 @@ __global__ void __launch_bounds__(kNT, 1)
             }
         }
     };
-    // q, k, v, dO tiles and the T image of chunk c; the H image too for the chunks that emit
+    // q, k, v, dO tiles and the T / Bw / Bu images of chunk c; the H image too for the chunks
+    // that emit.  The buffers' last generic reads and writes were before the caller's barrier.
     auto load_qkv = [&](int c, bool with_h) {
         if (tid == 0) {
             const int t0 = (int)(bos + (int64_t)c * kChunk);
-            mbar_arrive_expect_tx(bar_ld, 65536 + kTImg + (with_h ? kHImg : 0));
+            fence_proxy_async();
+            mbar_arrive_expect_tx(bar_ld, 65536 + kWyImgBytes + (with_h ? kHImg : 0));
             for (int a = 0; a < 2; ++a) {
                 tma_load_3d(sm + bQK + a * 16384, &tm_q, bar_ld, 64 * a, hk, t0);
                 tma_load_3d(sm + bQK + a * 16384 + 8192, &tm_k, bar_ld, 64 * a, hk, t0);
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(kNT, 1)
             }
             const int64_t gi = img_slot(bos, n, c) * Hv + h;
             if (with_h) bulk_load(sm + bHt, args.himg + gi * kHImg, kHImg, bar_ld);
-            bulk_load(sm + bT, args.timg + gi * kTImg, kTImg, bar_ld);
+            bulk_load(sm + bT, args.timg + gi * kWyImgBytes, kWyImgBytes, bar_ld);
         }
     };
 
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kNT, 1)
         __syncthreads();
         mma1();
         if (!(ok = mma_sync_wait())) break;
-        // P (rows 0..63) -> smem; Bw, Bu from the T image
+        // P (rows 0..63) -> smem
         if (m < 64) {  // P row m, this thread's half of the columns
             const int r = m;
             float v[32], E[32];
@@ -396,28 +399,6 @@ __global__ void __launch_bounds__(kNT, 1)
                 v[e] = (s <= r && r < lc) ? v[e] * E[e] : 0.f;
             }
             store_row32(sm + bP, r, 4 * hh, v);
-        }
-        {  // row nrow, columns [16 q, 16 q + 16)
-            const int nrow = tid >> 2, q = tid & 3;
-            float vw[16], vu[16];
-#pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-                const uint4 u = *reinterpret_cast<const uint4*>(sm + bT + sw128_off(nrow, 2 * q + hc));
-                const __nv_bfloat162* t2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    const float2 f = __bfloat1622float2(t2[e2]);
-                    const int e = 8 * hc + 2 * e2, s = 16 * q + e;
-                    vw[e] = f.x * vbG[s];
-                    vw[e + 1] = f.y * vbG[s + 1];
-                    vu[e] = f.x * vbeta[s];
-                    vu[e + 1] = f.y * vbeta[s + 1];
-                }
-            }
-            *reinterpret_cast<uint4*>(sm + bBw + sw128_off(nrow, 2 * q)) = pack8(vw);
-            *reinterpret_cast<uint4*>(sm + bBw + sw128_off(nrow, 2 * q + 1)) = pack8(vw + 8);
-            *reinterpret_cast<uint4*>(sm + bBu + sw128_off(nrow, 2 * q)) = pack8(vu);
-            *reinterpret_cast<uint4*>(sm + bBu + sw128_off(nrow, 2 * q + 1)) = pack8(vu + 8);
         }
         fence_proxy_async();
         tc_fence_before();

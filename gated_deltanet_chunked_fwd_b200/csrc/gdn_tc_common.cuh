@@ -21,12 +21,14 @@ using namespace sm100;
 
 __device__ __forceinline__ int nchunks_of(int64_t len) { return (int)((len + kChunk - 1) / kChunk); }
 
-// Per-(chunk, value head) images in the workspace (bf16 T of the WY step, one 8 KB
-// 128-byte-swizzled 64 x 64 tile each) are addressed by a slot: chunk c of sequence n, which
-// starts at token bos, has slot floor(bos / 64) + n + c.  Slots of different chunks never
+// Per-(chunk, value head) images in the workspace are addressed by a slot: chunk c of
+// sequence n, which starts at token bos, has slot floor(bos / 64) + n + c.  The WY step writes
+// three bf16 64 x 64 tiles per (slot, value head), each 8 KB and 128-byte-swizzled [n][s]:
+// T, then Bw = T diag(beta Gam), then Bu = T diag(beta).  Slots of different chunks never
 // coincide (a sequence's chunks end at most one slot past floor(end / 64) + n, and the next
 // sequence starts at floor(end / 64) + n + 1), and every slot is below img_slots().
-constexpr uint32_t kTImgBytes = 8192;
+constexpr uint32_t kTImgBytes = 8192;                // one 64 x 64 bf16 tile
+constexpr uint32_t kWyImgBytes = 3 * kTImgBytes;     // T, Bw, Bu of one (slot, value head)
 __host__ __device__ __forceinline__ int64_t img_slot(int64_t bos, int n, int c) {
     return bos / kChunk + n + c;
 }

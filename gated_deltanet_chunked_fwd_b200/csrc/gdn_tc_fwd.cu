@@ -50,8 +50,9 @@ using namespace tc;
 namespace {
 
 // Two groups of warps run a two-stage software pipeline over the chunks of a segment:
-//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T, P,
-//                                       Bw / Bu from the T image, W^T and Ut^T, W^T -> smem
+//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T, P and
+//                                       diag(Gam) Q, W^T and Ut^T (Bw / Bu images of the WY
+//                                       step as B operands), W^T -> smem
 //   group S (threads 256-383, 4 warps)  the state chain of chunk k-1..k: U^T = Ut^T - H^T W^T,
 //                                       H^T <- Gam_n H^T + (U^T diag(decay)) K, outputs, bf16 H
 // Each group has one tcgen05 issuer (threads 0 and 256) and its own commit
@@ -75,17 +76,16 @@ constexpr uint32_t kColHb = 448;  // bf16 H^T, A operand (K pairs per column) [4
 constexpr uint32_t kStageQK = 0;       // 2 x 32 KB: [dk atom][q rows 0-63 | k rows 64-127][128 B]
 constexpr uint32_t kStageV = 65536;    // 2 x 16 KB: [dv atom][64 rows][128 B]
 constexpr uint32_t kPt = 98304;        // 2 x 8 KB  P: [64 n rows][64 s], by chunk parity
-constexpr uint32_t kBw = 114688;       // 8 KB   T diag(beta Gam): [n][s]
-constexpr uint32_t kBu = 122880;       // 8 KB   T diag(beta): [n][s]
-constexpr uint32_t kWt = 131072;       // 16 KB  W^T: [128 dk rows][64 tokens]
-constexpr uint32_t kTimg = 147456;     // 2 x 8 KB  bf16 T images [n][s], by chunk parity
+constexpr uint32_t kBwu = 114688;      // 2 x 16 KB  Bw = T diag(beta Gam), Bu = T diag(beta)
+                                       // ([n][s] each, 8 KB apart), by chunk parity
+constexpr uint32_t kWt = 147456;       // 16 KB  W^T: [128 dk rows][64 tokens]
 constexpr uint32_t kVec = 163840;      // 4 x 2 KB of per-token vectors, by chunk index mod 4
 constexpr uint32_t kVecStride = 512;   // floats per buffer
 constexpr uint32_t kOst = kVec + 4 * kVecStride * 4;  // 16 KB bf16 o tile [dv atom][64 tokens][128 B]
 constexpr uint32_t kRed = kOst + 16384;                // 16 floats
 constexpr uint32_t kBar = kRed + 64;   // 9 mbarriers + TMEM base
 constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
-static_assert(kTimg + 2 * kTImgBytes <= kVec, "T images overlap the vectors");
+static_assert(kBwu + 4 * kTImgBytes <= kWt && kWt + 16384 <= kVec, "shared-memory regions overlap");
 
 struct TcArgs {
     Problem p;
@@ -94,7 +94,7 @@ struct TcArgs {
     int fixed_segs; // segments per sequence when cu_seqlens is absent
     int auto_warm;  // 1: gate-driven warm-up for segments that do not start a sequence
     float log_eps;  // warm-up stops once the summed log decay is <= log_eps
-    const uint8_t* timg;  // T images of the WY step, by (image slot, value head)
+    const uint8_t* timg;  // T / Bw / Bu images of the WY step, by (image slot, value head)
     const float2* summ;   // per (image slot, value head): summed log decay, norm-condition flag
     uint8_t* himg;        // replay mode (backward): bf16 H^T entry-state image per own chunk, by
                           // (image slot, value head); no outputs.  nullptr: the forward
@@ -241,15 +241,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t0 = (int)(bos + (int64_t)c * kChunk);
         uint8_t* qk = sm + kStageQK + stage * 32768;
         uint8_t* vv = sm + kStageV + stage * 16384;
-        mbar_arrive_expect_tx(&bar_tma[stage], 49152 + kTImgBytes);
+        mbar_arrive_expect_tx(&bar_tma[stage], 49152 + 2 * kTImgBytes);
         for (int a = 0; a < 2; ++a) {
             tma_load_3d(qk + a * 16384, &tm_q, &bar_tma[stage], 64 * a, hk, t0);
             tma_load_3d(qk + a * 16384 + 8192, &tm_k, &bar_tma[stage], 64 * a, hk, t0);
             tma_load_3d(vv + a * 8192, &tm_v, &bar_tma[stage], 64 * a, h, t0);
         }
-        bulk_load(sm + kTimg + stage * kTImgBytes,
-                  args.timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kTImgBytes, kTImgBytes,
-                  &bar_tma[stage]);
+        bulk_load(sm + kBwu + stage * 2 * kTImgBytes,
+                  args.timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kWyImgBytes + kTImgBytes,
+                  2 * kTImgBytes, &bar_tma[stage]);  // Bw and Bu
     };
 
     if (tid == 0) {
@@ -276,20 +276,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Gates run one chunk ahead in warp 2 (lane l: rows 2l, 2l+1), so chunk k+1's vectors
         // are in shared memory before chunk k is handed to group S.  g / beta of the chunk after
         // that are prefetched into registers.
-        float gx0 = 0.f, gx1 = 0.f, bx0 = 0.f, bx1 = 0.f;
+        float gx0 = 0.f, gx1 = 0.f;
         auto load_gates = [&](int kk) {
             const int cc = cstart + kk;
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lcc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
             const int r0 = 2 * lane;
-            gx0 = r0 < lcc ? p.g[(t0 + r0) * Hv + h] : 0.f;  // padding: g = 0, beta = 0
+            gx0 = r0 < lcc ? p.g[(t0 + r0) * Hv + h] : 0.f;  // padding: g = 0
             gx1 = r0 + 1 < lcc ? p.g[(t0 + r0 + 1) * Hv + h] : 0.f;
-            bx0 = r0 < lcc ? p.beta[(t0 + r0) * Hv + h] : 0.f;
-            bx1 = r0 + 1 < lcc ? p.beta[(t0 + r0 + 1) * Hv + h] : 0.f;
         };
-        // vectors of chunk kk (buffer kk mod 4): beta, gamma = cumsum g, Gam = exp(gamma),
-        // beta Gam, decay to the chunk end exp(gamma_n - gamma), the E factors a, b, and the
-        // flag that says whether E_rs = a_r b_s (every |gamma - gamma_31| < 80) or exp2(a_r - b_s)
+        // vectors of chunk kk (buffer kk mod 4; beta enters through the Bw / Bu images): gamma =
+        // cumsum g, Gam = exp(gamma), decay to the chunk end exp(gamma_n - gamma), the E factors
+        // a, b, and the flag that says whether E_rs = a_r b_s (every |gamma - gamma_31| < 80) or
+        // exp2(a_r - b_s)
         auto gates = [&](int kk) {
             float* vec = (float*)(sm + kVec) + (kk & 3) * kVecStride;
             float incl = gx0 + gx1;
@@ -305,10 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float LOG2E = 1.4426950408889634f;
             const float e0 = expf(g0), e1 = expf(g1);
             const int r0 = 2 * lane;
-            *reinterpret_cast<float2*>(vec + r0) = make_float2(bx0, bx1);
             *reinterpret_cast<float2*>(vec + 64 + r0) = make_float2(g0, g1);
             *reinterpret_cast<float2*>(vec + 128 + r0) = make_float2(e0, e1);
-            *reinterpret_cast<float2*>(vec + 192 + r0) = make_float2(bx0 * e0, bx1 * e1);
             *reinterpret_cast<float2*>(vec + 256 + r0) = make_float2(expf(gl - g0), expf(gl - g1));
             *reinterpret_cast<float2*>(vec + 320 + r0) =
                 fac ? make_float2(expf(g0 - gm), expf(g1 - gm)) : make_float2(g0 * LOG2E, g1 * LOG2E);
@@ -329,9 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t sV = sbase + kStageV + stage * 16384;
+            const uint32_t sBwu = sbase + kBwu + stage * 2 * kTImgBytes;
             const float* vec = (const float*)(sm + kVec) + (k & 3) * kVecStride;
-            const float* vbeta = vec;
-            const float* vbG = vec + 192;
             const float* va = vec + 320;
             const float* vb = vec + 384;
 
@@ -363,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool fac = vec[448] != 0.f;
 
             // P (TMEM lanes 0..63: warps 0, 1, 4, 5, columns [32 hf, 32 hf + 32)) and, meanwhile,
-            // the B operands of MMA_W / MMA_U from the T image (warps 2, 3, 6, 7):
-            // Bw = T diag(beta Gam), Bu = T diag(beta), in the image's swizzled layout
+            // Q rows <- Gam_n Q rows in place (warps 2, 3, 6, 7; MMA1 has read Q): the B operand
+            // of MMA_O, so that H^T (diag(Gam) Q)^T and U^T P^T accumulate into one buffer
             if ((warp & 3) < 2) {
                 if (emit) {
                     float v[32];
@@ -397,39 +393,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     store_row32(sm + kPt + stage * 8192, r, 4 * hf, v);
                 }
-            } else {
+            } else if (emit) {
                 const int li = ((warp >> 2) << 6) | ((warp & 1) << 5) | lane;  // 0..127
-                const int nr = li >> 1, c0 = 4 * (li & 1);
-                const uint8_t* timg_s = sm + kTimg + stage * kTImgBytes;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int chunk = c0 + cc;
-                    const uint32_t off = sw128_off(nr, chunk);
-                    uint4 u = *reinterpret_cast<const uint4*>(timg_s + off);
-                    const __nv_bfloat162* t2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-                    float tv[8], vw[8], vu[8];
+                const int srow = li >> 1;
+                uint8_t* qrow = sm + kStageQK + stage * 32768 + (li & 1) * 16384 + srow * 128;
+                const float gmul = vec[128 + srow];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(t2[e]);
-                        tv[2 * e] = f.x;
-                        tv[2 * e + 1] = f.y;
-                    }
-                    const float4 g0 = *reinterpret_cast<const float4*>(vbG + 8 * chunk);
-                    const float4 g1 = *reinterpret_cast<const float4*>(vbG + 8 * chunk + 4);
-                    const float4 b0 = *reinterpret_cast<const float4*>(vbeta + 8 * chunk);
-                    const float4 b1 = *reinterpret_cast<const float4*>(vbeta + 8 * chunk + 4);
-                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                    const float bb8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                for (int i8 = 0; i8 < 8; ++i8) {
+                    const int c8 = (i8 + srow) & 7;  // rotated: rows spread over banks
+                    uint4 u = *reinterpret_cast<uint4*>(qrow + 16 * c8);
+                    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        vw[e] = tv[e] * gg[e];
-                        vu[e] = tv[e] * bb8[e];
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float2 f = __bfloat1622float2(b2[e2]);
+                        b2[e2] = __floats2bfloat162_rn(f.x * gmul, f.y * gmul);
                     }
-                    *reinterpret_cast<uint4*>(sm + kBw + off) = pack8(vw);
-                    *reinterpret_cast<uint4*>(sm + kBu + off) = pack8(vu);
+                    *reinterpret_cast<uint4*>(qrow + 16 * c8) = u;
                 }
             }
-            fence_proxy_async();  // Pt, Bw, Bu are read by the tensor core
+            fence_proxy_async();  // Pt and diag(Gam) Q are read by the tensor core
             tc_fence_before();
             wg_sync(1, kThreadsP);
 
@@ -438,9 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
-                                desc_sw128(sbase + kBw + j * 32, 16, 1024), id_mn_n64, j > 0);
+                                desc_sw128(sBwu + j * 32, 16, 1024), id_mn_n64, j > 0);
                     mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
-                                desc_sw128(sbase + kBu + j * 32, 16, 1024), id_mn_n64, j > 0);
+                                desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
                 }
                 mma_commit(bar_mma_p);
             }
@@ -459,24 +441,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] = -v[e];  // MMA_HW accumulates -H^T W^T
                 store_row32(sm + kWt, row, 4 * hf, v);
-            }
-            if (emit) {  // Q rows <- Gam_n Q rows, in place (MMA1 has read Q): B operand of MMA_O,
-                         // so that H^T (diag(Gam) Q)^T and U^T P^T accumulate into one buffer
-                const int srow = t >> 2, q = t & 3;
-                uint8_t* qrow = sm + kStageQK + stage * 32768 + (q >> 1) * 16384 + srow * 128;
-                const float gmul = vec[128 + srow];
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int c8 = 4 * (q & 1) + ((i4 + srow) & 3);  // rotated: rows spread over banks
-                    uint4 u = *reinterpret_cast<uint4*>(qrow + 16 * c8);
-                    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(b2[e]);
-                        b2[e] = __floats2bfloat162_rn(f.x * gmul, f.y * gmul);
-                    }
-                    *reinterpret_cast<uint4*>(qrow + 16 * c8) = u;
-                }
             }
             fence_proxy_async();
             tc_fence_before();

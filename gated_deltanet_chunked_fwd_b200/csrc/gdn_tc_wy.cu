@@ -2,11 +2,11 @@
 // dk = 128 on sm_100a: for every (chunk, value head), independently of the state,
 //   gamma = in-chunk cumsum of g,   E_rs = exp(gamma_r - gamma_s),
 //   A     = strictly-lower(diag(beta) (K K^T o E)),
-//   T     = (I + A)^-1,
-// written to the workspace as one bf16 64 x 64 image per (chunk, value head) in the
+//   T     = (I + A)^-1,   Bw = T diag(beta Gam),   Bu = T diag(beta)   (Gam = exp(gamma)),
+// written to the workspace as three bf16 64 x 64 images per (chunk, value head) in the
 // 128-byte-swizzled layout that tcgen05 reads as an MMA operand (row n, 16-byte chunk c at
-// chunk position c ^ (n & 7)).  The forward's state chain then forms
-// W = T diag(beta Gam) K and Ut = T diag(beta) V from it.  This is the per-chunk WY / UT
+// chunk position c ^ (n & 7)).  The forward's state chain then forms W = Bw K and
+// Ut = Bu V on the tensor cores; the backward reads all three.  This is the per-chunk WY / UT
 // step of the chunked form of the gated delta rule (the GDN layer of the FlashQLA pages,
 // news.hamidun.com "What is FlashQLA"; the pages print no formula, the chunk algebra is
 // the one restated in gdn_internal.cuh).
@@ -46,8 +46,8 @@ constexpr int kXs = 72;          // row stride (floats) of X: conflict-free 64-b
 constexpr uint32_t wK = 0;                          // 16 KB bf16 K [dk half][64 rows][128 B];
                                                     // then fp32 X [64][kXs]
 constexpr uint32_t wYs = 64 * kXs * 4;              // fp32 [4 warps][16][9] merge scratch
-constexpr uint32_t wVec = wYs + 4 * 16 * 9 * 4;     // beta, gamma, a, b, |k|^2: 5 x 64 fp32
-constexpr uint32_t wBar = wVec + 5 * 64 * 4;        // mbarrier of the K tile
+constexpr uint32_t wVec = wYs + 4 * 16 * 9 * 4;     // beta, gamma, a, b, |k|^2, beta Gam: 6 x 64 fp32
+constexpr uint32_t wBar = wVec + 6 * 64 * 4;        // mbarrier of the K tile
 constexpr uint32_t wSmemBytes = wBar + 16 + 1024;   // + alignment slack
 static_assert(wYs >= 16384, "X covers the K tile it replaces");
 static_assert(wSmemBytes * kWyMinBlocks + kWyMinBlocks * 1024 <= 228 * 1024, "CTAs per SM");
@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     // started (it waits for this grid's completion before reading the images)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) prefetch_tensormap(&tm_k);  // its first use is a few hundred cycles away
     const int h = blockIdx.y, hk = h / p.group, Hv = p.Hv;
     int n = 0, c = 0;
     int64_t bos = 0, len = 0;
@@ -251,6 +252,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     float* va = vbeta + 128;
     float* vb = vbeta + 192;
     float* vnrm = vbeta + 256;
+    float* vbG = vbeta + 320;
     float gr = 0.f;
     if (tid < 64) {
 #pragma unroll
@@ -271,6 +273,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         const float LOG2E = 1.4426950408889634f;
         va[tid] = fac ? expf(gr - gm) : gr * LOG2E;
         vb[tid] = fac ? expf(gm - gr) : gr * LOG2E;
+        vbG[tid] = bt * expf(gr);
     }
 
     // ---- K K^T, lower block triangle: 20 tiles of 16 rows (m-tile) x 8 columns (n-tile), five
@@ -393,11 +396,11 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     merge_level<3>(X, ysw, warp, lane);
     __syncthreads();
 
-    // ---- bf16 image: thread = rows nr4 .. nr4 + 3, columns s0 .. s0 + 7 (one 16-byte chunk of
-    // each row), from T[r][s] = X[s][r] for r > s
+    // ---- bf16 images T, Bw, Bu: thread = rows nr4 .. nr4 + 3, columns s0 .. s0 + 7 (one 16-byte
+    // chunk of each row), from T[r][s] = X[s][r] for r > s
     {
         const int nr4 = 4 * (tid & 15), ch = tid >> 4, s0 = 8 * ch;
-        uint8_t* img = timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kTImgBytes;
+        uint8_t* img = timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kWyImgBytes;
         float v[4][8];
         if (s0 > nr4 + 3) {  // the block lies above the diagonal
 #pragma unroll
@@ -414,8 +417,27 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
                 v[3][e] = t_sel(col.w, nr4 + 3, s0 + e);
             }
         }
+        float sw[8], su[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(img + sw128_off(nr4 + q, ch)) = pack8(v[q]);
+        for (int e4 = 0; e4 < 2; ++e4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(vbG + s0 + 4 * e4);
+            const float4 u4 = *reinterpret_cast<const float4*>(vbeta + s0 + 4 * e4);
+            sw[4 * e4] = w4.x; sw[4 * e4 + 1] = w4.y; sw[4 * e4 + 2] = w4.z; sw[4 * e4 + 3] = w4.w;
+            su[4 * e4] = u4.x; su[4 * e4 + 1] = u4.y; su[4 * e4 + 2] = u4.z; su[4 * e4 + 3] = u4.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t off = sw128_off(nr4 + q, ch);
+            float bw[8], bu[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                bw[e] = v[q][e] * sw[e];
+                bu[e] = v[q][e] * su[e];
+            }
+            *reinterpret_cast<uint4*>(img + off) = pack8(v[q]);
+            *reinterpret_cast<uint4*>(img + kTImgBytes + off) = pack8(bw);
+            *reinterpret_cast<uint4*>(img + 2 * kTImgBytes + off) = pack8(bu);
+        }
     }
 }
 
@@ -434,8 +456,8 @@ gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* 
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-// workspace: the T images, then one float2 summary per (image slot, value head)
-size_t wy_tc_summary_offset(const Problem& p) { return (size_t)img_slots(p) * p.Hv * kTImgBytes; }
+// workspace: the T / Bw / Bu images, then one float2 summary per (image slot, value head)
+size_t wy_tc_summary_offset(const Problem& p) { return (size_t)img_slots(p) * p.Hv * kWyImgBytes; }
 size_t wy_tc_workspace(const Problem& p) {
     return p.num_chunks > 0 ? align_up(wy_tc_summary_offset(p), 256) + (size_t)img_slots(p) * p.Hv * 8 : 0;
 }

@@ -139,9 +139,10 @@ typedef struct gdn_bwd_args {
 /* Bytes of device workspace gdn_chunk_fwd needs for these arguments (the
  * pointers may be NULL here; only sizes, dtype and cu_seqlens_host are read).
  * Returns GDN_OK and sets *bytes, or an argument error.  The tensor-core path
- * (bf16, dk = dv = 128) keeps one 8 KB bf16 T = (I + A)^-1 image and one 8-byte
- * gate summary per (chunk slot, value head), with floor(T_total / 64) + N + 1
- * chunk slots; the CUDA-core path keeps fp32 W, U, gamma and chunk states. */
+ * (bf16, dk = dv = 128) keeps three 8 KB bf16 images (T = (I + A)^-1,
+ * T diag(beta Gam) and T diag(beta)) and one 8-byte gate summary per (chunk slot,
+ * value head), with floor(T_total / 64) + N + 1 chunk slots; the CUDA-core path
+ * keeps fp32 W, U, gamma and chunk states. */
 GDN_API gdn_status gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args, size_t* bytes);
 
 /* Forward: o and (optionally) S_T from q, k, v, beta, g and (optionally) S0.

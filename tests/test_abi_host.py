@@ -80,12 +80,12 @@ def test_misaligned_tensor_is_rejected(field, offset):
 
 
 def test_workspace_checks():
-    # the tensor-core path (bf16, 128 x 128) keeps one 8 KB T image and one 8-byte gate summary
-    # per (image slot, value head), slots = T_total // 64 + N + 1; the portable path keeps fp32
-    # W, U, gamma and states
+    # the tensor-core path (bf16, 128 x 128) keeps three 8 KB images (T, T diag(beta Gam),
+    # T diag(beta)) and one 8-byte gate summary per (image slot, value head),
+    # slots = T_total // 64 + N + 1; the portable path keeps fp32 W, U, gamma and states
     st, need_tc = ws_size(fwd_args())
     slots = 256 // 64 + 1 + 1
-    assert st == OK and need_tc == -(-(slots * 4 * 8192 + slots * 4 * 8) // 256) * 256
+    assert st == OK and need_tc == -(-(slots * 4 * 3 * 8192 + slots * 4 * 8) // 256) * 256
     assert call_fwd(fwd_args(), ws=0) == WORKSPACE
     a = fwd_args(flags=_abi.GDN_FLAG_PORTABLE)
     st, need = ws_size(a)
