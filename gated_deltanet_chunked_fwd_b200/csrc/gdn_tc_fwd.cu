@@ -50,11 +50,11 @@ using namespace tc;
 namespace {
 
 // Two groups of warps run a two-stage software pipeline over the chunks of a segment:
-//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: gates, Q K^T, P and
-//                                       diag(Gam) Q, W^T and Ut^T (Bw / Bu images of the WY
-//                                       step as B operands), W^T -> smem
-//   group S (threads 256-383, 4 warps)  the state chain of chunk k-1..k: U^T = Ut^T - H^T W^T,
-//                                       H^T <- Gam_n H^T + (U^T diag(decay)) K, outputs, bf16 H
+//   group P (threads 0-255, 8 warps)    chunk-local work of chunk k: the outputs of chunk k-2,
+//                                       gates, Q K^T, P and diag(Gam) Q, W^T and Ut^T (Bw / Bu
+//                                       images of the WY step as B operands), W^T -> smem
+//   group S (threads 256-383, 4 warps)  the state chain of chunk k: U^T = Ut^T - H^T W^T,
+//                                       O^T, H^T <- Gam_n H^T + (U^T diag(decay)) K, bf16 H
 // Each group has one tcgen05 issuer (threads 0 and 256) and its own commit
 // barrier; they hand chunks over through mbarriers (full / empty pairs).  Warp w
 // reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so group P's two warps per lane
@@ -67,8 +67,8 @@ constexpr int kTmemCols = 512;
 constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk     [0, 128)
 constexpr uint32_t kColR1 = 128;  // Q K^T (lanes 0-63), then W^T (group P)   [128, 192)
 constexpr uint32_t kColR2 = 192;  // 2 x (Ut^T -> U^T), by chunk parity      [192, 320)
-constexpr uint32_t kColO = 320;   // O^T = H^T (diag(Gam) Q)^T + U^T P^T      [320, 384)
-                                  // (columns [384, 448) are free)
+constexpr uint32_t kColO = 320;   // 2 x O^T = H^T (diag(Gam) Q)^T + U^T P^T,  [320, 448)
+                                  // by chunk parity
 constexpr uint32_t kColHb = 448;  // bf16 H^T, A operand (K pairs per column) [448, 512)
 // U^T in bf16 (A operand of MMA_UP / MMA_H) overwrites the first 32 columns of its R2 buffer.
 
@@ -318,6 +318,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             gates(0);
             if (nk > 1) load_gates(1);
         }
+        // Outputs of chunk kk (once group S has finished it): o[t0+n][h][m] = O^T[m][n] from the
+        // O^T buffer of parity kk; this thread holds dv row m = `row`, tokens [32 hf, 32 hf + 32).
+        // A whole chunk goes through a shared-memory tile and one TMA store per 64-column half:
+        // lanes m, m^1 swap one value so that each thread writes bf16 pairs (columns m & ~1,
+        // m | 1) of one token.  A chunk cut short by its sequence's end is stored element by
+        // element, masked to its tokens.
+        auto emits = [&](int kk) { return cstart + kk >= c0 && !args.himg; };
+        auto epilogue = [&](int kk) {
+            const int cc = cstart + kk;
+            const int64_t t0 = bos + (int64_t)cc * kChunk;
+            const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
+            const int m = row;
+            float ov[32];
+            tc_fence_after();
+            tmem_ld32(tl + kColO + 64 * (kk & 1) + 32 * hf, ov);
+            if (lc == kChunk) {
+                if (t == 0) bulk_wait_read0();  // the previous chunk's store has read the tile
+                wg_sync(1, kThreadsP);
+                const bool odd = m & 1;
+                const int c = m & ~1, cin = c & 63;
+                uint8_t* tile = sm + kOst + (c >> 6) * 8192;
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int nn = 32 * hf + e;
+                    const float x0 = ov[e], x1 = ov[e + 1];
+                    const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
+                    const uint32_t w = odd ? pack_bf16(recv, x1) : pack_bf16(x0, recv);
+                    const int orow = nn + (odd ? 1 : 0);
+                    *reinterpret_cast<uint32_t*>(tile + sw128_off(orow, cin >> 3) + (cin & 7) * 2) = w;
+                }
+                fence_proxy_async();  // the tile is read by the TMA store
+                wg_sync(1, kThreadsP);
+                if (t == 0) {
+                    tma_store_3d(&tm_o, sm + kOst, 0, h, (int)t0);
+                    tma_store_3d(&tm_o, sm + kOst + 8192, 64, h, (int)t0);
+                    bulk_commit();
+                }
+            } else {
+                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int nn = 32 * hf + e;
+                    if (nn < lc) op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(ov[e]);
+                }
+            }
+        };
 
         for (int k = 0; k < nk; ++k) {
             const int c = cstart + k;
@@ -331,10 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* va = vec + 320;
             const float* vb = vec + 384;
 
-            // buffers of parity `stage` are free once warpgroup S finished chunk k-2
+            // buffers of parity `stage` are free once warpgroup S finished chunk k-2, whose
+            // outputs are then final; group S writes the next O^T of this parity only after
+            // this chunk's hand-off
             if (k >= 2) {
                 ok = wg_and(1, kThreadsP, mbar_wait(&bar_s_done[stage], ((k - 2) >> 1) & 1));
                 if (!ok) break;
+                if (emits(k - 2)) epilogue(k - 2);
             }
             ok = wg_and(1, kThreadsP, mbar_wait(&bar_tma[stage], (k >> 1) & 1));
             if (!ok) break;
@@ -447,70 +496,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             wg_sync(1, kThreadsP);
             if (t == 0) mbar_arrive(bar_wt_full);
         }
+        for (int kk = max(nk - 2, 0); kk < nk && ok; ++kk) {  // the last two chunks' outputs
+            ok = wg_and(1, kThreadsP, mbar_wait(&bar_s_done[kk & 1], (kk >> 1) & 1));
+            if (ok && emits(kk)) epilogue(kk);
+        }
+        if (t == 0) bulk_wait0();  // every output tile has been written
     } else {
         // ======================= group S: the state chain =======================
-        // Per chunk k: MMA_HW, then (overlapping it) the outputs of chunk k-1; U^T -> bf16 in
-        // TMEM; MMA_O / MMA_H (A operands from TMEM); then one pass over H that
+        // Per chunk k: MMA_HW; U^T -> bf16 in TMEM; MMA_O (into the O^T buffer of the chunk's
+        // parity, which group P reads out at chunk k+2) / MMA_H (A operands from TMEM); then one
+        // pass over H that
         // writes its bf16 copy and pre-scales it by the next chunk's Gam_n (MMA_H of chunk
         // k+1 accumulates onto it).
         const int m = tid - kThreadsP;
         uint32_t ph = 0;  // parity of bar_mma_s
-        // o[t0+n][h][m] = O^T[m][n].  A whole chunk goes through a
-        // shared-memory tile and one TMA store per 64-column half: lanes m, m^1 swap one value so
-        // that each thread writes bf16 pairs (columns m & ~1, m | 1) of one token.  A chunk cut
-        // short by its sequence's end is stored element by element, masked to its tokens.
-        auto epilogue = [&](int kk) {
-            const int cc = cstart + kk;
-            const int64_t t0 = bos + (int64_t)cc * kChunk;
-            const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
-            if (lc == kChunk) {
-                if (m == 0) bulk_wait_read0();  // the previous chunk's store has read the tile
-                wg_sync(2, kThreadsS);
-                const bool odd = m & 1;
-                const int c = m & ~1, cin = c & 63;
-                uint8_t* tile = sm + kOst + (c >> 6) * 8192;
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    float ov[32];
-                    tmem_ld32(tl + kColO + 32 * hf, ov);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int nn = 32 * hf + e;
-                        const float x0 = ov[e], x1 = ov[e + 1];
-                        const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
-                        const uint32_t w = odd ? pack_bf16(recv, x1) : pack_bf16(x0, recv);
-                        const int row = nn + (odd ? 1 : 0);
-                        *reinterpret_cast<uint32_t*>(tile + sw128_off(row, cin >> 3) + (cin & 7) * 2) = w;
-                    }
-                }
-                fence_proxy_async();  // the tile is read by the TMA store
-                wg_sync(2, kThreadsS);
-                if (m == 0) {
-                    tma_store_3d(&tm_o, sm + kOst, 0, h, (int)t0);
-                    tma_store_3d(&tm_o, sm + kOst + 8192, 64, h, (int)t0);
-                    bulk_commit();
-                }
-            } else {
-                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float ov[32];
-                    tmem_ld32(tl + kColO + 32 * hf, ov);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int nn = 32 * hf + e;
-                        if (nn < lc) op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(ov[e]);
-                    }
-                }
-            }
-        };
         for (int k = 0; k < nk && ok; ++k) {
             const int c = cstart + k;
             const int stage = k & 1;
             const bool emit = c >= c0 && !args.himg;
-            const bool emit_prev = k > 0 && (c - 1) >= c0 && !args.himg;
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t colR2 = kColR2 + 64 * stage;
+            const uint32_t colO = kColO + 64 * stage;
 
             ok = wg_and(2, kThreadsS, mbar_wait(bar_wt_full, k & 1));
             if (!ok) break;
@@ -535,7 +541,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_bmn_n64, 1);
                 mma_commit(bar_mma_s);
             }
-            if (emit_prev) epilogue(k - 1);  // overlaps MMA_HW of this chunk
             if (args.himg && c >= c0) {
                 // replay mode: the chunk's entry state, as the bf16 H^T image [dk half][128 dv
                 // rows][128 B] (128-byte swizzled) that the backward loads; the bf16 copy in TMEM
@@ -583,12 +588,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                        mma_bf16_ts(tmem + kColO, tmem + kColHb + 8 * j, desc_sw128(sQK + koff, 16, 1024),
+                        mma_bf16_ts(tmem + colO, tmem + kColHb + 8 * j, desc_sw128(sQK + koff, 16, 1024),
                                     id_n64, j > 0);
                     }
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        mma_bf16_ts(tmem + kColO, tmem + colR2 + 8 * j,
+                        mma_bf16_ts(tmem + colO, tmem + colR2 + 8 * j,
                                     desc_sw128(sbase + kPt + stage * 8192 + j * 32, 16, 1024), id_n64, 1);
                 }
 #pragma unroll
@@ -627,8 +632,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             wg_sync(2, kThreadsS);
             if (m == 0) mbar_arrive(&bar_s_done[stage]);
         }
-        if (ok && nk > 0 && cstart + nk - 1 >= c0 && !args.himg) epilogue(nk - 1);
-        if (m == 0) bulk_wait0();  // every output tile has been written
         if (ok && p.ST && seg == segs_n - 1) {
             // final state S_T = H (stored [dk][dv]): thread m writes column m
             float* st = p.ST + ((int64_t)n * Hv + h) * dk * dv + m;
