@@ -2,7 +2,8 @@
 // sm_100a).  The backward of the GDN layer (FlashQLA pages: dothoosh.com article, opening
 // paragraph, "backward pass"; news.hamidun.com page, "large-scale pretraining" scenario).
 //
-// Four launches: the WY kernel (T images and per-chunk gate summaries), the fused forward
+// Four launches: the WY kernel (T, T diag(beta Gam), T diag(beta) images and per-chunk gate
+// summaries), the fused forward
 // kernel in replay mode (the bf16 entry state H^T of every chunk, as a ready-to-use
 // 128-byte-swizzled shared-memory image), this reverse kernel, and the reduction of dq / dk over
 // grouped value heads.  The reverse kernel runs one CTA per (sequence, value head, segment of
@@ -791,7 +792,7 @@ __global__ void __launch_bounds__(kNT, 1)
 
 bool tc_bwd_supported(const Problem& p) { return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128; }
 
-// workspace: the WY outputs (T images, gate summaries), the replayed H^T images, then (with
+// workspace: the WY outputs (T / Bw / Bu images, gate summaries), the replayed H^T images, then (with
 // grouped heads) fp32 dq and dk per value head, summed over each group by the reduction
 size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, size_t* off_dqw,
                         size_t* off_dkw) {

@@ -3,23 +3,24 @@
 //
 // Two launches do the whole forward.  The first (gdn_tc_wy.cu) forms, for every
 // (chunk, value head) at once, the state-independent WY / UT inverse
-// T = (I + A)^-1, A = strictly-lower(diag(beta) (K K^T o E)), as a bf16 image in the
-// workspace.  The second (this file) is the fused state chain: each CTA owns one
+// T = (I + A)^-1, A = strictly-lower(diag(beta) (K K^T o E)), and from it the bf16 images
+// Bw = T diag(beta Gam) and Bu = T diag(beta) in the workspace.  The second (this file) is
+// the fused state chain: each CTA owns one
 // (sequence, value head, segment of chunks) and walks its chunks in order, keeping
 // the fp32 state in TMEM; per chunk of C = 64 tokens (notation of gdn_internal.cuh):
 //   gates      gamma = cumsum g, Gam, E = exp(gamma_r - gamma_s)       CUDA cores
 //   MMA1       [Q;K] K^T -> Q K^T (rows 0-63 of the M=128 product)      tensor core
-//   Bw, Bu     T diag(beta Gam), T diag(beta) from the T image          CUDA cores
-//   MMA_W/U    W^T = K^T (T diag(beta Gam))^T,  Ut^T = V^T (T diag(beta))^T
+//   MMA_W/U    W^T = K^T Bw^T,  Ut^T = V^T Bu^T  (Bw, Bu: images of the WY step)
 //   MMA_HW     U^T = Ut^T - H^T W^T  (accumulated onto Ut^T, B = -W^T)
 //   MMA_O      O^T = H^T (diag(Gam) Q)^T + U^T P^T,  P = lower-incl(Q K^T o E)
-//              (Q scaled by Gam in shared memory once Q K^T has read it)
+//              (Q scaled by Gam in shared memory once Q K^T has read it; the outputs
+//              are stored by the chunk-local warp group two chunks later)
 //   MMA_H      H^T <- Gam_n H^T + (U^T diag(exp(gamma_n - gamma))) K
 // All matrices are oriented so that a 128-wide head dimension is the MMA's M
 // (TMEM lane = dv or dk index), so every MMA is M = 128 with N = 64 or 128.
 // Operands live in shared memory as 128-byte-swizzled tiles; q / k / v tiles
-// come in by TMA and the T image by a bulk copy (double-buffered: chunk c+1 loads
-// while chunk c computes).
+// come in by TMA and the Bw / Bu images by a bulk copy (double-buffered: chunk c+2
+// loads while chunks c and c+1 compute).
 //
 // Long sequences are split into segments that run on different SMs
 // (gate-driven context parallelism, dothoosh.com FlashQLA article, first
@@ -661,7 +662,7 @@ bool tc_fwd_supported(const Problem& p) {
     return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128;
 }
 
-// workspace: the T images of the WY step
+// workspace: the T / Bw / Bu images and gate summaries of the WY step
 size_t tc_fwd_workspace(const Problem& p) { return wy_tc_workspace(p); }
 int tc_fwd_launches(const Problem& p) { return (p.num_chunks > 0 ? 1 : 0) + 1; }
 
