@@ -23,8 +23,8 @@ from ._abi import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE, GDN_FLAG_SPLIT_OFF, 
                    GdnError, GdnFwdArgs)
 
 __all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_chunk_fwd_workspace_size",
-           "gdn_chunk_bwd_workspace_size", "GdnError", "GDN_FLAG_SPLIT_OFF",
-           "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE"]
+           "gdn_chunk_bwd_workspace_size", "chunk_fwd", "chunk_bwd", "GdnError",
+           "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE"]
 
 _DT = {torch.float32: _abi.GDN_F32, torch.bfloat16: _abi.GDN_BF16}
 
@@ -184,3 +184,9 @@ def launch_count(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None, initia
     _, host = _fill_common(a, q, k, v, beta, g, cu_seqlens, cu_seqlens_host, initial_state, flags)
     fn = _abi.lib().gdn_chunk_bwd_launch_count if backward else _abi.lib().gdn_chunk_fwd_launch_count
     return int(fn(ctypes.byref(a)))
+
+
+# short names: chunk_fwd(q, k, v, beta, g, cu_seqlens=None, initial_state=None) -> (o, S_T) and
+# chunk_bwd(...) -> (dq, dk, dv, dbeta, dg, dS0) are the same calls
+chunk_fwd = gdn_chunk_fwd
+chunk_bwd = gdn_chunk_bwd

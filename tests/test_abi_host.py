@@ -28,6 +28,13 @@ def test_library_exports_every_declared_function():
         assert hasattr(L, fn), fn
 
 
+def test_python_short_names():
+    import gated_deltanet_chunked_fwd_b200 as gdn
+
+    assert gdn.chunk_fwd is gdn.gdn_chunk_fwd and gdn.chunk_bwd is gdn.gdn_chunk_bwd
+    assert {"chunk_fwd", "chunk_bwd", "gdn_chunk_fwd", "gdn_chunk_bwd"} <= set(gdn.__all__)
+
+
 def test_status_strings():
     L = _abi.lib()
     for code in range(7):
