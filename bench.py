@@ -2,16 +2,23 @@
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
-A step is one forward pass of the layer over one batch of the bf16 workload
-B=1, T=4096, H=16, dk=dv=128 (C=64, random fp32 S0) through the C ABI, inputs
-already resident in HBM.  The L2 is flushed (a 2 x L2-size write) before every
-timed step, outside the timed events.  ``value`` is whole-job tokens/s; with N
-GPUs every rank runs its own replica (weak scaling, no collective on the data
-path) and the time is the max over ranks.  ``e2e`` times the same call with the
-inputs in pinned host memory, including the host->device copies of the inputs
-and the device->host copies of o and S_T.  ``bwd`` reports the backward on the
-B=4, T=8192, H=16, d=128 workload.  ``cpu_baseline`` times the float64 oracle on
-a bounded sample of the same workload on the host cores.
+A step is one forward pass of the layer over one batch of the long-context bf16
+workload: B=1, T=65,536 tokens, H=16 heads, dk=dv=128, C=64, slow decay
+(g = -softplus(N(-2,1))), zero initial state, through the C ABI, inputs already
+resident in HBM (1.08 GB of algorithmic traffic, well above the 126 MB L2; the
+L2 is also flushed by a 2 x L2-size write before every timed step, outside the
+timed events).  ``value`` is whole-job tokens/s; with N GPUs every rank runs
+its own replica (weak scaling, no collective on the data path) and the time is
+the max over ranks.  ``e2e`` times the same call with the inputs in pinned host
+memory, including the host->device copies of the inputs and the device->host
+copies of o and S_T.
+
+Extra keys, each timed the same way: ``fwd_workloads`` holds the 4,096-token
+forward with a random initial state, the packed varlen batch (8 sequences,
+16 q/k heads, 32 value heads) and the long context fed as 4 chained
+16,384-token calls; ``bwd`` the backward on the B=4, T=8192, H=16 workload.
+``cpu_baseline`` times the float64 oracle on a bounded sample of the headline
+workload on the host cores.
 
 ``--impl reference`` times the oracle (there is no other implementation of this
 layer to run here) on a bounded sample per step and prints the same line with
@@ -22,6 +29,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -35,6 +43,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GDN chunked-prefill fwd/bwd tokens/s and TFLOP/s vs BF16 roofline, 1×B200"
 CHUNK = 64
+HEADLINE = 3  # index of the 65,536-token slow-decay forward in inputs.WORKLOADS
+HEADLINE_DESC = "gdn_fwd bf16 B=1 T=65536 H=16 dk=dv=128 C=64 g=-softplus(N(-2,1)) S0=0 (one call)"
+ORACLE_SAMPLE_T = 8192  # tokens per head in one bounded oracle sample
 
 
 def flops_per_token_head(dk, dv, C=CHUNK, backward=False):
@@ -47,9 +58,10 @@ def flops_per_token_head(dk, dv, C=CHUNK, backward=False):
     return dense, tri
 
 
-def fwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
-    """Algorithmic HBM bytes of one forward: read q, k, v, beta, g, S0; write o, S_T."""
-    return T_total * (elt * (Hk * 2 * dk + Hv * 2 * dv) + Hv * 8) + 2 * N * Hv * dk * dv * 4
+def fwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2, s0=True, st=True):
+    """Algorithmic HBM bytes of one forward: read q, k, v, beta, g (and S0); write o (and S_T)."""
+    states = (int(s0) + int(st)) * N * Hv * dk * dv * 4
+    return T_total * (elt * (Hk * 2 * dk + Hv * 2 * dv) + Hv * 8) + states
 
 
 def bwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
@@ -57,29 +69,58 @@ def bwd_bytes(T_total, Hk, Hv, dk, dv, N, elt=2):
     return T_total * (elt * (Hk * 4 * dk + Hv * 3 * dv) + Hv * 16) + 2 * N * Hv * dk * dv * 4
 
 
+def roofline(flops_dense, byts, seconds, hbm_gbs, bf16_tflops, src):
+    """t_roof = max(FLOPs / tensor peak, bytes / HBM peak); frac = t_roof / measured time.  The
+    bound is whichever term is larger; both fractions are reported."""
+    t_hbm = byts / (hbm_gbs * 1e9)
+    t_tc = flops_dense / (bf16_tflops * 1e12)
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    achieved_gbs = byts / seconds / 1e9
+    achieved_tf = flops_dense / seconds / 1e12
+    if bound == "hbm":
+        ach, peak, unit = achieved_gbs, hbm_gbs, "GB/s"
+    else:
+        ach, peak, unit = achieved_tf, bf16_tflops, "TFLOP/s"
+    return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+            "t_roof_us": max(t_hbm, t_tc) * 1e6, "frac_hbm": achieved_gbs / hbm_gbs,
+            "frac_tensor": achieved_tf / bf16_tflops, "achieved_gbs": achieved_gbs,
+            "achieved_tflops_dense": achieved_tf, "peak_gbs": hbm_gbs, "peak_tflops": bf16_tflops,
+            "peak_source": src, "algorithmic_bytes": byts, "flops_dense": flops_dense}
+
+
 FWD_SOURCES = ("gdn_tc_wy.cu", "gdn_tc_fwd.cu", "gdn_tc_common.cuh", "gdn_sm100.cuh",
                "gdn_internal.cuh")
 
 
+def strip_comments(src: str) -> str:
+    """C / C++ source without comments and with runs of whitespace collapsed, so that a
+    fingerprint changes with the code, not with its comments (string literals in these files
+    hold no comment markers)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def source_sha16(files=FWD_SOURCES):
-    """Fingerprint of the tensor-core forward's sources (matches profiles/traffic.json)."""
+    """Fingerprint of the tensor-core forward's code, comments ignored (matches
+    profiles/traffic.json)."""
     import hashlib
 
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "gated_deltanet_chunked_fwd_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "gated_deltanet_chunked_fwd_b200", "csrc", f)) as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
-def traffic_per_call():
-    """DRAM bytes (read + write) of one forward call (the WY kernel and the fused kernel) from
-    the committed ncu capture, or None when the sources changed since that capture."""
+def traffic_per_call(workload):
+    """DRAM bytes (read + write) of one forward call (the WY kernel and the fused kernel) of
+    ``workload`` from the committed ncu capture, or None when the code changed since."""
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(tp):
         return None
     with open(tp) as f:
-        rec = json.load(f).get("fwd_bf16_T4096_H16_d128", {})
+        rec = json.load(f).get(workload, {})
     return rec.get("bytes_per_call") if rec.get("source_sha16") == source_sha16() else None
 
 
@@ -190,7 +231,7 @@ def job_throughput(units_per_rank, world, ms):
 def oracle_sample(inp, nheads, units_total):
     """Run the oracle on the first ``nheads`` value heads of a fixed-length workload
     in one call (OpenMP over the heads) and return (seconds, tokens/s scaled to
-    the full workload: tokens x nheads / units_total per second)."""
+    the full workload: tokens x nheads / units_total per second, nheads)."""
     import oracle
 
     x = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
@@ -206,13 +247,25 @@ def oracle_sample(inp, nheads, units_total):
     return dt, tokens / dt, nheads
 
 
+def oracle_sample_inputs():
+    """The headline workload's shapes and distributions, cut to ORACLE_SAMPLE_T tokens per head."""
+    from gated_deltanet_chunked_fwd_b200.inputs import make_workload
+
+    return make_workload(HEADLINE, seed=0, T=ORACLE_SAMPLE_T)
+
+
+def sample_desc(nh, Hv, reps, seconds):
+    return (f"{reps} passes over {nh} of {Hv} value heads x the first {ORACLE_SAMPLE_T} tokens of "
+            f"the headline workload's distribution (float64 token loop), {seconds:.1f} s; "
+            f"tokens/s scaled by {nh}/{Hv} heads")
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
     import oracle
-    from gated_deltanet_chunked_fwd_b200.inputs import make_workload
 
-    inp = make_workload(1, seed=0)
+    inp = oracle_sample_inputs()
     Hv = inp["v"].shape[2]
     nheads = min(Hv, oracle.num_threads())  # bounded sample: one head per host thread
     for _ in range(args.warmup):
@@ -221,20 +274,18 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         dt, _, nheads = oracle_sample(inp, nheads, Hv)
         times.append(dt)
-    T_tok = inp["q"].shape[1] * inp["q"].shape[0]
-    tok_per_step = T_tok * nheads / Hv
+    tok_per_step = ORACLE_SAMPLE_T * nheads / Hv
     value = tok_per_step * len(times) / sum(times)
     cores = min(nheads, oracle.num_threads())
-    heads = range(nheads)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "gdn_fwd bf16 B=1 T=4096 H=16 dk=dv=128 C=64 S0~0.1N(0,1)",
-                   "global_batch": 1, "seq_len": 4096, "parallelism": "none (host oracle)"},
+        "config": {"workload": HEADLINE_DESC, "global_batch": 1, "seq_len": 65536,
+                   "parallelism": "none (host oracle)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{len(heads)} of {Hv} value heads per step (float64 token loop)"},
+                         "sample": sample_desc(nheads, Hv, len(times), sum(times))},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -256,95 +307,161 @@ def time_steps(fn, steps, flush, stream):
     return ms
 
 
-def run_ours(args, world, rank, local):
-    import ctypes
+class FwdCall:
+    """One gdn_chunk_fwd call through the C ABI on fixed device buffers (struct filled once)."""
 
+    def __init__(self, inp, dev, stream, S0=None, ST=None):
+        import ctypes
+
+        import gated_deltanet_chunked_fwd_b200 as gdn
+        from gated_deltanet_chunked_fwd_b200 import _abi
+
+        self.gdn, self.ctypes, self.L = gdn, ctypes, _abi.lib()
+        q, k, v = inp["q"], inp["k"], inp["v"]
+        self.inp = inp
+        B, T, Hk, dk = q.shape
+        Hv, dv = v.shape[2], v.shape[3]
+        cu = inp.get("cu_seqlens")
+        self.N = B if cu is None else cu.numel() - 1
+        self.shape = dict(T_total=B * T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, N=self.N)
+        self.o = torch.empty(B, T, Hv, dv, dtype=q.dtype, device=dev)
+        self.ST = ST if ST is not None else torch.empty(self.N, Hv, dk, dv, dtype=torch.float32,
+                                                        device=dev)
+        self.S0 = S0 if S0 is not None else inp.get("initial_state")
+        a = _abi.GdnFwdArgs()
+        self.host = gdn._fill_common(a, q, k, v, inp["beta"], inp["g"], cu, inp.get("cu_seqlens_host"),
+                                     self.S0, 0)[1]
+        a.o, a.ST = self.o.data_ptr(), self.ST.data_ptr()
+        self.a = a
+        n = ctypes.c_size_t(0)
+        st = self.L.gdn_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
+        if st != 0:
+            raise gdn.GdnError("gdn_chunk_fwd_workspace_size", st)
+        self.ws_n = n.value
+        self.ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=dev)
+        self.launches = self.L.gdn_chunk_fwd_launch_count(ctypes.byref(a))
+        self.sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def __call__(self):
+        st = self.L.gdn_chunk_fwd(self.ctypes.byref(self.a), self.ctypes.c_void_p(self.ws.data_ptr()),
+                                  self.ws_n, self.sp)
+        if st != 0:
+            raise self.gdn.GdnError("gdn_chunk_fwd", st)
+
+    def bytes(self):
+        s = self.shape
+        return fwd_bytes(s["T_total"], s["Hk"], s["Hv"], s["dk"], s["dv"], s["N"],
+                         s0=self.S0 is not None, st=True)
+
+
+def run_ours(args, world, rank, local):
     import gated_deltanet_chunked_fwd_b200 as gdn
-    from gated_deltanet_chunked_fwd_b200 import _abi
-    from gated_deltanet_chunked_fwd_b200.inputs import make_workload
+    from gated_deltanet_chunked_fwd_b200.inputs import WORKLOADS, make_workload
 
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
-    L = _abi.lib()
-    inp = make_workload(1, seed=rank, device=dev)
-    q, k, v, beta, g, S0 = (inp[n] for n in ("q", "k", "v", "beta", "g", "initial_state"))
-    B, T, Hk, dk = q.shape
-    Hv, dv = v.shape[2], v.shape[3]
-    N = B
-    o = torch.empty(B, T, Hv, dv, dtype=q.dtype, device=dev)
-    ST = torch.empty(N, Hv, dk, dv, dtype=torch.float32, device=dev)
-    a = _abi.GdnFwdArgs()
-    gdn._fill_common(a, q, k, v, beta, g, None, None, S0, 0)
-    a.o, a.ST = o.data_ptr(), ST.data_ptr()
-    ws_n = gdn.gdn_chunk_fwd_workspace_size(q, k, v, beta, g, initial_state=S0)
-    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
-    launches = L.gdn_chunk_fwd_launch_count(ctypes.byref(a))
-    sp = ctypes.c_void_p(stream.cuda_stream)
-
-    def step():
-        st = L.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(ws.data_ptr()), ws_n, sp)
-        if st != 0:
-            raise gdn.GdnError("gdn_chunk_fwd", st)
-
+    hbm, bf16, src = measured_peaks()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     scratch = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
 
     def flush():
         scratch.fill_(1.0)
 
+    def measure(fn, steps, warm=3):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        ms = time_steps(fn, steps, flush, stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(sum(ms) / len(ms), world)
+
+    # ---- headline: one 65,536-token call
+    inp = make_workload(HEADLINE, seed=rank, device=dev)
+    call = FwdCall(inp, dev, stream)
+    Hv, dk, dv = call.shape["Hv"], call.shape["dk"], call.shape["dv"]
+    tokens = call.shape["T_total"]
     for _ in range(max(args.warmup, 3)):
-        step()
+        call()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     with Clocks(local) as clk:
-        ms = time_steps(step, args.steps, flush, stream)
+        ms = time_steps(call, args.steps, flush, stream)
         torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     ms_step = max_over_ranks(sum(ms) / len(ms), world)
-    tokens = B * T
     value = job_throughput(tokens, world, ms_step)
+    dense, tri = flops_per_token_head(dk, dv)
+    byts = call.bytes()
+    roof = roofline(dense * tokens * Hv, byts, ms_step * 1e-3, hbm, bf16, src)
+    roof["traffic"] = traffic_per_call(WORKLOADS[HEADLINE].name) if call.launches == 2 else None
+    roof["kernel"] = "whole forward call: gdn_wy_tc_kernel + gdn_fwd_tc_kernel"
+    tflops = {"dense": dense * tokens * Hv / (ms_step * 1e-3) / 1e12,
+              "triangular": tri * tokens * Hv / (ms_step * 1e-3) / 1e12, "peak_bf16": bf16}
 
     # ---- e2e: pinned host inputs, H2D + call + D2H of o and S_T, inside the timed region
-    host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("beta", beta),
-                                                  ("g", g), ("S0", S0))}
+    names = [n for n in ("q", "k", "v", "beta", "g") if inp.get(n) is not None]
+    host = {n: inp[n].cpu().pin_memory() for n in names}
     dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    ST_h = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
-    ae = _abi.GdnFwdArgs()
-    gdn._fill_common(ae, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["beta"], dbuf["g"], None, None,
-                     dbuf["S0"], 0)
-    ae.o, ae.ST = o.data_ptr(), ST.data_ptr()
+    e2e_inp = dict(dbuf)
+    ecall = FwdCall(e2e_inp, dev, stream)
+    o_h = torch.empty(ecall.o.shape, dtype=ecall.o.dtype).pin_memory()
+    ST_h = torch.empty(ecall.ST.shape, dtype=ecall.ST.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * ST_h.element_size()
 
     def e2e_step():
         for n_, t in host.items():
             dbuf[n_].copy_(t, non_blocking=True)
-        st = L.gdn_chunk_fwd(ctypes.byref(ae), ctypes.c_void_p(ws.data_ptr()), ws_n, sp)
-        if st != 0:
-            raise gdn.GdnError("gdn_chunk_fwd", st)
-        o_h.copy_(o, non_blocking=True)
-        ST_h.copy_(ST, non_blocking=True)
+        ecall()
+        o_h.copy_(ecall.o, non_blocking=True)
+        ST_h.copy_(ecall.ST, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    ms_e2e = max_over_ranks(sum(time_steps(e2e_step, args.steps, flush, stream)) / args.steps, world)
+    ms_e2e = measure(e2e_step, max(2, min(args.steps, 5)))
     e2e_value = job_throughput(tokens, world, ms_e2e)
+    del dbuf, e2e_inp, ecall
 
-    # ---- roofline of the forward call (the WY kernel + the fused state-chain kernel)
-    hbm, bf16, src = measured_peaks()
-    byts = fwd_bytes(tokens, Hk, Hv, dk, dv, N)
-    dense, tri = flops_per_token_head(dk, dv)
-    achieved = byts / (ms_step * 1e-3) / 1e9
-    tflops_dense = dense * tokens * Hv / (ms_step * 1e-3) / 1e12
-    tflops_tri = tri * tokens * Hv / (ms_step * 1e-3) / 1e12
-    traffic = traffic_per_call() if launches == 2 else None
+    # ---- the other forward workloads (extra keys)
+    extra = {}
+    if not args.no_extra:
+        for idx in (1, 2):
+            w = WORKLOADS[idx]
+            c = FwdCall(make_workload(idx, seed=rank, device=dev), dev, stream)
+            m = measure(c, args.steps)
+            t_ = c.shape["T_total"]
+            extra[w.name] = {
+                "ms": m, "tokens_per_s": job_throughput(t_, world, m), "tokens": t_,
+                "launches": c.launches,
+                "roofline": dict(roofline(dense * t_ * c.shape["Hv"], c.bytes(), m * 1e-3, hbm, bf16, src),
+                                 traffic=traffic_per_call(w.name) if c.launches == 2 else None)}
+            del c
+        # the headline's tokens fed as 4 chained 16,384-token calls (S_T -> S0)
+        parts = []
+        prev = None
+        for i in range(4):
+            sl = slice(i * 16384, (i + 1) * 16384)
+            sub = {n: inp[n][:, sl].contiguous() for n in ("q", "k", "v", "beta", "g")}
+            c = FwdCall(sub, dev, stream, S0=prev)
+            prev = c.ST
+            parts.append(c)
 
-    # ---- backward on its own workload (one step per measurement)
+        def chained():
+            for c in parts:
+                c()
+
+        m = measure(chained, args.steps)
+        cb = sum(c.bytes() for c in parts)
+        extra["fwd_bf16_T65536_H16_d128_slowdecay_4x16384_chained"] = {
+            "ms": m, "tokens_per_s": job_throughput(tokens, world, m), "tokens": tokens,
+            "launches": sum(c.launches for c in parts),
+            "roofline": roofline(dense * tokens * Hv, cb, m * 1e-3, hbm, bf16, src)}
+        del parts
+
+    # ---- backward on its own workload
     bwd = None
     if not args.no_bwd:
         bi = make_workload(4, seed=rank, device=dev, B=args.bwd_batch)
@@ -355,33 +472,28 @@ def run_ours(args, world, rank, local):
         def bstep():
             gdn.gdn_chunk_bwd(*qs, dST=bi["dST"], workspace=wsb)
 
-        bstep()
-        torch.cuda.synchronize()
-        bms = max_over_ranks(statistics.mean(time_steps(bstep, max(1, min(args.steps, 5)), flush,
-                                                        stream)), world)
+        bms = measure(bstep, max(1, min(args.steps, 5)), warm=1)
         bt = bi["q"].shape[0] * bi["q"].shape[1]
         bd, btri = flops_per_token_head(dk, dv, backward=True)
-        bb = bwd_bytes(bt, Hk, Hv, dk, dv, bi["q"].shape[0])
-        t_roof = max(bd * bt * Hv / (bf16 * 1e12), bb / (hbm * 1e9))  # seconds
+        bb = bwd_bytes(bt, bi["q"].shape[2], Hv, dk, dv, bi["q"].shape[0])
         bwd = {"workload": f"gdn_bwd bf16 B={args.bwd_batch} T=8192 H=16 dk=dv=128 C=64",
                "tokens_per_s": job_throughput(bt, world, bms),
                "ms": bms, "tflops_dense": bd * bt * Hv / (bms * 1e-3) / 1e12,
                "tflops_tri": btri * bt * Hv / (bms * 1e-3) / 1e12,
                "hbm_gbs": bb / (bms * 1e-3) / 1e9,
-               "roofline": {"bound": "tensor" if bd * bt * Hv / (bf16 * 1e12) >= bb / (hbm * 1e9) else "hbm",
-                            "t_roof_ms": t_roof * 1e3, "frac": t_roof / (bms * 1e-3),
-                            "peak_tflops": bf16, "peak_gbs": hbm, "peak_source": src},
+               "roofline": roofline(bd * bt * Hv, bb, bms * 1e-3, hbm, bf16, src),
                "path": "WY kernel + fused kernel (state replay) + reverse kernel"
-                       + (" + dq/dk group reduction" if Hv != Hk else ""),
+                       + (" + dq/dk group reduction" if bi["v"].shape[2] != bi["q"].shape[2] else ""),
                "launches": gdn.launch_count(*qs[:5], backward=True)}
+        del bi, qs, wsb
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu_base = None
     if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
 
+        inp_cpu = oracle_sample_inputs()
         nh = min(Hv, oracle.num_threads())
-        inp_cpu = make_workload(1, seed=0)
         # repeat the same bounded sample until about 10 s of host time have been measured
         dt_sum, tok_sum, reps = 0.0, 0.0, 0
         while dt_sum < 10.0 and reps < 1000:
@@ -389,10 +501,9 @@ def run_ours(args, world, rank, local):
             dt_sum += dt
             tok_sum += tps * dt
             reps += 1
-        cpu_base = {"value": tok_sum / dt_sum, "unit": "tokens/s", "cores": min(nh, oracle.num_threads()),
-                    "kind": "oracle",
-                    "sample": f"{reps} passes over {nh} of {Hv} value heads of the same workload "
-                              f"(all 4096 tokens each), float64 token loop, {dt_sum:.1f} s"}
+        cpu_base = {"value": tok_sum / dt_sum, "unit": "tokens/s",
+                    "cores": min(nh, oracle.num_threads()), "kind": "oracle",
+                    "sample": sample_desc(nh, Hv, reps, dt_sum)}
 
     if rank == 0:
         line = {
@@ -400,22 +511,21 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "gdn_fwd bf16 B=1 T=4096 H=16 dk=dv=128 C=64 S0~0.1N(0,1)",
-                       "global_batch": world, "seq_len": T, "heads": Hv, "head_dim": dk,
+            "config": {"workload": HEADLINE_DESC,
+                       "global_batch": world, "seq_len": 65536, "heads": Hv, "head_dim": dk,
                        "parallelism": f"replicas x{world} (no collective)",
-                       "l2": "flushed before every timed step (2x L2 write, outside the events)",
-                       "path": "tensor-core (WY kernel + fused state chain)" if launches <= 2 else "cuda-core 4-kernel"},
-            "tflops": {"dense": tflops_dense, "triangular": tflops_tri, "peak_bf16": bf16,
-                       "frac_dense": tflops_dense / bf16},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": traffic,
-                         "peak_source": src, "algorithmic_bytes": byts,
-                         "kernel": "whole forward call: gdn_wy_tc_kernel + gdn_fwd_tc_kernel"},
+                       "l2": "inputs (1.08 GB) larger than L2; L2 also flushed before every timed "
+                             "step (2x L2 write, outside the events)",
+                       "path": "tensor-core (WY kernel + fused state chain)" if call.launches <= 2
+                       else "cuda-core 4-kernel"},
+            "tflops": tflops,
+            "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches * args.steps,
+                    "d2h_bytes_per_step": d2h, "ms": ms_e2e},
+            "gpu_launches": call.launches * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu_base,
+            "fwd_workloads": extra,
             "bwd": bwd,
         }
         print(json.dumps(line), flush=True)
@@ -429,6 +539,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="headline forward only")
     ap.add_argument("--bwd-batch", type=int, default=4,
                     help="sequences in the backward workload (4 = the backward workload; fewer for a small profile)")
     args = ap.parse_args()

@@ -55,6 +55,16 @@ gdn_status check_tensor(const void* ptr, bool needed, uintptr_t align) {
     return aligned(ptr, align) ? GDN_OK : GDN_ERR_INVALID_ARG;
 }
 
+// true when the byte ranges [a, a + n) and [b, b + n) share a byte (both non-NULL)
+bool overlaps(const void* a, const void* b, size_t n) {
+    if (!a || !b || n == 0) return false;
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return x < y + n && y < x + n;
+}
+
+// bytes of one state array [N, Hv, dk, dv] fp32
+size_t state_bytes(const Problem& p) { return (size_t)p.N * p.Hv * p.dk * p.dv * sizeof(float); }
+
 }  // namespace
 
 gdn_status plan_fwd(const gdn_fwd_args* a, FwdPlan* plan) {
@@ -109,6 +119,9 @@ static gdn_status check_fwd_pointers(const gdn_fwd_args* a, const Problem& p) {
         (st = check_tensor(a->S0, false, 16)) || (st = check_tensor(a->ST, false, 16)) ||
         (st = check_tensor(a->dev_status, false, 4)) || (st = check_tensor(a->cu_seqlens, false, 4)))
         return st;
+    // S0 and S_T must not share memory: a segment of a split sequence may read S0 after the
+    // sequence's last segment (another CTA) has written S_T
+    if (overlaps(a->S0, a->ST, state_bytes(p))) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
 }
 
@@ -183,6 +196,10 @@ static gdn_status check_bwd_pointers(const gdn_bwd_args* a, const Problem& p) {
         (st = check_tensor(a->dST, false, 16)) || (st = check_tensor(a->dS0, false, 16)) ||
         (st = check_tensor(a->dev_status, false, 4)) || (st = check_tensor(a->cu_seqlens, false, 4)))
         return st;
+    // dS0 is written while other CTAs may still read S0 (state replay) or dS_T (segments that
+    // start their reverse walk exactly): no shared memory between them
+    const size_t sb = state_bytes(p);
+    if (overlaps(a->dS0, a->S0, sb) || overlaps(a->dS0, a->dST, sb)) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
 }
 

@@ -87,9 +87,10 @@ size_t tc_fwd_workspace(const Problem& p);
 size_t wy_tc_workspace(const Problem& p);
 size_t wy_tc_summary_offset(const Problem& p);
 // WY + fused kernel in replay mode: bf16 H^T entry-state image (32 KB) of every chunk, by
-// (image slot, value head), into himg; `ws` holds the WY outputs (wy_tc_workspace bytes)
-gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, char* ws, uint8_t* himg,
-                            cudaStream_t s);
+// (image slot, value head), into himg; `ws` holds the WY outputs (wy_tc_workspace bytes);
+// split_mode as in FwdPlan
+gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, int split_mode, char* ws,
+                            uint8_t* himg, cudaStream_t s);
 int tc_fwd_launches(const Problem& p);
 bool tc_fwd_supported(const Problem& p);
 

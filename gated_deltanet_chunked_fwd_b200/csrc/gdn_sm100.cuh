@@ -306,7 +306,6 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* v) {
         : "memory");
 }
 
-// 32 packed 32-bit words per thread -> 32 consecutive TMEM columns of this warp's lanes; waits.
 // 16 packed 32-bit words per thread -> 16 consecutive TMEM columns of this warp's lanes; waits.
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
     asm volatile(
@@ -318,6 +317,7 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
         : "memory");
 }
 
+// 32 packed 32-bit words per thread -> 32 consecutive TMEM columns of this warp's lanes; waits.
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* r) {
     tmem_st32(taddr, reinterpret_cast<const float*>(r));
 }

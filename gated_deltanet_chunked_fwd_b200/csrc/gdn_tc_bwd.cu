@@ -840,7 +840,7 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
     if (p.num_chunks > 0) {  // WY step + replay of the entry states
-        const gdn_status st = launch_replay_tc(p, plan.cu_host, ws + ot, (uint8_t*)(ws + oh), s);
+        const gdn_status st = launch_replay_tc(p, plan.cu_host, plan.split_mode, ws + ot, (uint8_t*)(ws + oh), s);
         if (st) return st;
     }
     gdn_bwd_tc_kernel<<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);

@@ -718,12 +718,12 @@ gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
     return launch_fwd_tc_impl(plan.p, plan.cu_host, plan.split_mode, ws, nullptr, s);
 }
 
-gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, char* ws, uint8_t* himg,
-                            cudaStream_t s) {
+gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, int split_mode, char* ws,
+                            uint8_t* himg, cudaStream_t s) {
     Problem q = p;  // states only: no o, no S_T
     q.o = nullptr;
     q.ST = nullptr;
-    return launch_fwd_tc_impl(q, cu_host, 0, ws, himg, s);
+    return launch_fwd_tc_impl(q, cu_host, split_mode, ws, himg, s);
 }
 
 }  // namespace gdn

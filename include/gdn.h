@@ -80,7 +80,10 @@ typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 /* flags (bitwise or); 0 selects the defaults */
 #define GDN_FLAG_SPLIT_OFF (1u << 0)   /* never split one sequence across SMs      */
 #define GDN_FLAG_SPLIT_FORCE (1u << 1) /* split every sequence into short segments */
-#define GDN_FLAG_PORTABLE (1u << 2)    /* CUDA-core kernels only (no tensor cores) */
+#define GDN_FLAG_PORTABLE (1u << 2)    /* test aid: run a shape that the tensor-core
+                                          kernels cover on the CUDA-core kernels instead
+                                          (fp32 arithmetic), to cross-check the two; not
+                                          a second backend for production use          */
 
 /* Arguments of the forward.  struct_size = sizeof(gdn_fwd_args),
  * abi_version = GDN_ABI_VERSION. */
@@ -102,7 +105,10 @@ typedef struct gdn_fwd_args {
     const int32_t* cu_seqlens_host; /* host copy, required with cu_seqlens       */
     const float* S0;                /* [N,Hv,dk,dv] or NULL (zero initial state) */
     void* o;                        /* out [B,T,Hv,dv], dtype                    */
-    float* ST;                      /* out [N,Hv,dk,dv] or NULL (not written)    */
+    float* ST;                      /* out [N,Hv,dk,dv] or NULL (not written);
+                                       must not overlap S0 (GDN_ERR_INVALID_ARG):
+                                       a split sequence may read S0 after S_T of
+                                       the same sequence was written              */
     int32_t* dev_status;            /* device int32 or NULL                      */
 } gdn_fwd_args;
 
@@ -132,13 +138,15 @@ typedef struct gdn_bwd_args {
     void* dv_out;      /* out [B,T,Hv,dv], dtype               */
     float* dbeta;      /* out [B,T,Hv] fp32                    */
     float* dg;         /* out [B,T,Hv] fp32 (w.r.t. raw g)     */
-    float* dS0;        /* out [N,Hv,dk,dv] fp32 or NULL (skip) */
+    float* dS0;        /* out [N,Hv,dk,dv] fp32 or NULL (skip);
+                          must overlap neither S0 nor dST      */
     int32_t* dev_status;
 } gdn_bwd_args;
 
 /* Bytes of device workspace gdn_chunk_fwd needs for these arguments (the
  * pointers may be NULL here; only sizes, dtype and cu_seqlens_host are read).
- * Returns GDN_OK and sets *bytes, or an argument error.  The tensor-core path
+ * Returns GDN_OK and sets *bytes, or an argument error (a status rather than a
+ * bare size, so that a bad argument cannot be mistaken for a size).  The tensor-core path
  * (bf16, dk = dv = 128) keeps three 8 KB bf16 images (T = (I + A)^-1,
  * T diag(beta Gam) and T diag(beta)) and one 8-byte gate summary per (chunk slot,
  * value head), with floor(T_total / 64) + N + 1 chunk slots; the CUDA-core path
@@ -146,6 +154,12 @@ typedef struct gdn_bwd_args {
 GDN_API gdn_status gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args, size_t* bytes);
 
 /* Forward: o and (optionally) S_T from q, k, v, beta, g and (optionally) S0.
+ * This is the forward kernel of the FlashQLA pages (news.hamidun.com "Qwen
+ * FlashQLA ... Hopper", section "What is FlashQLA": forward pass of GDN in
+ * chunked-prefill mode; its "Chunked Prefill" scenario for S0 -> S_T chaining).
+ * One sequence may be split over several SMs by its gate decay (dothoosh.com
+ * FlashQLA article, first innovation: gate-driven context parallelism) unless
+ * GDN_FLAG_SPLIT_OFF is set.
  * workspace: device memory of at least gdn_chunk_fwd_workspace_size() bytes,
  * 256-byte aligned, caller-owned, contents irrelevant on entry.
  * stream: a cudaStream_t (CUstream) handle, or NULL for the legacy stream. */
@@ -158,11 +172,15 @@ GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size
 GDN_API gdn_status gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args, size_t* bytes);
 
 /* Backward: dq, dk, dv, dbeta, dg and (optionally) dS0 of the forward above
- * for upstream gradients dout and dST.  Same workspace/stream rules. */
+ * for upstream gradients dout and dST.  Same workspace/stream rules.  This is
+ * the backward kernel of the FlashQLA pages (news.hamidun.com page, section
+ * "What is FlashQLA": forward and backward passes; dothoosh.com article,
+ * backward speed-up paragraph). */
 GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args* args, void* workspace, size_t workspace_bytes,
                          void* stream);
 
-/* Static, NUL-terminated description of a status code (never NULL). */
+/* Static, NUL-terminated description of a status code (never NULL).  The
+ * FlashQLA pages describe no interface; this belongs to the library. */
 GDN_API const char* gdn_status_string(int status);
 
 /* Forward without a workspace argument, for callers that cannot allocate device
@@ -184,12 +202,15 @@ GDN_API const char* gdn_status_string(int status);
  * The kernels write every scratch byte before reading it, so nothing needs
  * clearing between calls.  The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress, with that device current) and caches
- * it; make that first call before any stream capture. */
+ * it, keyed by the CUDA context; make that first call before any stream
+ * capture.  After cudaDeviceReset the next call looks the address up again
+ * (the new context holds a new copy of the array). */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, void* stream);
 
 /* Number of kernel launches gdn_chunk_fwd / gdn_chunk_bwd enqueue for these
- * arguments (a pure function of the arguments; -1 on an argument error). */
+ * arguments (a pure function of the arguments; -1 on an argument error).  The
+ * FlashQLA pages describe no interface; this is for launch accounting. */
 GDN_API int gdn_chunk_fwd_launch_count(const gdn_fwd_args* args);
 GDN_API int gdn_chunk_bwd_launch_count(const gdn_bwd_args* args);
 

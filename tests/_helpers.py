@@ -53,3 +53,46 @@ def gpu_unit(inp, o, ST, n, h):
         lo, hi = int(cu[n]), int(cu[n + 1])
         return o[0, lo:hi, h], ST[n, h]
     return o[n, :, h], ST[n, h]
+
+
+def units(inp, heads=None):
+    """Every (sequence, head) unit: (n, h, batch row, token slice); heads defaults to the
+    value heads."""
+    cu = inp.get("cu_seqlens")
+    heads = inp["v"].shape[2] if heads is None else heads
+    if cu is not None:
+        cu = [int(x) for x in cu.cpu()]
+        seqs = [(n, 0, slice(cu[n], cu[n + 1])) for n in range(len(cu) - 1)]
+    else:
+        seqs = [(n, n, slice(0, inp["q"].shape[1])) for n in range(inp["q"].shape[0])]
+    return [(n, h, b, sl) for n, b, sl in seqs for h in range(heads)]
+
+
+def per_unit_rel_l2(x, ref, inp, kind):
+    """rel-L2 of every (sequence, head) unit of a [B,T,H,...] token tensor (kind="tok"; H is
+    whichever head count the tensor has, q/k or value heads), a [B,T,H] per-token vector
+    (kind="vec") or a [N,Hv,dk,dv] state (kind="state").  Units whose reference is all zero
+    compare the absolute norm."""
+    x = np.asarray(x.detach().cpu().double().numpy() if hasattr(x, "detach") else x, dtype=np.float64)
+    ref = np.asarray(ref.detach().cpu().double().numpy() if hasattr(ref, "detach") else ref,
+                     dtype=np.float64)
+    out = {}
+    for n, h, b, sl in units(inp, heads=x.shape[1] if kind == "state" else x.shape[2]):
+        if kind == "state":
+            a, r = x[n, h], ref[n, h]
+        else:
+            a, r = x[b, sl, h], ref[b, sl, h]
+        den = np.linalg.norm(r.ravel())
+        num = np.linalg.norm((a - r).ravel())
+        out[(n, h)] = float(num / den) if den > 0 else float(num)
+    return out
+
+
+def assert_every_unit(x, ref, inp, kind, tol, name):
+    """Whole-tensor rel-L2 and every unit's rel-L2 below ``tol``; the message names the worst units."""
+    whole = rel_l2(x, ref)
+    per = per_unit_rel_l2(x, ref, inp, kind)
+    worst = sorted(per.items(), key=lambda kv: -kv[1])[:3]
+    assert whole < tol, f"{name}: whole-tensor rel-L2 {whole:.3e}"
+    assert worst[0][1] < tol, f"{name}: worst units {worst} (of {len(per)}), whole {whole:.3e}"
+    return whole, worst[0][1]

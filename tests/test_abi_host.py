@@ -139,3 +139,33 @@ def test_backward_argument_checks():
     assert L.gdn_chunk_bwd(ctypes.byref(a), ctypes.c_void_p(0), 0, None) == WORKSPACE
     a.dout = None
     assert L.gdn_chunk_bwd(ctypes.byref(a), ctypes.c_void_p(FAKE), n.value, None) == INVALID
+
+
+def test_aliased_states_are_rejected():
+    """S0 and S_T sharing bytes (the same buffer, or overlapping ranges) are rejected before any
+    launch: a later segment of a split sequence may read S0 after S_T was written."""
+    state = 4 * 128 * 128 * 4  # N * Hv * dk * dv fp32 of fwd_args()
+    for st_addr in (FAKE, FAKE + 256, FAKE + state - 256):
+        assert call_fwd(fwd_args(S0=FAKE, ST=st_addr)) == INVALID
+    a = GdnBwdArgs()
+    a.struct_size = ctypes.sizeof(a)
+    a.abi_version = 1
+    a.dtype = _abi.GDN_BF16
+    a.B, a.T, a.Hk, a.Hv, a.dk, a.dv = 1, 256, 2, 4, 128, 128
+    for f in ("q", "k", "v", "beta", "g", "dout", "dq", "dk_out", "dv_out", "dbeta", "dg"):
+        setattr(a, f, FAKE)
+    L = _abi.lib()
+    for s0, dst in ((FAKE, FAKE + state), (FAKE + state, FAKE)):
+        a.S0, a.dST, a.dS0 = s0, dst, FAKE + 256
+        assert L.gdn_chunk_bwd(ctypes.byref(a), ctypes.c_void_p(FAKE), 1 << 40, None) == INVALID
+
+
+def test_noalloc_checks_the_struct_before_reading_it():
+    """A caller built against a smaller (older) argument struct is rejected from its size field
+    alone, before the library copies the struct."""
+    L = _abi.lib()
+    short = (ctypes.c_uint32 * 2)(8, 1)  # struct_size = 8 bytes, abi_version = 1
+    assert L.gdn_chunk_fwd_noalloc(ctypes.cast(short, ctypes.POINTER(GdnFwdArgs)), None) == INVALID
+    wrong_abi = fwd_args(abi_version=2)
+    assert L.gdn_chunk_fwd_noalloc(ctypes.byref(wrong_abi), None) == INVALID
+    assert L.gdn_chunk_fwd_noalloc(None, None) == INVALID

@@ -1,6 +1,7 @@
 """GPU backward parity: libgdn's gdn_chunk_bwd against the oracle's float64
 adjoint on the same seeded inputs (dq, dk, dv, dbeta, dg, dS0), whole tensors
-at small sizes and sampled heads at the full backward workload size."""
+at small sizes, and whole tensors plus every (sequence, head) unit on its own at
+the full backward workload size."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +10,7 @@ import oracle
 from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE,
                                              GDN_FLAG_SPLIT_OFF, gdn_chunk_bwd)
 from gated_deltanet_chunked_fwd_b200.inputs import make_inputs, make_workload
-from tests._helpers import TOL, cpu, rel_l2
+from tests._helpers import TOL, assert_every_unit, cpu, rel_l2
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -74,16 +75,15 @@ def test_reduced_backward_workload_full_oracle():
     compare(run(inp), ref(inp), 1e-2, "reduced")
 
 
-def test_backward_workload_full_size_sampled_heads():
+def test_backward_workload_full_size_every_unit():
+    """B=4, T=8192, H=16, d=128: all six gradients against the oracle adjoint over whole
+    tensors and for every (sequence, head) unit on its own."""
     inp = make_workload(4, seed=0, device=DEV)
     mine = run(inp)
-    x = cpu(inp)
-    for b, h in [(0, 0), (3, 11)]:
-        sl = lambda t: t[b:b + 1, :, h:h + 1]
-        r = oracle.bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["beta"]), sl(x["g"]), sl(x["do"]),
-                       dST=x["dST"][b:b + 1, h:h + 1])
-        got = [sl(t) for t in mine[:5]] + [mine[5][b:b + 1, h:h + 1]]
-        compare(got, r, 1e-2, f"unit ({b},{h})")
+    refs = ref(inp)
+    kinds = ["tok", "tok", "tok", "vec", "vec", "state"]
+    for name, a, b, kind in zip(NAMES, mine, refs, kinds):
+        assert_every_unit(a, b, inp, kind, 1e-2, name)
 
 
 @pytest.mark.parametrize("flags", [0, GDN_FLAG_PORTABLE], ids=["tensor-core", "portable"])
@@ -121,3 +121,56 @@ def test_tensor_core_slow_decay_exact_fallback():
     inp = make_inputs(2, 700, 1, 2, 128, 128, dtype="bf16", seed=14, s0_std=0.1, g_mu=-6.0,
                       backward=True, device=DEV)
     compare(run(inp), ref(inp), TOL[inp["q"].dtype], "slow decay")
+
+
+def test_tensor_core_exp2_decay_fallback():
+    """Two tokens with g = -60 in one chunk push the chunk's in-chunk log-decay range past 80,
+    where the WY, replay and reverse kernels form exp(gamma_r - gamma_s) by exp2 per entry
+    instead of the factored a_r b_s."""
+    inp = make_inputs(1, 640, 2, 4, 128, 128, dtype="bf16", seed=25, s0_std=0.1, backward=True,
+                      device=DEV)
+    for c in (1, 5, 9):
+        inp["g"][0, 64 * c + 10, :] = -60.0
+        inp["g"][0, 64 * c + 40, :] = -60.0
+    r = ref(inp)
+    for flags in (0, GDN_FLAG_SPLIT_FORCE):
+        compare(run(inp, flags), r, TOL[inp["q"].dtype], f"exp2 flags={flags}")
+
+
+def test_tensor_core_norm_condition_fallback():
+    """Tokens with beta |k|^2 > 2 in every chunk: no segment may start from a truncated
+    warm-up (forward states or reverse adjoint), so every segment runs exactly."""
+    inp = make_inputs(1, 1024, 1, 2, 128, 128, dtype="bf16", seed=26, s0_std=0.1, backward=True,
+                      device=DEV)
+    k = inp["k"].float()
+    for c in range(16):
+        t = 64 * c + 13
+        k[0, t] = k[0, t] * 1.5
+        inp["beta"][0, t, :] = 1.9
+    inp["k"] = k.to(torch.bfloat16)
+    r = ref(inp)
+    for flags in (0, GDN_FLAG_SPLIT_FORCE):
+        compare(run(inp, flags), r, TOL[inp["q"].dtype], f"norm flags={flags}")
+
+
+def test_aliased_state_gradient_is_rejected():
+    """dS0 sharing memory with S0 or dS_T is rejected on the host before anything runs."""
+    import ctypes
+
+    from gated_deltanet_chunked_fwd_b200 import _abi, _fill_common
+
+    inp = make_inputs(1, 256, 1, 2, 128, 128, dtype="bf16", seed=27, s0_std=0.1, backward=True,
+                      device=DEV)
+    outs = [torch.empty_like(inp[n]) for n in ("q", "k", "v", "beta", "g")]
+    for alias in ("initial_state", "dST"):
+        a = _abi.GdnBwdArgs()
+        _, host = _fill_common(a, inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], None, None,
+                               inp["initial_state"], 0)
+        a.dout, a.dST = inp["do"].data_ptr(), inp["dST"].data_ptr()
+        a.dq, a.dk_out, a.dv_out, a.dbeta, a.dg = (t.data_ptr() for t in outs)
+        a.dS0 = inp[alias].data_ptr()
+        n = ctypes.c_size_t(0)
+        assert _abi.lib().gdn_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+        ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=DEV)
+        st = _abi.lib().gdn_chunk_bwd(ctypes.byref(a), ctypes.c_void_p(ws.data_ptr()), n.value, None)
+        assert st == 1, alias  # GDN_ERR_INVALID_ARG

@@ -1,7 +1,8 @@
 """GPU forward parity: libgdn (through the C ABI) against the float64 oracle on
 the same seeded inputs, element by element over whole tensors (rel-L2 bars in
 _helpers.TOL), at sizes that span several chunks and a ragged tail, and at the
-full workload sizes on sampled (sequence, head) units the oracle computes alone."""
+full workload sizes over whole tensors and every (sequence, value head) unit on
+its own."""
 import math
 
 import numpy as np
@@ -12,7 +13,7 @@ import oracle
 from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE,
                                              GDN_FLAG_SPLIT_OFF, gdn_chunk_fwd)
 from gated_deltanet_chunked_fwd_b200.inputs import make_inputs, make_workload
-from tests._helpers import TOL, cpu, gpu_unit, oracle_fwd_units, rel_l2
+from tests._helpers import TOL, assert_every_unit, cpu, rel_l2
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -116,28 +117,35 @@ def test_strong_gate_resets_state():
     check_full(inp)
 
 
+def check_every_unit(inp, o, ST, o_ref=None, ST_ref=None, tol=1e-2):
+    """o and S_T against the oracle over the whole tensors and unit by unit: every (sequence,
+    value head) unit's rel-L2 must pass on its own, so that one bad head or chunk cannot hide
+    in a whole-tensor norm."""
+    if o_ref is None:
+        o_ref, ST_ref = full_oracle(inp)
+    assert_every_unit(o, o_ref, inp, "tok", tol, "o")
+    assert_every_unit(ST, ST_ref, inp, "state", tol, "S_T")
+    return o_ref, ST_ref
+
+
 @pytest.mark.parametrize("seed", [0, 1])
-def test_workload1_full_size_sampled_heads(seed):
+def test_workload1_full_size_every_unit(seed):
+    """B=1, T=4096, H=16, d=128 with a random S0: all 16 heads against the oracle."""
     inp = make_workload(1, seed=seed, device=DEV)
     o, ST = run(inp)
-    assert torch.isfinite(o.float()).all()
-    for (n, h), (o_ref, ST_ref) in oracle_fwd_units(inp, [(0, 0), (0, 9), (0, 15)]).items():
-        og, Sg = gpu_unit(inp, o, ST, n, h)
-        assert rel_l2(og, o_ref) < 1e-2, (h, rel_l2(og, o_ref))
-        assert rel_l2(Sg, ST_ref) < 1e-2
+    check_every_unit(inp, o, ST)
 
 
-def test_workload2_full_size_sampled_units():
+def test_workload2_full_size_every_unit():
+    """8 packed sequences (512..16384 tokens), 16 q/k heads, 32 value heads: all 256 units."""
     inp = make_workload(2, seed=0, device=DEV)
     o, ST = run(inp)
-    for (n, h), (o_ref, ST_ref) in oracle_fwd_units(inp, [(0, 0), (3, 17), (7, 31)]).items():
-        og, Sg = gpu_unit(inp, o, ST, n, h)
-        assert rel_l2(og, o_ref) < 1e-2, ((n, h), rel_l2(og, o_ref))
-        assert rel_l2(Sg, ST_ref) < 1e-2
+    check_every_unit(inp, o, ST)
 
 
 def test_workload3_chained_prefill_equals_single_call():
-    """Four 16384-token calls chained through S_T -> S_0 equal one 65536-token call."""
+    """Four 16384-token calls chained through S_T -> S_0 equal one 65536-token call, and both
+    match the oracle on every head."""
     inp = make_workload(3, seed=0, device=DEV)
     o, ST = run(inp)
     S = None
@@ -151,8 +159,70 @@ def test_workload3_chained_prefill_equals_single_call():
     oc = torch.cat(parts, 1)
     assert rel_l2(oc, o) < 2e-3
     assert rel_l2(S, ST) < 2e-3
-    for (n, h), (o_ref, ST_ref) in oracle_fwd_units(inp, [(0, 5)]).items():
-        assert rel_l2(o[0, :, h], o_ref) < 1e-2
-        assert rel_l2(ST[0, h], ST_ref) < 1e-2
-        assert rel_l2(oc[0, :, h], o_ref) < 1e-2
-        assert rel_l2(S[0, h], ST_ref) < 1e-2
+    o_ref, ST_ref = check_every_unit(inp, o, ST)
+    check_every_unit(inp, oc, S, o_ref, ST_ref)
+
+
+# ---- branches of the tensor-core kernels that the workload distributions never reach
+
+def test_tensor_core_exp2_decay_fallback():
+    """Inside a chunk the decay factor E_rs = exp(gamma_r - gamma_s) is formed as a_r b_s while
+    every |gamma - gamma_31| < 80, else as one exp2 per entry.  Two tokens with g = -60 in the
+    same chunk push the in-chunk range past 80 (the tokens before them sit ~60 + the chunk's
+    other decay above gamma_31, the last ones ~60 below), so the WY kernel and the fused kernel
+    take their exp2 branch for that chunk; the other chunks stay factored."""
+    inp = make_inputs(1, 640, 2, 4, 128, 128, dtype="bf16", seed=21, s0_std=0.1, device=DEV)
+    for c in (1, 5, 9):  # chunks 1, 5 and 9 of every head
+        inp["g"][0, 64 * c + 10, :] = -60.0
+        inp["g"][0, 64 * c + 40, :] = -60.0
+    g = inp["g"][0, 64:128, 0].double()
+    gam = torch.cumsum(g, 0)
+    assert (gam - gam[31]).abs().max() >= 80.0  # the branch condition holds
+    for flags in (0, GDN_FLAG_SPLIT_FORCE):
+        o, ST = run(inp, flags)
+        check_every_unit(inp, o, ST)
+
+
+def test_tensor_core_norm_condition_fallback():
+    """A segment that does not start its sequence begins from a zero state a few chunks early
+    only while every warm-up token keeps 0 <= beta |k|^2 <= 2 (then each token's state map has
+    norm <= exp(g)); a token with beta |k|^2 > 2 in the warm-up makes the segment replay its
+    sequence exactly from S0.  Forced short segments (two chunks) and one token per chunk with
+    beta = 1.9, |k|^2 = 2.25 (beta |k|^2 = 4.3) reach that branch in every later segment."""
+    inp = make_inputs(1, 1024, 1, 2, 128, 128, dtype="bf16", seed=22, s0_std=0.1, device=DEV)
+    k = inp["k"].float()
+    for c in range(16):
+        t = 64 * c + 13
+        k[0, t] = k[0, t] * 1.5  # |k|^2 = 2.25 (k is unit-norm)
+        inp["beta"][0, t, :] = 1.9
+    inp["k"] = k.to(torch.bfloat16)
+    assert (inp["beta"][0, 13, 0] * inp["k"][0, 13, 0].float().pow(2).sum()) > 2.0
+    for flags in (0, GDN_FLAG_SPLIT_FORCE):
+        o, ST = run(inp, flags)
+        check_every_unit(inp, o, ST)
+
+
+def test_tensor_core_weak_decay_forward_fallback():
+    """Weak decay, g = -softplus(N(-6, 1)) (about -0.0025 per token): the summed log decay of a
+    64-chunk sequence never reaches log(2^-30), so every segment after the first replays its
+    sequence from S0 and writes its own outputs (auto split)."""
+    inp = make_inputs(1, 4096, 2, 4, 128, 128, dtype="bf16", seed=23, s0_std=0.1, g_mu=-6.0,
+                      device=DEV)
+    assert float(inp["g"][0, :, 0].double().sum()) > -30 * math.log(2)
+    o, ST = run(inp)
+    check_every_unit(inp, o, ST)
+
+
+def test_aliased_initial_and_final_state_is_rejected():
+    """S0 and S_T in one buffer (an in-place state update) is rejected on the host: a later
+    segment of a split sequence may read S0 after S_T was written."""
+    from gated_deltanet_chunked_fwd_b200 import GdnError
+
+    inp = make_inputs(1, 2048, 1, 2, 128, 128, dtype="bf16", seed=24, s0_std=0.1, g_mu=-2.0,
+                      device=DEV)
+    S = inp["initial_state"]
+    for flags in (0, GDN_FLAG_SPLIT_FORCE):
+        with pytest.raises(GdnError) as e:
+            gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], initial_state=S,
+                          final_state=S, flags=flags)
+        assert e.value.status == 1  # GDN_ERR_INVALID_ARG

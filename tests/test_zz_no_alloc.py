@@ -3,18 +3,20 @@
 
 It keeps its scratch in a fixed device array inside libgdn.so instead of a
 caller-provided workspace.  Checked here through the C ABI against the regular
-gdn_chunk_fwd on the same inputs, on two calls in a row (the array keeps the
-previous call's contents, which must not leak into the next result).  This file
+gdn_chunk_fwd on the same inputs and against the float64 oracle, on two calls
+in a row (the array keeps the previous call's contents, which must not leak
+into the next result).  This file
 is collected last on purpose, so that a failure here stops a `-x` run only after
 every other test has run."""
 import ctypes
 
+import oracle
 import pytest
 import torch
 
 from gated_deltanet_chunked_fwd_b200 import _abi, _fill_common, gdn_chunk_fwd
 from gated_deltanet_chunked_fwd_b200.inputs import make_inputs
-from tests._helpers import TOL, rel_l2
+from tests._helpers import TOL, cpu, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +51,11 @@ def test_noalloc_matches_gdn_chunk_fwd_twice(dt, lengths, s0):
         tol = TOL[x["q"].dtype]
         assert rel_l2(o, o_ref) < tol, rel_l2(o, o_ref)
         assert rel_l2(ST, ST_ref) < tol, rel_l2(ST, ST_ref)
+        c = cpu(x)
+        o_or, ST_or = oracle.fwd(c["q"], c["k"], c["v"], c["beta"], c["g"],
+                                 cu_seqlens=c.get("cu_seqlens"), initial_state=c.get("initial_state"))
+        assert rel_l2(o, o_or) < tol, rel_l2(o, o_or)
+        assert rel_l2(ST, ST_or) < tol, rel_l2(ST, ST_or)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
