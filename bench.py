@@ -17,6 +17,8 @@ Extra keys, each timed the same way: ``fwd_workloads`` holds the 4,096-token
 forward with a random initial state, the packed varlen batch (8 sequences,
 16 q/k heads, 32 value heads) and the long context fed as 4 chained
 16,384-token calls; ``bwd`` the backward on the B=4, T=8192, H=16 workload.
+``fwd_workloads`` also holds the decode step (one token for each of 64
+sequences, 16 q/k heads, 32 value heads, fp32 states updated in place).
 ``cpu_baseline`` times the float64 oracle on a bounded sample of the headline
 workload on the host cores.
 
@@ -354,6 +356,46 @@ class FwdCall:
                          s0=self.S0 is not None, st=True)
 
 
+DECODE = dict(N=64, Hk=16, Hv=32, dk=128, dv=128)
+
+
+def decode_bytes(N, Hk, Hv, dk, dv, elt=2):
+    """Algorithmic HBM bytes of one decode step: read and write every fp32 state; read q, k, v,
+    beta, g; write o."""
+    return N * (Hv * (2 * dk * dv * 4 + 2 * dv * elt + 8) + 2 * Hk * dk * elt)
+
+
+def decode_bench(dev, stream, rank, measure, world, hbm, bf16, src, steps):
+    """One decode token for each of 64 sequences (16 q/k heads, 32 value heads, d = 128, bf16
+    tokens, fp32 states updated in place) through the C ABI."""
+    import ctypes
+
+    import gated_deltanet_chunked_fwd_b200 as gdn
+    from gated_deltanet_chunked_fwd_b200 import _abi
+    from gated_deltanet_chunked_fwd_b200.inputs import make_inputs
+
+    d = DECODE
+    x = make_inputs(d["N"], 1, d["Hk"], d["Hv"], d["dk"], d["dv"], dtype="bf16", seed=rank,
+                    s0_std=0.1, device=dev)
+    c0 = {n: x[n][:, 0].contiguous() for n in ("q", "k", "v", "beta", "g")}
+    S = x["initial_state"]
+    o = torch.empty(c0["v"].shape, dtype=torch.bfloat16, device=dev)
+    a = gdn._decode_args(c0["q"], c0["k"], c0["v"], c0["beta"], c0["g"], S, None, o)
+    L = _abi.lib()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def step():
+        st = L.gdn_decode_step(ctypes.byref(a), sp)
+        if st != 0:
+            raise gdn.GdnError("gdn_decode_step", st)
+
+    m = measure(step, steps)
+    byts = decode_bytes(**d)
+    flops = d["N"] * d["Hv"] * 8 * d["dk"] * d["dv"]  # two dots and the rank-1 update per state
+    return {"ms": m, "tokens_per_s": job_throughput(d["N"], world, m), "launches": 1,
+            "roofline": roofline(flops, byts, m * 1e-3, hbm, bf16, src)}
+
+
 def run_ours(args, world, rank, local):
     import gated_deltanet_chunked_fwd_b200 as gdn
     from gated_deltanet_chunked_fwd_b200.inputs import WORKLOADS, make_workload
@@ -460,6 +502,8 @@ def run_ours(args, world, rank, local):
             "launches": sum(c.launches for c in parts),
             "roofline": roofline(dense * tokens * Hv, cb, m * 1e-3, hbm, bf16, src)}
         del parts
+        extra["decode_bf16_N64_Hk16_Hv32_d128"] = decode_bench(dev, stream, rank, measure, world,
+                                                               hbm, bf16, src, args.steps)
 
     # ---- backward on its own workload
     bwd = None

@@ -1,7 +1,7 @@
 """GDN chunked prefill (forward and backward) on NVIDIA B200 -- Python binding.
 
-``gdn_chunk_fwd`` / ``gdn_chunk_bwd`` mirror the C entry points of
-``include/gdn.h`` one to one.  This module marshals torch tensors into the C
+``gdn_chunk_fwd`` / ``gdn_chunk_bwd`` / ``gdn_decode_step`` mirror the C entry
+points of ``include/gdn.h`` one to one.  This module marshals torch tensors into the C
 argument structs, allocates the outputs and the workspace with torch (device
 memory) and passes torch's current CUDA stream.  All arithmetic runs in the
 library's CUDA kernels; there is no CPU or PyTorch fallback.
@@ -20,11 +20,11 @@ import torch
 
 from . import _abi
 from ._abi import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE, GDN_FLAG_SPLIT_OFF, GdnBwdArgs,
-                   GdnError, GdnFwdArgs)
+                   GdnDecodeArgs, GdnError, GdnFwdArgs)
 
-__all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_chunk_fwd_workspace_size",
+__all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_size",
            "gdn_chunk_bwd_workspace_size", "chunk_fwd", "chunk_bwd", "GdnError",
-           "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE"]
+           "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE", "decode_step"]
 
 _DT = {torch.float32: _abi.GDN_F32, torch.bfloat16: _abi.GDN_BF16}
 
@@ -177,6 +177,51 @@ def gdn_chunk_bwd(q, k, v, beta, g, do, cu_seqlens=None, initial_state=None, dST
     return dq, dk, dv, dbeta, dg, dS0
 
 
+def _decode_args(q, k, v, beta, g, state, state_indices, o):
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[0] != q.shape[0]:
+        raise ValueError("q, k must be [N, Hk, dk] and v [N, Hv, dv]")
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype: float32 or bfloat16")
+    if beta.dtype != torch.float32 or g.dtype != torch.float32 or state.dtype != torch.float32:
+        raise ValueError("beta, g and the state must be float32")
+    N, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    a = GdnDecodeArgs()
+    a.struct_size = ctypes.sizeof(a)
+    a.abi_version = _abi.GDN_ABI_VERSION
+    a.dtype = _DT[q.dtype]
+    a.N, a.Hk, a.Hv, a.dk, a.dv = N, Hk, Hv, dk, dv
+    if state_indices is not None:
+        if state_indices.dtype != torch.int32 or state_indices.shape != (N,):
+            raise ValueError("state_indices must be int32 [N]")
+        a.num_slots = state.shape[0]
+    elif state.shape[0] != N:
+        raise ValueError("without state_indices the state must be [N, Hv, dk, dv]")
+    if tuple(state.shape[1:]) != (Hv, dk, dv):
+        raise ValueError(f"state must be float32 [slots, {Hv}, {dk}, {dv}]")
+    a.q, a.k, a.v, a.beta, a.g = _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g)
+    a.S, a.state_indices, a.o = _ptr(state), _ptr(state_indices), _ptr(o)
+    return a
+
+
+def gdn_decode_step(q, k, v, beta, g, state, state_indices=None, *, out=None,
+                    check_device_status: bool = False):
+    """One decode token per sequence; updates ``state`` in place and returns o [N, Hv, dv].
+
+    q, k: [N, Hk, dk]; v: [N, Hv, dv] (one dtype, fp32 or bf16); beta, g: [N, Hv] fp32;
+    state: fp32 [N, Hv, dk, dv] (H = S^T, as S_T of gdn_chunk_fwd), or a pool of slots
+    [num_slots, Hv, dk, dv] indexed by ``state_indices`` (int32 [N] on the device; negative
+    = skip that sequence).
+    """
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    a = _decode_args(q, k, v, beta, g, state, state_indices, o)
+    st = _dev_status(q.device, check_device_status)
+    a.dev_status = _ptr(st)
+    _check("gdn_decode_step", _abi.lib().gdn_decode_step(ctypes.byref(a), _stream(q.device)))
+    _raise_dev_status("gdn_decode_step", st)
+    return o
+
+
 def launch_count(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None, initial_state=None,
                  flags: int = 0, backward: bool = False) -> int:
     """Kernel launches one gdn_chunk_fwd (or _bwd) call enqueues for these arguments."""
@@ -190,3 +235,4 @@ def launch_count(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None, initia
 # chunk_bwd(...) -> (dq, dk, dv, dbeta, dg, dS0) are the same calls
 chunk_fwd = gdn_chunk_fwd
 chunk_bwd = gdn_chunk_bwd
+decode_step = gdn_decode_step

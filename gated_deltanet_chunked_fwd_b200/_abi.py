@@ -52,10 +52,19 @@ class GdnBwdArgs(ctypes.Structure):
     ]
 
 
+class GdnDecodeArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _u32), ("abi_version", _u32), ("dtype", _i32), ("N", _i32),
+        ("Hk", _i32), ("Hv", _i32), ("dk", _i32), ("dv", _i32), ("num_slots", _i32),
+        ("flags", _u32), ("q", _p), ("k", _p), ("v", _p), ("beta", _p), ("g", _p), ("S", _p),
+        ("state_indices", _p), ("o", _p), ("dev_status", _p),
+    ]
+
+
 EXPORTS = [
     "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_launch_count",
     "gdn_chunk_bwd_workspace_size", "gdn_chunk_bwd", "gdn_chunk_bwd_launch_count",
-    "gdn_status_string", "gdn_chunk_fwd_noalloc",
+    "gdn_status_string", "gdn_chunk_fwd_noalloc", "gdn_decode_step",
 ]
 
 _lib = None
@@ -86,6 +95,8 @@ def lib() -> ctypes.CDLL:
         for fn in ("gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
                    "gdn_chunk_bwd", "gdn_chunk_fwd_launch_count", "gdn_chunk_bwd_launch_count"):
             getattr(L, fn).restype = ctypes.c_int
+        L.gdn_decode_step.argtypes = [ctypes.POINTER(GdnDecodeArgs), _p]
+        L.gdn_decode_step.restype = ctypes.c_int
         L.gdn_chunk_fwd_noalloc.argtypes = [F, _p]
         L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]

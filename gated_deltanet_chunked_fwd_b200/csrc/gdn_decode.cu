@@ -1,0 +1,207 @@
+// gdn_decode.cu -- one recurrent (decode) step of the gated delta rule per (sequence, value
+// head), applied to the state in place.  This is the step that follows a chunked prefill when
+// a model generates token by token (news.hamidun.com "Qwen FlashQLA ... Hopper", scenario list:
+// edge inference and distributed inference, several model calls in one stream); it consumes
+// the S_T that gdn_chunk_fwd returns, in the same transposed layout H = S^T, [dk][dv].
+//
+// Per (sequence n, value head h), with H the state of slot s(n):
+//   H <- exp(g) H,   p = H^T k,   H <- H + beta k (v - p)^T,   o = H^T q.
+// Column j of H (a dv index) only meets k, q, v_j and the scalars, so with
+//   a_j = H_old[:, j] . k,  b_j = H_old[:, j] . q,  d_j = beta (v_j - exp(g) a_j):
+//   H_new[:, j] = exp(g) H_old[:, j] + d_j k,   o_j = exp(g) b_j + (k . q) d_j.
+// The step is bound by HBM: each state (dk x dv fp32) is read once and written once.
+//
+// Kernel: one 256-thread CTA per (sequence, value head).  Thread t owns the four state columns
+// 4 (t % 32) .. + 3 and the rows t / 32, t / 32 + 8, ... (16 rows at dk = 128), so that warp w
+// reads and writes whole 512-byte rows with 16-byte accesses.  The state goes into registers
+// with all loads in flight at once (64 KB per CTA at d = 128), the two column dots are reduced
+// over the eight row groups in shared memory, and the new state is written back from registers:
+// no thread reads a state element after another thread wrote it, so the update in place is safe
+// within a CTA, and different CTAs own different states.
+#include "gdn_dtype.cuh"
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kDecThreads = 256;
+constexpr int kRowGroups = kDecThreads / 32;           // 8
+constexpr int kRowsPerThread = kMaxHead / kRowGroups;  // 16
+
+struct DecodeArgs {
+    int N, Hk, Hv, dk, dv, group, num_slots;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* beta;
+    const float* g;
+    float* S;
+    const int32_t* idx;
+    void* o;
+    int32_t* status;
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArgs a) {
+    __shared__ float sk[kMaxHead], sq[kMaxHead], sv[kMaxHead];
+    __shared__ float4 pa[kRowGroups][32], pb[kRowGroups][32];  // partial column dots
+    __shared__ float colA[kMaxHead], colB[kMaxHead];
+    __shared__ float skq;
+    const int h = blockIdx.x % a.Hv, n = blockIdx.x / a.Hv, hk = h / a.group;
+    const int t = threadIdx.x, cg = t & 31, rg = t >> 5;
+    const int dk = a.dk, dv = a.dv;
+    const int slot = a.idx ? a.idx[n] : n;
+    Tin* o = (Tin*)a.o + ((int64_t)n * a.Hv + h) * dv;
+    if (slot < 0) {  // padding entry of a batch: no state, zero output
+        if (t < dv) store_as(o + t, 0.f);
+        return;
+    }
+    if (slot >= a.num_slots) {
+        if (t == 0) report(a.status, GDN_ERR_DEVICE);
+        return;
+    }
+    float* S = a.S + ((int64_t)slot * a.Hv + h) * dk * dv;
+    const bool col_ok = 4 * cg < dv;
+
+    // ---- the state into registers: every load issued before any is used
+    float4 Hr[kRowsPerThread];
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        const int i = rg + kRowGroups * r;
+        Hr[r] = (col_ok && i < dk) ? *reinterpret_cast<const float4*>(S + (int64_t)i * dv + 4 * cg)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const Tin* qp = (const Tin*)a.q + ((int64_t)n * a.Hk + hk) * dk;
+    const Tin* kp = (const Tin*)a.k + ((int64_t)n * a.Hk + hk) * dk;
+    const Tin* vp = (const Tin*)a.v + ((int64_t)n * a.Hv + h) * dv;
+    if (t < dk) {
+        sk[t] = to_f(kp[t]);
+        sq[t] = to_f(qp[t]);
+    }
+    if (t < dv) sv[t] = to_f(vp[t]);
+    const float eg = expf(a.g[(int64_t)n * a.Hv + h]);
+    const float bt = a.beta[(int64_t)n * a.Hv + h];
+    __syncthreads();
+    if (rg == 0) {  // k . q by warp 0
+        float s = 0.f;
+        for (int i = cg; i < dk; i += 32) s += sk[i] * sq[i];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (cg == 0) skq = s;
+    }
+
+    // ---- column dots a_j = H[:, j] . k and b_j = H[:, j] . q over this thread's rows
+    float4 da = make_float4(0.f, 0.f, 0.f, 0.f), db = da;
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        const int i = rg + kRowGroups * r;
+        const float kk = i < dk ? sk[i] : 0.f, qq = i < dk ? sq[i] : 0.f;
+        da.x += Hr[r].x * kk; da.y += Hr[r].y * kk; da.z += Hr[r].z * kk; da.w += Hr[r].w * kk;
+        db.x += Hr[r].x * qq; db.y += Hr[r].y * qq; db.z += Hr[r].z * qq; db.w += Hr[r].w * qq;
+    }
+    pa[rg][cg] = da;
+    pb[rg][cg] = db;
+    __syncthreads();
+    if (t < 2 * 32) {  // sum the eight row groups: threads 0-31 for a, 32-63 for b
+        const int c = t & 31;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int g8 = 0; g8 < kRowGroups; ++g8) {
+            const float4 x = t < 32 ? pa[g8][c] : pb[g8][c];
+            s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
+        }
+        float* dst = t < 32 ? colA : colB;
+        if (4 * c < dv) *reinterpret_cast<float4*>(dst + 4 * c) = s;
+    }
+    __syncthreads();
+
+    // ---- d_j, the new state, and the output
+    if (!col_ok) return;
+    float d[4], ob[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int j = 4 * cg + e;
+        d[e] = bt * (sv[j] - eg * colA[j]);
+        ob[e] = eg * colB[j] + skq * d[e];
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        const int i = rg + kRowGroups * r;
+        if (i < dk) {
+            const float kk = sk[i];
+            float4 w;
+            w.x = eg * Hr[r].x + kk * d[0];
+            w.y = eg * Hr[r].y + kk * d[1];
+            w.z = eg * Hr[r].z + kk * d[2];
+            w.w = eg * Hr[r].w + kk * d[3];
+            *reinterpret_cast<float4*>(S + (int64_t)i * dv + 4 * cg) = w;
+        }
+    }
+    if (rg == 0) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) store_as(o + 4 * cg + e, ob[e]);
+    }
+}
+
+}  // namespace
+
+gdn_status plan_decode(const gdn_decode_args* a) {
+    if (!a) return GDN_ERR_INVALID_ARG;
+    if (a->struct_size < sizeof(gdn_decode_args) || a->abi_version != GDN_ABI_VERSION)
+        return GDN_ERR_INVALID_ARG;
+    if (a->dtype != GDN_F32 && a->dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (a->N < 0 || a->Hk < 1 || a->Hv < 1 || a->Hv % a->Hk != 0) return GDN_ERR_INVALID_ARG;
+    if (a->dk < 1 || a->dv < 1 || a->dk > kMaxHead || a->dv > kMaxHead || a->dv % 4 != 0)
+        return GDN_ERR_UNSUPPORTED;
+    const int64_t slots = a->state_indices ? (int64_t)a->num_slots : (int64_t)a->N;
+    if (a->state_indices && a->num_slots < 1) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)a->N * a->Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (a->N == 0) return GDN_OK;
+    const uintptr_t align16 = 15;
+    if (!a->q || !a->k || !a->v || !a->beta || !a->g || !a->S || !a->o) return GDN_ERR_INVALID_ARG;
+    if (((uintptr_t)a->S & align16) || ((uintptr_t)a->beta & 3) || ((uintptr_t)a->g & 3) ||
+        ((uintptr_t)a->state_indices & 3) || ((uintptr_t)a->dev_status & 3))
+        return GDN_ERR_INVALID_ARG;
+    const size_t elt = a->dtype == GDN_BF16 ? 2 : 4;
+    if (((uintptr_t)a->q | (uintptr_t)a->k | (uintptr_t)a->v | (uintptr_t)a->o) % elt)
+        return GDN_ERR_INVALID_ARG;
+    (void)slots;
+    return GDN_OK;
+}
+
+gdn_status launch_decode(const gdn_decode_args* a, cudaStream_t s) {
+    if (a->N == 0) return GDN_OK;
+    DecodeArgs d;
+    d.N = a->N;
+    d.Hk = a->Hk;
+    d.Hv = a->Hv;
+    d.dk = a->dk;
+    d.dv = a->dv;
+    d.group = a->Hv / a->Hk;
+    d.num_slots = a->state_indices ? a->num_slots : a->N;
+    d.q = a->q;
+    d.k = a->k;
+    d.v = a->v;
+    d.beta = a->beta;
+    d.g = a->g;
+    d.S = a->S;
+    d.idx = a->state_indices;
+    d.o = a->o;
+    d.status = a->dev_status;
+    const unsigned grid = (unsigned)((int64_t)a->N * a->Hv);
+    if (a->dtype == GDN_BF16)
+        gdn_decode_kernel<__nv_bfloat16><<<grid, kDecThreads, 0, s>>>(d);
+    else
+        gdn_decode_kernel<float><<<grid, kDecThreads, 0, s>>>(d);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace gdn
+
+extern "C" gdn_status gdn_decode_step(const gdn_decode_args* args, void* stream) {
+    using namespace gdn;
+    const gdn_status st = plan_decode(args);
+    if (st) return st;
+    (void)cudaGetLastError();
+    return launch_decode(args, (cudaStream_t)stream);
+}

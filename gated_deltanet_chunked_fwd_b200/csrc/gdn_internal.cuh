@@ -120,6 +120,10 @@ gdn_status launch_simt_state(const Problem& p, const ChunkTable& ct, const float
 gdn_status launch_simt_output(const Problem& p, const ChunkTable& ct, const float* U,
                               const float* gam, const float* Hc, cudaStream_t s);
 
+// decode step (gdn_decode.cu)
+gdn_status plan_decode(const gdn_decode_args* a);
+gdn_status launch_decode(const gdn_decode_args* a, cudaStream_t s);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace gdn

@@ -208,6 +208,45 @@ GDN_API const char* gdn_status_string(int status);
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, void* stream);
 
+/* Arguments of one decode step: one new token for each of N sequences.
+ * struct_size = sizeof(gdn_decode_args), abi_version = GDN_ABI_VERSION. */
+typedef struct gdn_decode_args {
+    uint32_t struct_size;
+    uint32_t abi_version;
+    int32_t dtype;     /* gdn_dtype of q, k, v and o                                */
+    int32_t N;         /* sequences in the batch (one token each); 0 is a no-op      */
+    int32_t Hk, Hv;    /* q/k heads, value heads (Hv % Hk == 0, contiguous groups)   */
+    int32_t dk, dv;    /* head dims, 1..128, dv a multiple of 4                      */
+    int32_t num_slots; /* states in S when state_indices != NULL (else N)            */
+    uint32_t flags;    /* reserved, 0                                                */
+    const void* q;     /* [N, Hk, dk] dtype                                          */
+    const void* k;     /* [N, Hk, dk] dtype                                          */
+    const void* v;     /* [N, Hv, dv] dtype                                          */
+    const float* beta; /* [N, Hv] fp32                                               */
+    const float* g;    /* [N, Hv] fp32, raw log decay, finite                        */
+    float* S;          /* in/out [num_slots, Hv, dk, dv] fp32, H = S^T layout as S_T;
+                          16-byte aligned                                            */
+    const int32_t* state_indices; /* device int32 [N] or NULL: sequence n updates
+                          slot state_indices[n] of S (a state pool, as in continuous
+                          batching); a negative index skips the sequence and writes
+                          zeros to its o; indices must be distinct (two sequences on
+                          one slot race); NULL means slot n                          */
+    void* o;           /* out [N, Hv, dv] dtype                                      */
+    int32_t* dev_status; /* device int32 or NULL: GDN_ERR_DEVICE for an index
+                          >= num_slots (that sequence is skipped)                    */
+} gdn_decode_args;
+
+/* Decode step: for every sequence n and value head h, with H the state in its slot,
+ *     H <- exp(g) H,   H <- H + beta k (v - H^T k)^T,   o = H^T q,
+ * i.e. one token of the gated delta rule applied to S in place (S_T of a prefill
+ * call can be passed as S directly).  This is the token-by-token step that
+ * follows chunked prefill in the inference scenarios of the FlashQLA pages
+ * (news.hamidun.com "Qwen FlashQLA ... Hopper", scenario list: edge inference;
+ * distributed inference with several model calls in one stream).  One kernel
+ * launch; each state is read once and written once.  Asynchronous on `stream`;
+ * argument errors return before anything is enqueued.  Needs no workspace. */
+GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, void* stream);
+
 /* Number of kernel launches gdn_chunk_fwd / gdn_chunk_bwd enqueue for these
  * arguments (a pure function of the arguments; -1 on an argument error).  The
  * FlashQLA pages describe no interface; this is for launch accounting. */

@@ -169,3 +169,32 @@ def test_noalloc_checks_the_struct_before_reading_it():
     wrong_abi = fwd_args(abi_version=2)
     assert L.gdn_chunk_fwd_noalloc(ctypes.byref(wrong_abi), None) == INVALID
     assert L.gdn_chunk_fwd_noalloc(None, None) == INVALID
+
+
+def test_decode_argument_checks():
+    """gdn_decode_step rejects bad arguments on the host; N = 0 is a no-op."""
+    L = _abi.lib()
+
+    def dargs(**kw):
+        a = _abi.GdnDecodeArgs()
+        a.struct_size = ctypes.sizeof(a)
+        a.abi_version = 1
+        a.dtype = _abi.GDN_BF16
+        a.N, a.Hk, a.Hv, a.dk, a.dv = 4, 2, 4, 128, 128
+        a.q = a.k = a.v = a.o = a.S = FAKE
+        a.beta = a.g = FAKE
+        for k_, v_ in kw.items():
+            setattr(a, k_, v_)
+        return a
+
+    call = lambda a: L.gdn_decode_step(ctypes.byref(a), None)
+    assert call(dargs(struct_size=8)) == INVALID
+    assert call(dargs(abi_version=3)) == INVALID
+    assert call(dargs(dtype=5)) == UNSUPPORTED
+    assert call(dargs(Hv=3)) == INVALID
+    assert call(dargs(dv=130)) == UNSUPPORTED
+    assert call(dargs(dv=30)) == UNSUPPORTED  # dv must be a multiple of 4
+    assert call(dargs(S=FAKE + 8)) == INVALID  # 16-byte aligned state
+    assert call(dargs(q=None)) == INVALID
+    assert call(dargs(state_indices=FAKE, num_slots=0)) == INVALID
+    assert call(dargs(N=0)) == OK

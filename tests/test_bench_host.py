@@ -47,3 +47,9 @@ def test_roofline_bound_is_the_larger_time():
     r = bench.roofline(flops_dense=1e13, byts=1e6, seconds=0.02, hbm_gbs=hbm, bf16_tflops=tc, src="x")
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["frac"] == pytest.approx(r["frac_tensor"])
+
+
+def test_decode_bytes():
+    # one state read and written (2 x 64 KB) + q, k (shared by 2 heads) + v, o bf16 + beta, g
+    b = bench.decode_bytes(1, 1, 2, 128, 128)
+    assert b == 2 * (2 * 65536 + 2 * 256 + 8) + 2 * 256
