@@ -599,11 +599,15 @@ __global__ void __launch_bounds__(kNT, 1)
                             for (int e = 0; e < 8; ++e) E[e] = exp2f(ar - bb[e]);
                         }
                     }
+                    // Outside the causal mask E may overflow (the decay factor of an entry above the
+                    // diagonal is a growth factor): every product below uses E only through a
+                    // select, so that no 0 * inf reaches the sums.
                     if (m < 64) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int s = sb + e;
                             const bool in = (s <= r && r < lc);
+                            E[e] = in ? E[e] : 0.f;
                             const float P = in ? x[e] * E[e] : 0.f;
                             const float dP = in ? d[e] : 0.f;
                             rowsum += dP * P;
@@ -617,6 +621,7 @@ __global__ void __launch_bounds__(kNT, 1)
                         for (int e = 0; e < 8; ++e) {
                             const int s = sb + e;
                             const bool in = (s < r && r < lc);
+                            E[e] = in ? E[e] : 0.f;
                             const float dA = in ? -d[e] : 0.f;
                             const float KE = x[e] * E[e];
                             const float A = br * KE;
