@@ -306,6 +306,18 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* v) {
         : "memory");
 }
 
+// 16 consecutive 32-bit TMEM columns of this warp's lanes -> 16 registers per thread; waits.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 // 16 packed 32-bit words per thread -> 16 consecutive TMEM columns of this warp's lanes; waits.
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
     asm volatile(

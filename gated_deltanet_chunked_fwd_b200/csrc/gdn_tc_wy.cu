@@ -13,12 +13,12 @@
 //
 // The work per chunk is small and latency-bound (a 64 x 64 x 128 Gram block and a 64 x 64
 // triangular inverse), so the kernel is built for many chunks in flight rather than for one
-// fast chunk: 128 threads, 72 registers and about 23 KB of shared memory per CTA, seven CTAs
-// per SM, so that a 4096-token, 16-head call (1024 chunks) runs as one wave.  The K tile
-// comes in by TMA.  The Gram block K K^T is formed with warp-level mma.sync (bf16 in, fp32
-// out): its fragments stay in registers, where the gate scaling turns them into A without a
-// TMEM round trip.  The inverse is blocked: the four 16 x 16 diagonal blocks by fp32
-// substitution, then three merge levels on the tensor cores (warp mma.sync in tf32).
+// fast chunk: 128 threads, 72 registers, about 25 KB of shared memory and 64 TMEM columns per
+// CTA, seven CTAs per SM, so that a 4096-token, 16-head call (1024 chunks) runs as one wave.  The
+// K tile comes in by TMA.  The Gram block K K^T is one tcgen05 MMA group (M = 128, N = 64, bf16
+// in, fp32 out in TMEM); two warps read its rows and scale them into A.  The inverse is blocked:
+// the four 16 x 16 diagonal blocks by fp32 substitution, then three merge levels as warp-level
+// tf32 MMAs (gdn_tc_inverse.cuh).
 //
 // A and T share one fp32 64 x 64 array X: A is strictly lower and T unit lower-triangular,
 // so A sits below the diagonal and T (off its unit diagonal) above it, transposed:
@@ -47,26 +47,17 @@ constexpr uint32_t wK = 0;                          // 16 KB bf16 K [dk half][64
                                                     // then fp32 X [64][kXs]
 constexpr uint32_t wYs = 64 * kXs * 4;              // fp32 [4 warps][16][9] merge scratch
 constexpr uint32_t wVec = wYs + 4 * 16 * 9 * 4;     // beta, gamma, a, b, |k|^2, beta Gam: 6 x 64 fp32
-constexpr uint32_t wBar = wVec + 6 * 64 * 4;        // mbarrier of the K tile
-constexpr uint32_t wSmemBytes = wBar + 16 + 1024;   // + alignment slack
+constexpr uint32_t wBar = wVec + 6 * 64 * 4;        // mbarriers of the K tile and the Gram MMA,
+                                                    // TMEM base
+// The Gram MMA reads its A operand as 128 rows (1024-byte groups of 8): the K tile's rows are
+// 0-63; rows 64-127 of the second k-half lie 8 KB past the tile and only feed D rows 64-127,
+// which are never read.  They must still lie inside this CTA's shared memory.
+constexpr uint32_t wAReach = wK + 3 * 8192;
+constexpr uint32_t wSmemBytes = (wBar + 32 > wAReach ? wBar + 32 : wAReach) + 1024;  // + alignment slack
+constexpr uint32_t kWyTmemCols = 64;                // D = [K;*] K^T: 128 lanes x 64 fp32 columns
 static_assert(wYs >= 16384, "X covers the K tile it replaces");
 static_assert(wSmemBytes * kWyMinBlocks + kWyMinBlocks * 1024 <= 228 * 1024, "CTAs per SM");
-
-// 4 8x8 b16 matrices from shared memory (lane groups of 8 give the row addresses of matrix 0..3)
-__device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-// D += A B for one 16 x 8 x 16 tile: A row-major bf16, B column-major bf16, D fp32
-__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-        "{%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
+static_assert(kWyTmemCols * kWyMinBlocks <= 512, "TMEM columns per SM");
 
 // Image slot x -> (sequence n, chunk c of it, its first token and length); false when the
 // slot belongs to no chunk.  The slot of sequence n's first chunk, floor(bos_n / 64) + n, is
@@ -98,24 +89,34 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
                      float2* __restrict__ summ) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    // the forward's state-chain kernel may be scheduled as soon as every CTA of this grid has
-    // started (it waits for this grid's completion before reading the images)
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) prefetch_tensormap(&tm_k);  // its first use is a few hundred cycles away
     const int h = blockIdx.y, hk = h / p.group, Hv = p.Hv;
     int n = 0, c = 0;
     int64_t bos = 0, len = 0;
-    if (!locate_slot(p, blockIdx.x, &n, &c, &bos, &len)) return;  // CTA-uniform
+    const bool live = locate_slot(p, blockIdx.x, &n, &c, &bos, &len);  // CTA-uniform
+    uint64_t* bar = (uint64_t*)(sm + wBar);
+    uint64_t* bar_mma = bar + 1;
+    uint32_t* tmem_slot = (uint32_t*)(bar + 2);
+    // TMEM for the Gram block, taken before the dependent grid may launch: that grid's CTAs take
+    // all 512 columns of an SM and then wait for this grid, so they must find ours already held
+    if (live && warp == 0) {
+        tmem_alloc(tmem_slot, kWyTmemCols);
+        tmem_relinquish();
+    }
+    // the forward's state-chain kernel may be scheduled as soon as every CTA of this grid has
+    // started (it waits for this grid's completion before reading the images)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!live) return;
     const int64_t t0 = bos + (int64_t)c * kChunk;
     const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-    uint64_t* bar = (uint64_t*)(sm + wBar);
 
     // ---- K tile by TMA ([dk half][64 rows][128 B], 128-byte swizzled).  Rows past the chunk
     // (the next sequence's tokens, or zeros past the tensor's end) only reach entries of A that
     // the mask below sets to zero.  The chunk's gates are loaded meanwhile.
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar_mma, 1);
         fence_barrier_init();
     }
     float x = 0.f, bt = 0.f;
@@ -123,7 +124,10 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         x = p.g[(t0 + tid) * Hv + h];
         bt = p.beta[(t0 + tid) * Hv + h];
     }
-    __syncthreads();  // the barrier is initialised
+    tc_fence_before();
+    __syncthreads();  // the barriers are initialised, the TMEM base is written
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
         mbar_arrive_expect_tx(bar, 16384);
         tma_load_3d(sm + wK, &tm_k, bar, 0, hk, (int)t0);
@@ -160,104 +164,70 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         vbG[tid] = bt * expf(gr);
     }
 
-    // ---- K K^T, lower block triangle: 20 tiles of 16 rows (m-tile) x 8 columns (n-tile), five
-    // per warp.  m-tiles 0 and 3 (2 + 8 tiles) are shared by warps 0 and 1, m-tiles 1 and 2
-    // (4 + 6 tiles) by warps 2 and 3; a warp's tiles are one run of n-tiles in m-tile mA and
-    // possibly a second run in m-tile mB.
-    const int g8 = lane >> 2, t4 = lane & 3;
-    int mA, jA, nA, mB, jB;
-    switch (warp) {
-        case 0: mA = 0; jA = 0; nA = 2; mB = 3; jB = 0; break;   // (0: 0-1), (3: 0-2)
-        case 1: mA = 3; jA = 3; nA = 5; mB = 3; jB = 8; break;   // (3: 3-7)
-        case 2: mA = 1; jA = 0; nA = 4; mB = 2; jB = 0; break;   // (1: 0-3), (2: 0)
-        default: mA = 2; jA = 1; nA = 5; mB = 2; jB = 6; break;  // (2: 1-5)
-    }
-    const bool twoA = nA < 5;  // warp-uniform: a second m-tile run exists
-    float acc[5][4];
+    // ---- K K^T on the tensor core: D = A K^T with A the K tile read as 128 rows (D rows 0-63 are
+    // the Gram block; rows 64-127 come from the bytes after the tile and are not read), N = 64,
+    // bf16 in, fp32 out in TMEM lanes 0-63 (one K row per lane)
+    bool ok = __syncthreads_and(mbar_wait(bar, 0));  // vectors written, the K tile has landed
+    if (ok && tid == 0) {
+        const uint64_t dK = desc_sw128(smem_u32(sm + wK), 16, 1024);
+        tc_fence_after();
 #pragma unroll
-    for (int i = 0; i < 5; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    __syncthreads();  // vectors
-    if (!__syncthreads_and(mbar_wait(bar, 0))) {  // the K tile has landed (bounded wait)
+        for (int j = 0; j < 8; ++j)  // K steps of 16: four per 64-wide k half (8 KB apart)
+            mma_bf16_ss(tmem, dK + (((j >> 2) * 8192 + (j & 3) * 32) >> 4),
+                        dK + (((j >> 2) * 8192 + (j & 3) * 32) >> 4), idesc_bf16(128, 64, 0, 0), j > 0);
+        mma_commit(bar_mma);
+    }
+    ok = ok && __syncthreads_and(mbar_wait(bar_mma, 0));
+    if (!ok) {
         if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
-        return;
-    }
-    {
-        const uint32_t sK = smem_u32(sm + wK);
+    } else {
+        tc_fence_after();
+        // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> X, row r by thread r (warps 0 and 1 read
+        // TMEM lanes 0-63).  X overwrites the K tile, which the MMA has read.  Entries below the
+        // diagonal 16 x 16 blocks are merge operands only: stored rounded to tf32.  The diagonal of
+        // K K^T gives |k_r|^2 for the chunk summary.
+        float* X = (float*)(sm + wK);
+        if (warp < 2) {
+            const int r = tid;
+            const float br = vbeta[r], ar = va[r];
+            float* xr = X + r * kXs;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {  // 16 columns s = 16 q .. 16 q + 15 at a time
+                float v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + 16 * q, v);
+                if ((r >> 4) == q) {  // the diagonal entry, by an unrolled select (no indexed registers)
+                    float dg = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < 8; kk += 2) {  // pairs of 16-wide k steps
-            const uint32_t half = sK + (kk >> 2) * 8192;
-            const int ch = 2 * (kk & 3);
-            uint32_t aA0[4], aA1[4], aB0[4], aB1[4];
-            ldsm_x4(aA0, half + sw128_off(16 * mA + (lane & 15), ch + (lane >> 4)));
-            ldsm_x4(aA1, half + sw128_off(16 * mA + (lane & 15), ch + 2 + (lane >> 4)));
-            if (twoA) {
-                ldsm_x4(aB0, half + sw128_off(16 * mB + (lane & 15), ch + (lane >> 4)));
-                ldsm_x4(aB1, half + sw128_off(16 * mB + (lane & 15), ch + 2 + (lane >> 4)));
-            }
+                    for (int e = 0; e < 16; ++e) dg = (e == (r & 15)) ? v[e] : dg;
+                    vnrm[r] = dg;
+                }
+                // E_rs = a_r b_s, or exp2(a_r - b_s) when the chunk's decay range is too wide
+                // (block-uniform branch: one loop per form); E is used only under the mask:
+                // above the diagonal it may overflow.  Entries below the diagonal 16 x 16 blocks
+                // (q < r / 16) are merge operands only: stored rounded to tf32.
+                const bool below = q < (r >> 4);
+                if (fac) {
 #pragma unroll
-            for (int i = 0; i < 5; ++i) {
-                const bool inA = i < nA;  // warp-uniform
-                const int j = inA ? jA + i : jB + (i - nA);
-                uint32_t b[4];
-                ldsm_x4(b, half + sw128_off(8 * j + (lane & 7), ch + (lane >> 3)));
-                if (inA) {
-                    mma_16816(acc[i], aA0, b[0], b[1]);
-                    mma_16816(acc[i], aA1, b[2], b[3]);
+                    for (int e = 0; e < 16; ++e) v[e] *= ar * vb[16 * q + e];
                 } else {
-                    mma_16816(acc[i], aB0, b[0], b[1]);
-                    mma_16816(acc[i], aB1, b[2], b[3]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] *= exp2f(ar - vb[16 * q + e]);
+                }
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    float o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int s = 16 * q + 4 * e4 + e;
+                        const float x = (s < r && r < lc) ? br * v[4 * e4 + e] : 0.f;
+                        o[e] = below ? tf32r(x) : x;
+                    }
+                    *reinterpret_cast<float4*>(xr + 16 * q + 4 * e4) = make_float4(o[0], o[1], o[2], o[3]);
                 }
             }
         }
-    }
-    __syncthreads();  // every warp is done with the K tile: X overwrites it
-
-    // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> X (entries on and above the diagonal
-    // that a tile covers are written as zeros and later overwritten by T).  Blocks below the
-    // diagonal block are merge operands only: stored rounded to tf32.  The diagonal of K K^T
-    // gives |k_r|^2 for the chunk summary.
-    float* X = (float*)(sm + wK);
-    {
-        float arA[2], brA[2], arB[2], brB[2];
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            arA[hr] = va[16 * mA + g8 + 8 * hr];
-            brA[hr] = vbeta[16 * mA + g8 + 8 * hr];
-            arB[hr] = va[16 * mB + g8 + 8 * hr];
-            brB[hr] = vbeta[16 * mB + g8 + 8 * hr];
-        }
-#pragma unroll
-        for (int i = 0; i < 5; ++i) {
-            const bool inA = i < nA;
-            const int m = inA ? mA : mB, j = inA ? jA + i : jB + (i - nA);
-            const int s = 8 * j + 2 * t4;
-            const bool below = (j >> 1) < m;  // warp-uniform
-            const float2 b2 = *reinterpret_cast<const float2*>(vb + s);
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int r = 16 * m + g8 + 8 * hr;
-                const float ar = inA ? arA[hr] : arB[hr], br = inA ? brA[hr] : brB[hr];
-                float e0, e1;
-                if (fac) {  // block-uniform
-                    e0 = ar * b2.x;
-                    e1 = ar * b2.y;
-                } else {
-                    e0 = exp2f(ar - b2.x);
-                    e1 = exp2f(ar - b2.y);
-                }
-                float2 w;
-                w.x = (s < r && r < lc) ? br * acc[i][2 * hr] * e0 : 0.f;
-                w.y = (s + 1 < r && r < lc) ? br * acc[i][2 * hr + 1] * e1 : 0.f;
-                if (below) {
-                    w.x = tf32r(w.x);
-                    w.y = tf32r(w.y);
-                }
-                *reinterpret_cast<float2*>(X + r * kXs + s) = w;
-                if (s == r) vnrm[r] = acc[i][2 * hr];
-                if (s + 1 == r) vnrm[r] = acc[i][2 * hr + 1];
-            }
-        }
-    }
+        tc_fence_before();
+        __syncthreads();
     // Chunk summary for the forward's gate-driven split: the summed log decay of the chunk and
     // whether some token breaks 0 <= beta |k|^2 <= 2 (the condition under which each token's
     // state map has norm <= exp(g)).
@@ -322,6 +292,13 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
             *reinterpret_cast<uint4*>(img + kTImgBytes + off) = pack8(bw);
             *reinterpret_cast<uint4*>(img + 2 * kTImgBytes + off) = pack8(bu);
         }
+    }
+    }  // ok
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kWyTmemCols);
     }
 }
 
