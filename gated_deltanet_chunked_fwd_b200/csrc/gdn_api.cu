@@ -91,7 +91,7 @@ gdn_status plan_fwd(const gdn_fwd_args* a, FwdPlan* plan) {
     const int64_t nc = p.num_chunks;
     size_t off = 0;
     if (plan->use_tc) {
-        plan->total = align_up(tc_fwd_workspace(p), kAlign);
+        plan->total = align_up(tc_fwd_workspace(p, plan->cu_host, plan->split_mode), kAlign);
         plan->launches = tc_fwd_launches(p);
         return GDN_OK;
     }
@@ -156,7 +156,7 @@ gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan) {
     plan->split_mode = (a->flags & GDN_FLAG_SPLIT_OFF) ? 1 : (a->flags & GDN_FLAG_SPLIT_FORCE) ? 2 : 0;
     if (plan->use_tc) {
         size_t o1, o2, o3, o4;
-        plan->total = align_up(tc_bwd_workspace(p, &o1, &o2, &o3, &o4), kAlign);
+        plan->total = align_up(tc_bwd_workspace(p, plan->cu_host, plan->split_mode, &o1, &o2, &o3, &o4), kAlign);
         plan->launches = tc_bwd_launches(p);
         return GDN_OK;
     }

@@ -83,7 +83,7 @@ struct FwdPlan {
 gdn_status plan_fwd(const gdn_fwd_args* a, FwdPlan* plan);
 gdn_status launch_fwd_simt(const FwdPlan& plan, char* ws, cudaStream_t s);
 gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s);
-size_t tc_fwd_workspace(const Problem& p);
+size_t tc_fwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode);
 size_t wy_tc_workspace(const Problem& p);
 size_t wy_tc_summary_offset(const Problem& p);
 // WY + fused kernel in replay mode: bf16 H^T entry-state image (32 KB) of every chunk, by
@@ -106,8 +106,8 @@ gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan);
 gdn_status launch_bwd_simt(const BwdPlan& plan, char* ws, cudaStream_t s);
 gdn_status launch_bwd_reduce(const BwdProblem& b, const float* dqw, const float* dkw, cudaStream_t s);
 bool tc_bwd_supported(const Problem& p);
-size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, size_t* off_dqw,
-                        size_t* off_dkw);
+size_t tc_bwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode, size_t* off_himg,
+                        size_t* off_timg, size_t* off_dqw, size_t* off_dkw);
 int tc_bwd_launches(const Problem& p);
 gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s);
 

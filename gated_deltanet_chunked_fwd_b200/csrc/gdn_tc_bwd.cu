@@ -799,11 +799,11 @@ bool tc_bwd_supported(const Problem& p) { return p.dtype == GDN_BF16 && p.dk == 
 
 // workspace: the WY outputs (T / Bw / Bu images, gate summaries), the replayed H^T images, then (with
 // grouped heads) fp32 dq and dk per value head, summed over each group by the reduction
-size_t tc_bwd_workspace(const Problem& p, size_t* off_himg, size_t* off_timg, size_t* off_dqw,
-                        size_t* off_dkw) {
+size_t tc_bwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode, size_t* off_himg,
+                        size_t* off_timg, size_t* off_dqw, size_t* off_dkw) {
     size_t off = 0;
-    *off_timg = off;
-    off = align_up(off + wy_tc_workspace(p), 256);
+    *off_timg = off;  // the forward's workspace (WY images and summaries, the scan) for the replay
+    off = align_up(off + tc_fwd_workspace(p, cu_host, split_mode), 256);
     *off_himg = off;
     off = align_up(off + (p.num_chunks > 0 ? (size_t)img_slots(p) * p.Hv * kHImg : 0), 256);
     const size_t per = p.group > 1 ? sizeof(float) * (size_t)p.T_total * p.Hv * p.dk : 0;
@@ -822,7 +822,7 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     TcBwdArgs a;
     a.b = bp;
     size_t oh, ot, oq, ok_;
-    tc_bwd_workspace(p, &oh, &ot, &oq, &ok_);
+    tc_bwd_workspace(p, plan.cu_host, plan.split_mode, &oh, &ot, &oq, &ok_);
     a.himg = (const uint8_t*)(ws + oh);
     a.timg = (const uint8_t*)(ws + ot);
     a.summ = (const float2*)(ws + ot + wy_tc_summary_offset(p));

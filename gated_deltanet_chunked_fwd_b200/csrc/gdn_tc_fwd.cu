@@ -29,12 +29,21 @@
 // is <= log(eps).  While 0 <= beta |k|^2 <= 2 each token's state map has norm
 // <= exp(g_t), so the truncated past contributes at most eps * |H| to the
 // segment's entry state.  If the decay never reaches eps, or some warm-up
-// token breaks the norm condition, the segment starts exactly from the
-// sequence start (from S0) instead.
+// token breaks the norm condition, the segment's entry state comes from an exact
+// affine scan instead when that is cheaper than replaying the sequence from S0
+// (long segments late in a sequence of at least scan_min_segs segments).  Every chunk maps the
+// state affinely, H' = M_c H + B_c, so a segment's chunks compose to
+// H_exit = M_j H_entry + B_j.  The segment folds (M_j, B_j) by walking its own
+// chunks twice -- from H = 0 with the real values (B_j), then from H = I with
+// v = 0 (M_j) -- and publishes them; it then looks back for the nearest earlier
+// segment whose exit state is published (segments publish their exit when they
+// end) and applies the folds in between, X <- M X + B, in fp32, which gives its
+// exact entry state; a third walk from that state writes the outputs.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cmath>
 #include <vector>
 
@@ -99,7 +108,129 @@ struct TcArgs {
     const float2* summ;   // per (image slot, value head): summed log decay, norm-condition flag
     uint8_t* himg;        // replay mode (backward): bf16 H^T entry-state image per own chunk, by
                           // (image slot, value head); no outputs.  nullptr: the forward
+    // affine scan for segments that cannot warm up: per CTA (= blockIdx.x) a flag and three fp32
+    // [dk][dv] records (exit state, M, B); nullptr (no sequence has scan_min_segs segments): such
+    // a segment replays its sequence from S0 instead
+    int32_t* scan_flags;
+    float* scan_rec;
+    int scan_min_segs;
 };
+
+// Warm-up start of the segment that begins at chunk c0 of sequence n (value head h): the largest
+// w < c0 whose chunks w .. c0-1 sum to a log decay <= log_eps (the per-chunk sums of the WY step's
+// summaries), searched 32 chunks at a time by a whole warp (every lane returns the same); -1 when
+// the sum never gets there, or when one of those chunks breaks 0 <= beta |k|^2 <= 2.
+__device__ __forceinline__ int warmup_start(const float2* summ, int64_t bos, int n, int h, int Hv, int c0,
+                                            float log_eps, int lane) {
+    float cum = 0.f;
+    bool bad = false;
+    for (int top = c0 - 1; top >= 0; top -= 32) {
+        const int w = top - lane;  // lane l looks at chunk top - l
+        const float2 cs = w >= 0 ? summ[img_slot(bos, n, w) * Hv + h] : make_float2(0.f, 0.f);
+        float x = cs.x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, w >= 0 && cum + x <= log_eps);
+        if (hit) {
+            const int first = __ffs(hit) - 1;
+            bad |= __any_sync(0xffffffffu, lane <= first && cs.y != 0.f);
+            return bad ? -1 : top - first;
+        }
+        bad |= __any_sync(0xffffffffu, w >= 0 && cs.y != 0.f);
+        cum += __shfl_sync(0xffffffffu, x, 31);
+    }
+    return -1;
+}
+
+// the scan's flags: 0 nothing yet, 1 the segment's fold (M, B) is published, 2 its exit state is
+__device__ __forceinline__ void flag_release(int32_t* f, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ int flag_acquire(const int32_t* f) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+// Start state of the next walk of an affine scan, written to TMEM by the thread of state column m
+// (lane m of the warp's quarter at tl): H = I when flags == nullptr; else the exit state of
+// segment `base` (records at recs + base * stride: [exit, M, B], each [128][128] fp32, segments
+// hv apart in the flags) carried through the folds of segments base + 1 .. seg - 1,
+// X <- M X + B, in fp32; zero when base < 0 (a look-back that timed out).  The column of X lives
+// in the fp32 state columns of TMEM while the folds run (32 x 32 blocks of M times 32 of its
+// values at a time); `tmp` (this CTA's exit record) holds a fold's result column.  Ends with the
+// bf16 copy in the A-operand columns and the fp32 state pre-scaled by Gn (the first chunk's Gam_n).
+__device__ __forceinline__ void scan_start_state(uint32_t tl, int m, const int32_t* flags, int hv,
+                                                 const float* recs, int64_t stride, int base, int seg,
+                                                 float* tmp, float Gn) {
+    constexpr int kD = 128;
+    float v[32];
+    if (!flags || base < 0) {
+#pragma unroll 1
+        for (int a = 0; a < 4; ++a) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = (flags == nullptr && 32 * a + e == m) ? 1.f : 0.f;
+            tmem_st32(tl + kColH + 32 * a, v);
+        }
+    } else {
+        (void)flag_acquire(flags + base * hv);  // this thread's own acquire of the records it reads
+        const float* ex = recs + base * stride + m;
+#pragma unroll 1
+        for (int a = 0; a < 4; ++a) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = ex[(int64_t)(32 * a + e) * kD];
+            tmem_st32(tl + kColH + 32 * a, v);
+        }
+        for (int t = base + 1; t < seg; ++t) {
+            (void)flag_acquire(flags + t * hv);
+            const float* Mt = recs + t * stride + kD * kD;
+            const float* Bt = Mt + kD * kD;
+#pragma unroll 1
+            for (int ib = 0; ib < 4; ++ib) {  // rows 32 ib .. 32 ib + 31 of the new column
+                float acc[32];
+#pragma unroll
+                for (int ii = 0; ii < 32; ++ii) acc[ii] = Bt[(int64_t)(32 * ib + ii) * kD + m];
+#pragma unroll 1
+                for (int lb = 0; lb < 4; ++lb) {  // times X rows 32 lb .. 32 lb + 31
+                    tmem_ld32(tl + kColH + 32 * lb, v);
+#pragma unroll 4
+                    for (int ii = 0; ii < 32; ++ii) {
+                        const float4* mr = reinterpret_cast<const float4*>(Mt + (int64_t)(32 * ib + ii) * kD + 32 * lb);
+                        float sacc = 0.f;
+#pragma unroll
+                        for (int l4 = 0; l4 < 8; ++l4) {
+                            const float4 mv = mr[l4];
+                            sacc += mv.x * v[4 * l4] + mv.y * v[4 * l4 + 1] + mv.z * v[4 * l4 + 2] + mv.w * v[4 * l4 + 3];
+                        }
+                        acc[ii] += sacc;
+                    }
+                }
+#pragma unroll
+                for (int ii = 0; ii < 32; ++ii) tmp[(int64_t)(32 * ib + ii) * kD + m] = acc[ii];
+            }
+#pragma unroll 1
+            for (int a = 0; a < 4; ++a) {  // the new column replaces X
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = tmp[(int64_t)(32 * a + e) * kD + m];
+                tmem_st32(tl + kColH + 32 * a, v);
+            }
+        }
+    }
+    uint32_t w[16];
+#pragma unroll 1
+    for (int a = 0; a < 4; ++a) {
+        tmem_ld32(tl + kColH + 32 * a, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        tmem_st16u(tl + kColHb + 16 * a, w);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= Gn;
+        tmem_st32(tl + kColH + 32 * a, v);
+    }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -220,24 +351,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- warm-up start (gate-driven); exact start from S0 when seg == 0.  The WY step left,
     // per chunk, its summed log decay and whether some token breaks 0 <= beta |k|^2 <= 2.
+    // a segment without a warm-up takes the scan when its three walks over the own chunks and
+    // one fold product per earlier segment (about three chunk steps each) cost less than
+    // replaying the sequence's first chunks; else the replay from S0
+    auto scan_pays = [&](int sj, int c0j, int c1j) {
+        return args.scan_rec != nullptr && c0j > 2 * (c1j - c0j) + 3 * (sj - 1);
+    };
     int cstart = 0;
+    bool scan = false;  // entry state by the affine scan: three walks over the own chunks
     if (!known_exact) {
-        float cum = 0.f;
-        int w = c0;
-        bool bad = false;
-        while (w > 0 && cum > args.log_eps) {
-            --w;
-            const float2 cs = args.summ[img_slot(bos, n, w) * Hv + h];
-            cum += cs.x;
-            bad |= cs.y != 0.f;
+        const int w = warmup_start(args.summ, bos, n, h, Hv, c0, args.log_eps, lane);
+        if (w < 0) {
+            scan = scan_pays(seg, c0, c1);
+            cstart = scan ? c0 : 0;
+        } else {
+            cstart = w;
         }
-        cstart = (cum > args.log_eps || bad) ? 0 : w;
     }
     const bool exact = (cstart == 0);
-    const int nk = c1 - cstart;  // chunks this CTA walks (warm-up + own)
-    if (!known_exact && tid >= kThreadsP) load_state(exact);
-    auto issue_tma = [&](int k) {
-        const int c = cstart + k;
+    const int nkp = c1 - cstart;          // chunks per walk (warm-up + own)
+    const int npass = scan ? 3 : 1;       // walks: [B fold, M fold,] final
+    const int nk = npass * nkp;           // steps of the pipeline
+    // step k of the pipeline: chunk cstart + k % nkp of walk k / nkp; walk 1 of a scan has v = 0
+    auto chunk_of = [&](int k) {  // k < 3 nkp: two compares instead of a division
+        int kk = k;
+        if (kk >= nkp) kk -= nkp;
+        if (kk >= nkp) kk -= nkp;
+        return cstart + kk;
+    };
+    auto final_walk = [&](int k) { return k >= (npass - 1) * nkp; };
+    auto v_on = [&](int k) { return !(scan && k >= nkp && k < 2 * nkp); };  // walk 1: v = 0
+    // records of the scan, shared with the later segments of the sequence
+    float* rec = args.scan_rec ? args.scan_rec + (int64_t)blockIdx.x * 3 * dk * dv : nullptr;
+    if (!known_exact && tid >= kThreadsP) load_state(exact && !scan);
+    auto issue_tma_at = [&](int k, int c) {  // step k, chunk c
         const int stage = k & 1;
         const int t0 = (int)(bos + (int64_t)c * kChunk);
         uint8_t* qk = sm + kStageQK + stage * 32768;
@@ -252,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   args.timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kWyImgBytes + kTImgBytes,
                   2 * kTImgBytes, &bar_tma[stage]);  // Bw and Bu
     };
+    auto issue_tma = [&](int k) { issue_tma_at(k, chunk_of(k)); };
 
     if (tid == 0) {
         if (nk > 0) issue_tma(0);
@@ -274,12 +422,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hf = t >> 7;                       // which 32-column half of a TMEM row
         const int row = ((warp & 3) << 5) | lane;    // TMEM lane (= MMA row) this thread reads
         uint32_t ph = 0;  // parity of bar_mma_p
+        // The loops come in two compiled forms: one walk over the chunks (every segment that does
+        // not take the scan), or the three walks of the scan.
+        auto run_p = [&](auto walks) {
+        constexpr int NP = decltype(walks)::value;
+        auto chunk_ofn = [&](int k) { return NP == 1 ? cstart + k : chunk_of(k); };
+        auto final_walkn = [&](int k) { return NP == 1 || final_walk(k); };
+        auto v_onn = [&](int k) { return NP == 1 || v_on(k); };
         // Gates run one chunk ahead in warp 2 (lane l: rows 2l, 2l+1), so chunk k+1's vectors
         // are in shared memory before chunk k is handed to group S.  g / beta of the chunk after
         // that are prefetched into registers.
         float gx0 = 0.f, gx1 = 0.f;
         auto load_gates = [&](int kk) {
-            const int cc = cstart + kk;
+            const int cc = chunk_ofn(kk);
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lcc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
             const int r0 = 2 * lane;
@@ -325,9 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lanes m, m^1 swap one value so that each thread writes bf16 pairs (columns m & ~1,
         // m | 1) of one token.  A chunk cut short by its sequence's end is stored element by
         // element, masked to its tokens.
-        auto emits = [&](int kk) { return cstart + kk >= c0 && !args.himg; };
+        auto emits = [&](int kk) { return final_walkn(kk) && chunk_ofn(kk) >= c0 && !args.himg; };
         auto epilogue = [&](int kk) {
-            const int cc = cstart + kk;
+            const int cc = chunk_ofn(kk);
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
             const int m = row;
@@ -367,9 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 
         for (int k = 0; k < nk; ++k) {
-            const int c = cstart + k;
+            const int c = chunk_ofn(k);
             const int stage = k & 1;
-            const bool emit = c >= c0 && !args.himg;
+            const bool emit = emits(k);
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t sV = sbase + kStageV + stage * 16384;
@@ -465,14 +620,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             wg_sync(1, kThreadsP);
 
-            if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1);  MMA_U: Ut^T = V^T Bu^T (R2[stage])
+            if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1);  MMA_U: Ut^T = V^T Bu^T (R2[stage]), unless the
+                           // walk has v = 0 (the M fold of a scan: U = -W H)
+                const bool with_v = v_onn(k);
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
                                 desc_sw128(sBwu + j * 32, 16, 1024), id_mn_n64, j > 0);
-                    mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
-                                desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
+                    if (with_v)
+                        mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
+                                    desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
                 }
                 mma_commit(bar_mma_p);
             }
@@ -502,6 +660,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && emits(kk)) epilogue(kk);
         }
         if (t == 0) bulk_wait0();  // every output tile has been written
+        };
+        if (npass == 1)
+            run_p(std::integral_constant<int, 1>{});
+        else
+            run_p(std::integral_constant<int, 3>{});
     } else {
         // ======================= group S: the state chain =======================
         // Per chunk k: MMA_HW; U^T -> bf16 in TMEM; MMA_O (into the O^T buffer of the chunk's
@@ -511,10 +674,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         // k+1 accumulates onto it).
         const int m = tid - kThreadsP;
         uint32_t ph = 0;  // parity of bar_mma_s
-        for (int k = 0; k < nk && ok; ++k) {
-            const int c = cstart + k;
+        // This segment's exit state is published when a later segment of the sequence takes the
+        // scan: the same decision, made here from the same summaries, one warp per later segment
+        // (while the first chunk is prepared by group P).
+        bool later_scans = false;
+        if (args.scan_rec != nullptr && args.auto_warm) {
+            for (int j = seg + 1 + (warp & 3); j < segs_n; j += kThreadsS / 32) {
+                const int c0j = min(nck, args.lead + j * args.L), c1j = min(nck, args.lead + (j + 1) * args.L);
+                if (scan_pays(j, c0j, c1j) && warmup_start(args.summ, bos, n, h, Hv, c0j, args.log_eps, lane) < 0)
+                    later_scans = true;
+            }
+        }
+        const bool publish = wg_or(2, kThreadsS, later_scans);
+        auto run_s = [&](auto walks) {
+        constexpr int NP = decltype(walks)::value;
+        auto issue_tman = [&](int k) {
+            if (NP == 1) issue_tma_at(k, cstart + k);
+            else issue_tma(k);
+        };
+        for (int walk = 0; walk < NP && ok; ++walk) {
+        const bool fin = walk == NP - 1;       // the walk that writes outputs / entry images
+        const bool with_v = NP == 1 || walk != 1; // walk 1 of a scan (the M fold) has v = 0
+        for (int kk = 0; kk < nkp && ok; ++kk) {
+            const int k = walk * nkp + kk;  // pipeline step
+            const int c = cstart + kk;
             const int stage = k & 1;
-            const bool emit = c >= c0 && !args.himg;
+            const bool emit = fin && c >= c0 && !args.himg;
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t colR2 = kColR2 + 64 * stage;
             const uint32_t colO = kColO + 64 * stage;
@@ -534,15 +719,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st64(tl + kColH + 64 * a, v);
                 }
             }
-            if (m == 0) {  // MMA_HW: U^T = Ut^T + H^T (-W^T)
+            if (m == 0) {  // MMA_HW: U^T = Ut^T + H^T (-W^T)  (U^T = -H^T W^T when the walk has v = 0)
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     mma_bf16_ts(tmem + colR2, tmem + kColHb + 8 * j,
-                                desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_bmn_n64, 1);
+                                desc_sw128(sbase + kWt + j * 2048, 8192, 1024), id_bmn_n64, with_v || j > 0);
                 mma_commit(bar_mma_s);
             }
-            if (args.himg && c >= c0) {
+            if (args.himg && c >= c0 && fin) {
                 // replay mode: the chunk's entry state, as the bf16 H^T image [dk half][128 dv
                 // rows][128 B] (128-byte swizzled) that the backward loads; the bf16 copy in TMEM
                 // holds it (dk pairs per column)
@@ -607,11 +792,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ph ^= 1;
             if (!ok) break;
             tc_fence_after();
-            if (m == 0 && k + 2 < nk) issue_tma(k + 2);  // stage `stage` is no longer read
+            if (m == 0 && k + 2 < nk) issue_tman(k + 2);  // stage `stage` is no longer read
 
             // bf16 copy of the new state (A operand of the next chunk's MMAs); pre-scale by its Gam_n
-            // (chunk k+1's vectors were written before chunk k was handed over)
-            const bool more = k + 1 < nk;
+            // (chunk k+1's vectors were written before chunk k was handed over).  The last chunk
+            // of a fold walk leaves H as it is: the next walk starts from another state (below).
+            const bool more = kk + 1 < nkp;
             {
                 const float Gn = more ? ((const float*)(sm + kVec))[((k + 1) & 3) * kVecStride + 128 + 63] : 1.f;
                 float v[64];
@@ -632,6 +818,81 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             wg_sync(2, kThreadsS);
             if (m == 0) mbar_arrive(&bar_s_done[stage]);
+        }
+        if (NP > 1 && ok && walk + 1 < NP) {
+            // A fold walk ended: H is B_j (walk 0, from H = 0) or M_j (walk 1, from H = I with
+            // v = 0); the next walk starts from I or from the scanned entry state.  Its first
+            // chunk's vectors were written before the last chunk was handed over.
+            tc_fence_after();
+            const bool second = walk == 1;  // records of this CTA: [exit, M, B], each [dk][dv]
+            {
+                float* dst = rec + (int64_t)(second ? 1 : 2) * dk * dv + m;
+                float v[64];
+#pragma unroll 1
+                for (int a = 0; a < 2; ++a) {
+                    tmem_ld64(tl + kColH + 64 * a, v);
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) dst[(int64_t)(64 * a + e) * dv] = v[e];
+                }
+            }
+            const float Gn = ((const float*)(sm + kVec))[(((walk + 1) * nkp) & 3) * kVecStride + 128 + 63];
+            if (!second) {
+                scan_start_state(tl, m, nullptr, 0, nullptr, 0, 0, 0, nullptr, Gn);  // H = I
+            } else {
+                // publish the fold, then look back: the nearest earlier segment whose exit state
+                // is published (segment 0 always publishes one), and the folds in between
+                __threadfence();
+                wg_sync(2, kThreadsS);
+                int32_t* flags = args.scan_flags + (blockIdx.x - (unsigned)seg * Hv);  // segment 0
+                if (m == 0) flag_release(flags + seg * Hv, 1);
+                int* lb = (int*)(sm + kRed);
+                if (m == 0) {
+                    int i = seg - 1;
+                    bool okl = true;
+                    const uint64_t t0 = globaltimer();
+                    while (true) {
+                        const int f = flag_acquire(flags + i * Hv);
+                        if (f == 2) break;
+                        if (f == 1) {
+                            --i;
+                            continue;
+                        }
+                        if (globaltimer() - t0 > kWaitTimeoutNs) {
+                            okl = false;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                    lb[0] = i;
+                    lb[1] = okl ? 1 : 0;
+                }
+                wg_sync(2, kThreadsS);
+                ok = lb[1] != 0;
+                const float* recs = args.scan_rec + (int64_t)(blockIdx.x - (unsigned)seg * Hv) * 3 * dk * dv;
+                scan_start_state(tl, m, flags, Hv, recs, (int64_t)Hv * 3 * dk * dv, ok ? lb[0] : -1, seg, rec, Gn);
+            }
+            tc_fence_before();
+            wg_sync(2, kThreadsS);
+        }
+        }  // walks
+        };
+        if (npass == 1)
+            run_s(std::integral_constant<int, 1>{});
+        else
+            run_s(std::integral_constant<int, 3>{});
+        if (ok && publish) {
+            // the exit state for later segments that look back (the scan)
+            float* ex = rec + m;
+            float v[64];
+#pragma unroll 1
+            for (int a = 0; a < 2; ++a) {
+                tmem_ld64(tl + kColH + 64 * a, v);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) ex[(int64_t)(64 * a + e) * dv] = v[e];
+            }
+            __threadfence();
+            wg_sync(2, kThreadsS);
+            if (m == 0) flag_release(args.scan_flags + blockIdx.x, 2);
         }
         if (ok && p.ST && seg == segs_n - 1) {
             // final state S_T = H (stored [dk][dv]): thread m writes column m
@@ -662,8 +923,43 @@ bool tc_fwd_supported(const Problem& p) {
     return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128;
 }
 
-// workspace: the T / Bw / Bu images and gate summaries of the WY step
-size_t tc_fwd_workspace(const Problem& p) { return wy_tc_workspace(p); }
+namespace {
+
+constexpr int kScanMinSegs = 4;  // the affine scan pays off from four segments on (three walks)
+
+// The split of the chains over CTAs: the first segment of a sequence starts exactly, so it takes
+// one chunk more than the others (a warm-up is at least one chunk).
+struct ChainSplit {
+    std::vector<int> nck;
+    SplitChoice sc;
+    bool scan;  // some sequence has enough segments for the affine scan
+};
+
+ChainSplit chain_split(const Problem& p, const int32_t* cu_host, int split_mode) {
+    ChainSplit cs;
+    cs.nck = chunk_counts(p, cu_host);
+    cs.sc = choose_split(cs.nck, p.Hv, split_mode, sm_count(), 1.5, 1);
+    cs.scan = false;
+    for (int c : cs.nck) cs.scan |= segments_of(c, cs.sc.L, cs.sc.lead) >= kScanMinSegs;
+    cs.scan &= split_mode != 1;
+    return cs;
+}
+
+// bytes of the scan's flags (one int32 per CTA, 256-aligned) and records (three fp32 states
+// [dk][dv] per CTA: exit state, M, B)
+size_t scan_flag_bytes(int64_t ctas) { return align_up((size_t)ctas * 4, 256); }
+size_t scan_bytes(const ChainSplit& cs, const Problem& p) {
+    return cs.scan ? scan_flag_bytes(cs.sc.ctas) + (size_t)cs.sc.ctas * 3 * p.dk * p.dv * sizeof(float) : 0;
+}
+
+}  // namespace
+
+// workspace: the T / Bw / Bu images and gate summaries of the WY step, then (when some sequence
+// is split into enough segments) the affine scan's flags and records
+size_t tc_fwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode) {
+    const size_t wy = align_up(wy_tc_workspace(p), 256);
+    return p.num_chunks > 0 ? wy + scan_bytes(chain_split(p, cu_host, split_mode), p) : 0;
+}
 int tc_fwd_launches(const Problem& p) { return (p.num_chunks > 0 ? 1 : 0) + 1; }
 
 // The WY kernel, then the fused kernel (forward, or replay of the states when himg != nullptr)
@@ -675,10 +971,17 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
     a.timg = (const uint8_t*)ws;
     a.summ = (const float2*)(ws + wy_tc_summary_offset(p));
     a.himg = himg;
-    const std::vector<int> nck = chunk_counts(p, cu_host);
-    // the first segment of a sequence starts exactly, so it takes one chunk more than the others
-    // (a warm-up is at least one chunk)
-    const SplitChoice sc = choose_split(nck, p.Hv, split_mode, sm_count(), 1.5, 1);
+    const ChainSplit cs = chain_split(p, cu_host, split_mode);
+    const std::vector<int>& nck = cs.nck;
+    const SplitChoice& sc = cs.sc;
+    a.scan_min_segs = kScanMinSegs;
+    a.scan_flags = nullptr;
+    a.scan_rec = nullptr;
+    if (cs.scan && p.num_chunks > 0) {
+        char* base = ws + align_up(wy_tc_workspace(p), 256);
+        a.scan_flags = (int32_t*)base;
+        a.scan_rec = (float*)(base + scan_flag_bytes(sc.ctas));
+    }
     a.L = sc.L;
     a.lead = sc.lead;
     a.fixed_segs = p.cu ? 0 : (nck.empty() ? 1 : segments_of(nck[0], sc.L, sc.lead));
@@ -694,7 +997,7 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
                              (int)kSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
-    const gdn_status st = launch_wy_tc(p, mk, (uint8_t*)ws, s);
+    const gdn_status st = launch_wy_tc(p, mk, (uint8_t*)ws, a.scan_flags, a.scan_flags ? (int)sc.ctas : 0, s);
     if (st) return st;
     // Programmatic dependent launch: the fused kernel may start while the WY kernel drains; it
     // sets up and loads S0 for exact segments, then waits (griddepcontrol.wait) for the WY

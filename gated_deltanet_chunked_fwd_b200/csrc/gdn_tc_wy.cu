@@ -86,7 +86,7 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
 
 __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     gdn_wy_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const Problem p, uint8_t* __restrict__ timg,
-                     float2* __restrict__ summ) {
+                     float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -94,6 +94,9 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     const int h = blockIdx.y, hk = h / p.group, Hv = p.Hv;
     int n = 0, c = 0;
     int64_t bos = 0, len = 0;
+    // the state chain's scan flags start at zero (CTA (x, h) clears flag x Hv + h; the chain's CTAs
+    // are fewer than the image slots times the value heads)
+    if (tid == 0 && (int64_t)blockIdx.x * Hv + h < nflags) flags[(int64_t)blockIdx.x * Hv + h] = 0;
     const bool live = locate_slot(p, blockIdx.x, &n, &c, &bos, &len);  // CTA-uniform
     uint64_t* bar = (uint64_t*)(sm + wBar);
     uint64_t* bar_mma = bar + 1;
@@ -304,7 +307,8 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
 
 }  // namespace
 
-gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, cudaStream_t s) {
+gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, int32_t* flags, int nflags,
+                            cudaStream_t s) {
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
@@ -312,8 +316,9 @@ gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* 
                              (int)wSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     const dim3 grid((unsigned)slots, (unsigned)p.Hv);
-    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws,
-                                                          (float2*)(ws + wy_tc_summary_offset(p)));
+    if ((int64_t)nflags > slots * p.Hv) return GDN_ERR_DEVICE;  // every flag has a CTA to clear it
+    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws, (float2*)(ws + wy_tc_summary_offset(p)),
+                                                          flags, nflags);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -174,3 +174,12 @@ def test_aliased_state_gradient_is_rejected():
         ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=DEV)
         st = _abi.lib().gdn_chunk_bwd(ctypes.byref(a), ctypes.c_void_p(ws.data_ptr()), n.value, None)
         assert st == 1, alias  # GDN_ERR_INVALID_ARG
+
+
+def test_tensor_core_weak_decay_affine_scan_replay():
+    """The backward's state replay with weak decay on 8192 tokens x 16 heads: segments 3-8 of each
+    head take their entry state from the affine scan (see the forward test); all six gradients
+    against the oracle adjoint."""
+    inp = make_inputs(1, 8192, 16, 16, 128, 128, dtype="bf16", seed=29, s0_std=0.1, g_mu=-7.0,
+                      backward=True, device=DEV)
+    compare(run(inp), ref(inp), TOL[inp["q"].dtype], "weak decay scan")

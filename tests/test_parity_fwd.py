@@ -226,3 +226,18 @@ def test_aliased_initial_and_final_state_is_rejected():
             gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], initial_state=S,
                           final_state=S, flags=flags)
         assert e.value.status == 1  # GDN_ERR_INVALID_ARG
+
+
+def test_tensor_core_weak_decay_affine_scan():
+    """Weak decay (g = -softplus(N(-7, 1))) on 8192 tokens x 16 heads: the split gives nine segments
+    of 15 chunks per head and no warm-up reaches log(2^-30), so segments 3-8 take their entry state
+    from the affine scan (fold M, B over their own chunks, look back for the nearest published exit
+    state, apply the folds in between) and segments 1-2 replay from S0.  Every unit against the
+    oracle, and the split run against the unsplit one."""
+    inp = make_inputs(1, 8192, 16, 16, 128, 128, dtype="bf16", seed=28, s0_std=0.1, g_mu=-7.0,
+                      device=DEV)
+    assert float(inp["g"][0, :, :].double().sum(0).max()) > -30 * math.log(2)
+    o, ST = run(inp)
+    check_every_unit(inp, o, ST)
+    o1, ST1 = run(inp, GDN_FLAG_SPLIT_OFF)
+    assert rel_l2(o, o1) < 5e-3 and rel_l2(ST, ST1) < 5e-3
