@@ -398,6 +398,30 @@ def decode_bench(dev, stream, rank, measure, world, hbm, bf16, src, steps):
             "roofline": roofline(flops, byts, m * 1e-3, hbm, bf16, src)}
 
 
+def e2e_leg(inp, dev, stream, measure, steps, tokens, world):
+    """The headline call with pinned host inputs: the H2D copies of q, k, v, beta, g, the call
+    through the C ABI, and the D2H copies of o and S_T, all inside the timed region."""
+    names = [n for n in ("q", "k", "v", "beta", "g") if inp.get(n) is not None]
+    host = {n: inp[n].cpu().pin_memory() for n in names}
+    dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    ecall = FwdCall(dict(dbuf), dev, stream)
+    o_h = torch.empty(ecall.o.shape, dtype=ecall.o.dtype).pin_memory()
+    ST_h = torch.empty(ecall.ST.shape, dtype=ecall.ST.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * ST_h.element_size()
+
+    def e2e_step():
+        for n_, t in host.items():
+            dbuf[n_].copy_(t, non_blocking=True)
+        ecall()
+        o_h.copy_(ecall.o, non_blocking=True)
+        ST_h.copy_(ecall.ST, non_blocking=True)
+
+    ms_e2e = measure(e2e_step, max(2, min(steps, 5)))
+    return {"value": job_throughput(tokens, world, ms_e2e), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms": ms_e2e}
+
+
 def run_ours(args, world, rank, local):
     import gated_deltanet_chunked_fwd_b200 as gdn
     from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_SPLIT_OFF
@@ -423,8 +447,8 @@ def run_ours(args, world, rank, local):
         barrier(world)
         return max_over_ranks(sum(ms) / len(ms), world)
 
-    # ---- headline: one 65,536-token call
-    inp = make_workload(HEADLINE, seed=rank, device=dev)
+    # ---- headline: one 65,536-token call (fewer with --tokens, to profile a small case)
+    inp = make_workload(HEADLINE, seed=rank, device=dev, **({"T": args.tokens} if args.tokens else {}))
     call = FwdCall(inp, dev, stream)
     Hv, dk, dv = call.shape["Hv"], call.shape["dk"], call.shape["dv"]
     tokens = call.shape["T_total"]
@@ -449,26 +473,7 @@ def run_ours(args, world, rank, local):
               "triangular": tri * tokens * Hv / (ms_step * 1e-3) / 1e12, "peak_bf16": bf16}
 
     # ---- e2e: pinned host inputs, H2D + call + D2H of o and S_T, inside the timed region
-    names = [n for n in ("q", "k", "v", "beta", "g") if inp.get(n) is not None]
-    host = {n: inp[n].cpu().pin_memory() for n in names}
-    dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
-    e2e_inp = dict(dbuf)
-    ecall = FwdCall(e2e_inp, dev, stream)
-    o_h = torch.empty(ecall.o.shape, dtype=ecall.o.dtype).pin_memory()
-    ST_h = torch.empty(ecall.ST.shape, dtype=ecall.ST.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * ST_h.element_size()
-
-    def e2e_step():
-        for n_, t in host.items():
-            dbuf[n_].copy_(t, non_blocking=True)
-        ecall()
-        o_h.copy_(ecall.o, non_blocking=True)
-        ST_h.copy_(ecall.ST, non_blocking=True)
-
-    ms_e2e = measure(e2e_step, max(2, min(args.steps, 5)))
-    e2e_value = job_throughput(tokens, world, ms_e2e)
-    del dbuf, e2e_inp, ecall
+    e2e = None if args.no_e2e else e2e_leg(inp, dev, stream, measure, args.steps, tokens, world)
 
     # ---- the other forward workloads (extra keys)
     extra = {}
@@ -570,8 +575,9 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": HEADLINE_DESC,
-                       "global_batch": world, "seq_len": 65536, "heads": Hv, "head_dim": dk,
+            "config": {"workload": HEADLINE_DESC if not args.tokens else
+                       HEADLINE_DESC.replace("T=65536", f"T={tokens}"),
+                       "global_batch": world, "seq_len": tokens, "heads": Hv, "head_dim": dk,
                        "parallelism": f"replicas x{world} (no collective)",
                        "l2": "inputs (1.08 GB) larger than L2; L2 also flushed before every timed "
                              "step (2x L2 write, outside the events)",
@@ -579,8 +585,7 @@ def run_ours(args, world, rank, local):
                        else "cuda-core 4-kernel"},
             "tflops": tflops,
             "roofline": roof,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms": ms_e2e},
+            "e2e": e2e,
             "gpu_launches": call.launches * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu_base,
@@ -599,6 +604,9 @@ def main():
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="headline forward only")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-copy leg (profiling)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="headline shape with this many tokens (profiling a small case; 0 = 65,536)")
     ap.add_argument("--bwd-batch", type=int, default=4,
                     help="sequences in the backward workload (4 = the backward workload; fewer for a small profile)")
     args = ap.parse_args()

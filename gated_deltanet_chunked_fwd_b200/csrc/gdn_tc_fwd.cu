@@ -997,7 +997,8 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
                              (int)kSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
-    const gdn_status st = launch_wy_tc(p, mk, (uint8_t*)ws, a.scan_flags, a.scan_flags ? (int)sc.ctas : 0, s);
+    const gdn_status st =
+        launch_wy_tc(p, mk, (uint8_t*)ws, a.scan_flags, a.scan_flags ? (int)sc.ctas : 0, himg != nullptr, s);
     if (st) return st;
     // Programmatic dependent launch: the fused kernel may start while the WY kernel drains; it
     // sets up and loads S0 for exact segments, then waits (griddepcontrol.wait) for the WY

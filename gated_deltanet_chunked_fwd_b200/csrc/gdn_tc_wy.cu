@@ -86,7 +86,7 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
 
 __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     gdn_wy_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const Problem p, uint8_t* __restrict__ timg,
-                     float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags) {
+                     float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags, int with_t) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -253,8 +253,8 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
     merge_level<3>(X, ysw, warp, lane);
     __syncthreads();
 
-    // ---- bf16 images T, Bw, Bu: thread = rows nr4 .. nr4 + 3, columns s0 .. s0 + 7 (one 16-byte
-    // chunk of each row), from T[r][s] = X[s][r] for r > s
+    // ---- bf16 images T (for the backward only), Bw, Bu: thread = rows nr4 .. nr4 + 3, columns
+    // s0 .. s0 + 7 (one 16-byte chunk of each row), from T[r][s] = X[s][r] for r > s
     {
         const int nr4 = 4 * (tid & 15), ch = tid >> 4, s0 = 8 * ch;
         uint8_t* img = timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kWyImgBytes;
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
                 bw[e] = v[q][e] * sw[e];
                 bu[e] = v[q][e] * su[e];
             }
-            *reinterpret_cast<uint4*>(img + off) = pack8(v[q]);
+            if (with_t) *reinterpret_cast<uint4*>(img + off) = pack8(v[q]);  // the backward reads T
             *reinterpret_cast<uint4*>(img + kTImgBytes + off) = pack8(bw);
             *reinterpret_cast<uint4*>(img + 2 * kTImgBytes + off) = pack8(bu);
         }
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
 }  // namespace
 
 gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, int32_t* flags, int nflags,
-                            cudaStream_t s) {
+                            bool with_t, cudaStream_t s) {
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
@@ -318,7 +318,7 @@ gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* 
     const dim3 grid((unsigned)slots, (unsigned)p.Hv);
     if ((int64_t)nflags > slots * p.Hv) return GDN_ERR_DEVICE;  // every flag has a CTA to clear it
     gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws, (float2*)(ws + wy_tc_summary_offset(p)),
-                                                          flags, nflags);
+                                                          flags, nflags, with_t ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
