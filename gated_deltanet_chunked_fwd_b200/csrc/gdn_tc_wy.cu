@@ -42,6 +42,8 @@ namespace {
 
 constexpr int kWyThreads = 128;
 constexpr int kWyMinBlocks = 7;  // CTAs per SM the shared memory and registers are sized for
+constexpr int kWyMinBlocksGrouped = 6;  // with grouped value heads: the loop over the group keeps
+                                        // a few more values live (80 registers)
 // shared memory (bytes from a 1024-aligned base: the TMA destination is 128-byte swizzled)
 constexpr uint32_t wK = 0;                          // 16 KB bf16 K [dk half][64 rows][128 B];
                                                     // then fp32 X [64][kXs]
@@ -84,19 +86,24 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
     return true;
 }
 
-__global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
+// kGrouped: value heads share q/k heads (p.group > 1); the CTA loops over the group.  Without
+// grouping the loop has one pass and compiles away.
+template <bool kGrouped>
+__global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : kWyMinBlocks)
     gdn_wy_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const Problem p, uint8_t* __restrict__ timg,
                      float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags, int with_t) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) prefetch_tensormap(&tm_k);  // its first use is a few hundred cycles away
-    const int h = blockIdx.y, hk = h / p.group, Hv = p.Hv;
+    // one CTA per (chunk slot, q/k head): the Gram block of the head's K is formed once and serves
+    // every value head of its group (value heads hk G .. hk G + G - 1 share k)
+    const int hk = blockIdx.y, G = kGrouped ? p.group : 1, Hv = p.Hv;
     int n = 0, c = 0;
     int64_t bos = 0, len = 0;
-    // the state chain's scan flags start at zero (CTA (x, h) clears flag x Hv + h; the chain's CTAs
-    // are fewer than the image slots times the value heads)
-    if (tid == 0 && (int64_t)blockIdx.x * Hv + h < nflags) flags[(int64_t)blockIdx.x * Hv + h] = 0;
+    // the state chain's scan flags start at zero (CTA (x, hk) clears flags x Hv + hk G + i; the
+    // chain's CTAs are fewer than the image slots times the value heads)
+    if (tid < G && (int64_t)blockIdx.x * Hv + hk * G + tid < nflags) flags[(int64_t)blockIdx.x * Hv + hk * G + tid] = 0;
     const bool live = locate_slot(p, blockIdx.x, &n, &c, &bos, &len);  // CTA-uniform
     uint64_t* bar = (uint64_t*)(sm + wBar);
     uint64_t* bar_mma = bar + 1;
@@ -116,17 +123,18 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
 
     // ---- K tile by TMA ([dk half][64 rows][128 B], 128-byte swizzled).  Rows past the chunk
     // (the next sequence's tokens, or zeros past the tensor's end) only reach entries of A that
-    // the mask below sets to zero.  The chunk's gates are loaded meanwhile.
+    // the mask below sets to zero.  The first value head's gates are loaded meanwhile.
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar_mma, 1);
         fence_barrier_init();
     }
-    float x = 0.f, bt = 0.f;
-    if (tid < lc) {  // lc <= 64
-        x = p.g[(t0 + tid) * Hv + h];
-        bt = p.beta[(t0 + tid) * Hv + h];
-    }
+    float xg = 0.f, bt = 0.f;
+    auto load_gates = [&](int h) {
+        xg = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;  // lc <= 64
+        bt = tid < lc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
+    };
+    load_gates(hk * G);
     tc_fence_before();
     __syncthreads();  // the barriers are initialised, the TMEM base is written
     tc_fence_after();
@@ -136,16 +144,35 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         tma_load_3d(sm + wK, &tm_k, bar, 0, hk, (int)t0);
         tma_load_3d(sm + wK + 8192, &tm_k, bar, 64, hk, (int)t0);
     }
-
-    // ---- gates: gamma = cumsum g (two warp scans), E_rs = a_r b_s when factorable
     float* vbeta = (float*)(sm + wVec);
     float* vgam = vbeta + 64;
     float* va = vbeta + 128;
     float* vb = vbeta + 192;
     float* vnrm = vbeta + 256;
     float* vbG = vbeta + 320;
+    float* X = (float*)(sm + wK);
+
+    // ---- K K^T on the tensor core: D = A K^T with A the K tile read as 128 rows (D rows 0-63 are
+    // the Gram block; rows 64-127 come from the bytes after the tile and are not read), N = 64,
+    // bf16 in, fp32 out in TMEM lanes 0-63 (one K row per lane)
+    bool ok = __syncthreads_and(mbar_wait(bar, 0));  // the K tile has landed
+    if (ok && tid == 0) {
+        const uint64_t dK = desc_sw128(smem_u32(sm + wK), 16, 1024);
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)  // K steps of 16: four per 64-wide k half (8 KB apart)
+            mma_bf16_ss(tmem, dK + (((j >> 2) * 8192 + (j & 3) * 32) >> 4),
+                        dK + (((j >> 2) * 8192 + (j & 3) * 32) >> 4), idesc_bf16(128, 64, 0, 0), j > 0);
+        mma_commit(bar_mma);
+    }
+    if (!ok && tid == 0) report(p.status, GDN_ERR_TIMEOUT);
+
+    for (int gi = 0; gi < G && ok; ++gi) {
+    const int h = hk * G + gi;  // the value head of this pass
+    // ---- gates: gamma = cumsum g (two warp scans), E_rs = a_r b_s when factorable
     float gr = 0.f;
     if (tid < 64) {
+        float x = xg;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -166,24 +193,18 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         vb[tid] = fac ? expf(gm - gr) : gr * LOG2E;
         vbG[tid] = bt * expf(gr);
     }
-
-    // ---- K K^T on the tensor core: D = A K^T with A the K tile read as 128 rows (D rows 0-63 are
-    // the Gram block; rows 64-127 come from the bytes after the tile and are not read), N = 64,
-    // bf16 in, fp32 out in TMEM lanes 0-63 (one K row per lane)
-    bool ok = __syncthreads_and(mbar_wait(bar, 0));  // vectors written, the K tile has landed
-    if (ok && tid == 0) {
-        const uint64_t dK = desc_sw128(smem_u32(sm + wK), 16, 1024);
-        tc_fence_after();
-#pragma unroll
-        for (int j = 0; j < 8; ++j)  // K steps of 16: four per 64-wide k half (8 KB apart)
-            mma_bf16_ss(tmem, dK + (((j >> 2) * 8192 + (j & 3) * 32) >> 4),
-                        dK + (((j >> 2) * 8192 + (j & 3) * 32) >> 4), idesc_bf16(128, 64, 0, 0), j > 0);
-        mma_commit(bar_mma);
-    }
-    ok = ok && __syncthreads_and(mbar_wait(bar_mma, 0));
-    if (!ok) {
-        if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
+    if (gi + 1 < G) load_gates(h + 1);  // the next value head's gates, while this one runs
+    // the Gram block is in TMEM (the first pass waits for it) and the vectors are written
+    if (gi == 0) {
+        ok = __syncthreads_and(mbar_wait(bar_mma, 0));
+        if (!ok) {
+            if (tid == 0) report(p.status, GDN_ERR_TIMEOUT);
+            break;
+        }
     } else {
+        __syncthreads();
+    }
+    {
         tc_fence_after();
         // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> X, row r by thread r (warps 0 and 1 read
         // TMEM lanes 0-63).  X overwrites the K tile, which the MMA has read.  Entries below the
@@ -231,6 +252,7 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
         }
         tc_fence_before();
         __syncthreads();
+    }
     // Chunk summary for the forward's gate-driven split: the summed log decay of the chunk and
     // whether some token breaks 0 <= beta |k|^2 <= 2 (the condition under which each token's
     // state map has norm <= exp(g)).
@@ -296,7 +318,8 @@ __global__ void __launch_bounds__(kWyThreads, kWyMinBlocks)
             *reinterpret_cast<uint4*>(img + 2 * kTImgBytes + off) = pack8(bu);
         }
     }
-    }  // ok
+    __syncthreads();  // the images have read X and the vectors: the next value head may overwrite them
+    }  // value heads
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -312,13 +335,13 @@ gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* 
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(gdn_wy_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)wSmemBytes) != cudaSuccess)
+    auto kern = p.group > 1 ? gdn_wy_tc_kernel<true> : gdn_wy_tc_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const dim3 grid((unsigned)slots, (unsigned)p.Hv);
+    const dim3 grid((unsigned)slots, (unsigned)p.Hk);
     if ((int64_t)nflags > slots * p.Hv) return GDN_ERR_DEVICE;  // every flag has a CTA to clear it
-    gdn_wy_tc_kernel<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws, (float2*)(ws + wy_tc_summary_offset(p)),
-                                                          flags, nflags, with_t ? 1 : 0);
+    kern<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws, (float2*)(ws + wy_tc_summary_offset(p)), flags, nflags,
+                                              with_t ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
