@@ -13,8 +13,8 @@
 //
 // The work per chunk is small and latency-bound (a 64 x 64 x 128 Gram block and a 64 x 64
 // triangular inverse), so the kernel is built for many chunks in flight rather than for one
-// fast chunk: 128 threads, 72 registers, about 25 KB of shared memory and 64 TMEM columns per
-// CTA, seven CTAs per SM, so that a 4096-token, 16-head call (1024 chunks) runs as one wave.  The
+// fast chunk: 128 threads, 64 registers, about 25 KB of shared memory and 64 TMEM columns per
+// CTA, eight CTAs per SM, so that a 4096-token, 16-head call (1024 chunks) runs as one wave.  The
 // K tile comes in by TMA.  The Gram block K K^T is one tcgen05 MMA group (M = 128, N = 64, bf16
 // in, fp32 out in TMEM); two warps read its rows and scale them into A.  The inverse is blocked:
 // the four 16 x 16 diagonal blocks by fp32 substitution, then three merge levels as warp-level
@@ -41,7 +41,7 @@ using namespace tc;
 namespace {
 
 constexpr int kWyThreads = 128;
-constexpr int kWyMinBlocks = 7;  // CTAs per SM the shared memory and registers are sized for
+constexpr int kWyMinBlocks = 8;  // CTAs per SM the shared memory and registers are sized for (64 registers)
 constexpr int kWyMinBlocksGrouped = 6;  // with grouped value heads: the loop over the group keeps
                                         // a few more values live (80 registers)
 // shared memory (bytes from a 1024-aligned base: the TMA destination is 128-byte swizzled)
@@ -209,14 +209,17 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
         // ---- A = strictly-lower(beta_r (K K^T)_rs E_rs) -> X, row r by thread r (warps 0 and 1 read
         // TMEM lanes 0-63).  X overwrites the K tile, which the MMA has read.  Entries below the
         // diagonal 16 x 16 blocks are merge operands only: stored rounded to tf32.  The diagonal of
-        // K K^T gives |k_r|^2 for the chunk summary.
+        // K K^T gives |k_r|^2 for the chunk summary.  Blocks above the diagonal ones are neither
+        // read nor stored: their places in X receive T before anything reads them.  Warp 0 (rows
+        // 0-31) has no entries in column blocks 2 and 3.
         float* X = (float*)(sm + wK);
         if (warp < 2) {
             const int r = tid;
             const float br = vbeta[r], ar = va[r];
             float* xr = X + r * kXs;
+            const int qn = warp == 0 ? 2 : 4;  // warp-uniform: the TMEM load is warp-collective
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {  // 16 columns s = 16 q .. 16 q + 15 at a time
+            for (int q = 0; q < qn; ++q) {  // 16 columns s = 16 q .. 16 q + 15 at a time
                 float v[16];
                 tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + 16 * q, v);
                 if ((r >> 4) == q) {  // the diagonal entry, by an unrolled select (no indexed registers)
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
                 // above the diagonal it may overflow.  Entries below the diagonal 16 x 16 blocks
                 // (q < r / 16) are merge operands only: stored rounded to tf32.
                 const bool below = q < (r >> 4);
+                const bool store = q <= (r >> 4);
                 if (fac) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) v[e] *= ar * vb[16 * q + e];
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
                         const float x = (s < r && r < lc) ? br * v[4 * e4 + e] : 0.f;
                         o[e] = below ? tf32r(x) : x;
                     }
-                    *reinterpret_cast<float4*>(xr + 16 * q + 4 * e4) = make_float4(o[0], o[1], o[2], o[3]);
+                    if (store) *reinterpret_cast<float4*>(xr + 16 * q + 4 * e4) = make_float4(o[0], o[1], o[2], o[3]);
                 }
             }
         }
