@@ -56,7 +56,8 @@ constexpr uint32_t cR1 = 192;  // Q K^T / K K^T, later dk^T (main part)
 constexpr uint32_t cR2 = 256;  // W^T, later TdU^T, later dKd^T
 constexpr uint32_t cR3 = 320;  // Ut^T -> U^T, later [dP ; dA'], later K^T (dP o E)^T
 constexpr uint32_t cR4 = 384;  // dO^T P, later H dO^T
-constexpr uint32_t cR5 = 448;  // dH^T K^T, then bf16 dU^T (cols 0..31), later TdW^T
+constexpr uint32_t cR5 = 448;  // dH^T K^T, then bf16 dU^T (cols 0..31), later H TdU^T = -TdW^T
+                               // (the second half of one N = 128 product with R4)
 
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t bQK = 0;        // 32 KB [dk atom][q rows 0-63 | k rows 64-127][128 B]
@@ -69,7 +70,7 @@ constexpr uint32_t bBu = 131072;   // 8 KB  T diag(beta)      (over Bw + Bu)
 // T, Bw, Bu arrive together: one copy of the WY step's three images
 static_assert(bBw == bT + kTImgBytes && bBu == bBw + kTImgBytes, "WY images are contiguous");
 constexpr uint32_t bP = 139264;    // 8 KB  P [64 r][64 s]; later dP o E
-constexpr uint32_t bWt = 147456;   // 16 KB -W^T [128 dk rows][64 s]; later -TdU^T [128 dv rows][64 r]
+constexpr uint32_t bWt = 147456;   // 16 KB -W^T [128 dk rows][64 s]
 constexpr uint32_t bUt = 163840;   // 16 KB U^T [128 dv rows][64 s]
 constexpr uint32_t bDHt = 180224;  // 32 KB bf16 dH^T [dk atom][128 dv rows][128 B]
 constexpr uint32_t bVec = 212992;  // per-token vectors (8 x 64 floats)
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(kNT, 1)
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(bar_mma, 2);  // one arrival per MMA issuer
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -238,10 +239,23 @@ __global__ void __launch_bounds__(kNT, 1)
     const uint32_t id_mm64 = idesc_bf16(128, 64, 1, 1);
     const uint32_t id_mm128 = idesc_bf16(128, 128, 1, 1);
     const uint32_t id_kk128 = idesc_bf16(128, 128, 0, 0);
+    const uint32_t id_mk128 = idesc_bf16(128, 128, 1, 0);
     const float LOG2E = 1.4426950408889634f;
 
-    auto mma_sync_wait = [&]() -> bool {
-        if (tid == 0) mma_commit(bar_mma);
+    // Two threads in different warps (0 and 32) issue the MMAs of a batch that write different
+    // accumulators: one thread issues an N = 64 MMA about every 60 cycles, about twice the tensor
+    // pipe's time for it, so two issuers finish a batch sooner.  Each commits its own MMAs to
+    // bar_mma (two arrivals); a thread that issued none in a batch arrives directly.
+    constexpr int kIss2 = 32;
+    auto mma_sync_wait = [&](bool first, bool second) -> bool {
+        if (tid == 0) {
+            if (first) mma_commit(bar_mma);
+            else mbar_arrive(bar_mma);
+        }
+        if (tid == kIss2) {
+            if (second) mma_commit(bar_mma);
+            else mbar_arrive(bar_mma);
+        }
         const bool r = __syncthreads_and(mbar_wait(bar_mma, ph_mma));
         ph_mma ^= 1;
         tc_fence_after();
@@ -325,24 +339,42 @@ __global__ void __launch_bounds__(kNT, 1)
             }
         }
     };
-    // q, k, v, dO tiles and the T / Bw / Bu images of chunk c; the H image too for the chunks
-    // that emit.  The buffers' last generic reads and writes were before the caller's barrier.
-    auto load_qkv = [&](int c, bool with_h) {
+    // Inputs of chunk c, all on bar_ld (one phase per chunk).  dO and the H image (chunks that
+    // emit) are fetched as soon as the previous chunk in the walk has finished with their buffers
+    // (after its [dP ; dA'] / H [dO ; TdU]^T products), v once its buffer has served as G there;
+    // those fetches add their bytes to the phase without arriving.  q, k and the WY images follow
+    // at the top of chunk c with the phase's one arrival.  The buffers' last generic reads and
+    // writes were before the caller's barrier.
+    auto load_do_h = [&](int c, bool with_h) {
         if (tid == 0) {
             const int t0 = (int)(bos + (int64_t)c * kChunk);
             fence_proxy_async();
-            mbar_arrive_expect_tx(bar_ld, 65536 + kWyImgBytes + (with_h ? kHImg : 0));
+            mbar_expect_tx(bar_ld, 16384 + (with_h ? kHImg : 0));  // dO: 2 x 8 KB (rows 0-63 of its tile)
+            for (int a = 0; a < 2; ++a) tma_load_3d(sm + bDO + a * 16384, &tm_do, bar_ld, 64 * a, h, t0);
+            if (with_h) bulk_load(sm + bHt, args.himg + (img_slot(bos, n, c) * Hv + h) * kHImg, kHImg, bar_ld);
+        }
+    };
+    auto load_v = [&](int c) {
+        if (tid == 0) {
+            const int t0 = (int)(bos + (int64_t)c * kChunk);
+            fence_proxy_async();
+            mbar_expect_tx(bar_ld, 16384);  // v: 2 x 8 KB
+            for (int a = 0; a < 2; ++a) tma_load_3d(sm + bV + a * 8192, &tm_v, bar_ld, 64 * a, h, t0);
+        }
+    };
+    auto load_qk_wy = [&](int c) {
+        if (tid == 0) {
+            const int t0 = (int)(bos + (int64_t)c * kChunk);
+            fence_proxy_async();
+            mbar_arrive_expect_tx(bar_ld, 32768 + kWyImgBytes);  // q, k: 4 x 8 KB
             for (int a = 0; a < 2; ++a) {
                 tma_load_3d(sm + bQK + a * 16384, &tm_q, bar_ld, 64 * a, hk, t0);
                 tma_load_3d(sm + bQK + a * 16384 + 8192, &tm_k, bar_ld, 64 * a, hk, t0);
-                tma_load_3d(sm + bV + a * 8192, &tm_v, bar_ld, 64 * a, h, t0);
-                tma_load_3d(sm + bDO + a * 16384, &tm_do, bar_ld, 64 * a, h, t0);
             }
-            const int64_t gi = img_slot(bos, n, c) * Hv + h;
-            if (with_h) bulk_load(sm + bHt, args.himg + gi * kHImg, kHImg, bar_ld);
-            bulk_load(sm + bT, args.timg + gi * kWyImgBytes, kWyImgBytes, bar_ld);
+            bulk_load(sm + bT, args.timg + (img_slot(bos, n, c) * Hv + h) * kWyImgBytes, kWyImgBytes, bar_ld);
         }
     };
+    bool pre = false;  // dO, H and v of this chunk were fetched during the previous one
 
     // ===================== reverse walk with the state adjoint =====================
     {  // dH^T <- dS_T at the sequence end, zero at the start of a reverse warm-up
@@ -378,7 +410,12 @@ __global__ void __launch_bounds__(kNT, 1)
             acc_b[tid] = 0.f;
         }
         if (tid < 8) acc_s[tid] = 0.f;
-        load_qkv(c, emit);
+        if (!pre) {
+            load_do_h(c, emit);
+            load_v(c);
+        }
+        load_qk_wy(c);
+        pre = false;
         const bool fac = gates(c, lc);
         ok = __syncthreads_and(mbar_wait(bar_ld, ph_ld));
         ph_ld ^= 1;
@@ -387,7 +424,7 @@ __global__ void __launch_bounds__(kNT, 1)
         tc_fence_before();
         __syncthreads();
         mma1();
-        if (!(ok = mma_sync_wait())) break;
+        if (!(ok = mma_sync_wait(true, false))) break;
         // P (rows 0..63) -> smem
         if (m < 64) {  // P row m, this thread's half of the columns
             const int r = m;
@@ -413,6 +450,9 @@ __global__ void __launch_bounds__(kNT, 1)
                 mma_bf16_ss(tmem + cR3, desc_sw128(sb + bV + j * 2048, 8192, 1024),
                             desc_sw128(sb + bBu + j * 32, 16, 1024), id_mk64, j > 0);
             }
+        }
+        if (tid == kIss2) {
+            tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 4; ++j)  // dO^T P (R4): A = dO^T MN-major, B = P MN-major (N = s)
                 mma_bf16_ss(tmem + cR4, desc_sw128(sb + bDO + j * 2048, 16384, 1024),
@@ -424,7 +464,7 @@ __global__ void __launch_bounds__(kNT, 1)
                             id_kk64, j > 0);
             }
         }
-        if (!(ok = mma_sync_wait())) break;
+        if (!(ok = mma_sync_wait(true, true))) break;
         {  // -W^T -> Wt;  Q rows * Gam -> Qg (over Bw/Bu);  dU^T -> bf16 (R5 cols 0..31);
            // <dH_c, H_c>, then dH^T <- Gam_n dH^T
             float v[64];
@@ -503,6 +543,9 @@ __global__ void __launch_bounds__(kNT, 1)
                     mma_bf16_ts(tmem + cR2, tmem + cR5 + 8 * j, desc_sw128(sb + bT + j * 2048, 8192, 1024),
                                 id_km64, j > 0);
             }
+        }
+        if (tid == kIss2) {
+            tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 4; ++j)  // dH^T += dO^T Qg   (B = Qg MN-major, N = dk)
                 mma_bf16_ss(tmem + cH, desc_sw128(sb + bDO + j * 2048, 16384, 1024),
@@ -512,9 +555,9 @@ __global__ void __launch_bounds__(kNT, 1)
                 mma_bf16_ts(tmem + cH, tmem + cR5 + 8 * j, desc_sw128(sb + bWt + j * 32, 16, 1024),
                             id_kk128, 1);
         }
-        if (!(ok = mma_sync_wait())) break;
+        if (!(ok = mma_sync_wait(emit, true))) break;
         if (emit) {  // the chunk's gradients (own chunks only)
-            {  // U^T -> Ut;  TdU: dv out, rows 64..127 of the dO tile, -TdU^T -> Wt, dbeta part;
+            {  // U^T -> Ut;  TdU: dv out, rows 64..127 of the dO tile, dbeta part;
                // this thread: row m of U^T and of TdU^T, tokens [32 hh, 32 hh + 32) in groups of 8
                 __nv_bfloat16* dvp = (__nv_bfloat16*)b.dv + (t0 * Hv + h) * dv + m;
 #pragma unroll 1
@@ -535,9 +578,7 @@ __global__ void __launch_bounds__(kNT, 1)
                         // TdU row r of the stacked [dO ; TdU] tile: element (64 + r, m)
                         *reinterpret_cast<__nv_bfloat16*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
                                                           (m & 7) * 2) = __float2bfloat16_rn(t8[e]);
-                        t8[e] = -t8[e];
                     }
-                    *reinterpret_cast<uint4*>(sm + bWt + sw128_off(m, tb >> 3)) = pack8(t8);
                     // sums over this warp's 32 m for each token: lane l ends with token tb + l / 4
                     warp_reduce_scatter<8>(bvals, lane);
                     bvals[0] += __shfl_xor_sync(0xffffffffu, bvals[0], 2);
@@ -561,21 +602,25 @@ __global__ void __launch_bounds__(kNT, 1)
                                 desc_sw128(sb + bUt + j * 2048, 8192, 1024), id_km64, j > 0);
                 }
     #pragma unroll
-                for (int j = 0; j < 8; ++j) {  // H dO^T (R4): A = H (MN-major view of H^T), B = dO rows
-                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
-                    mma_bf16_ss(tmem + cR4, desc_sw128(sb + bHt + j * 2048, 16384, 1024),
-                                desc_sw128(sb + bDO + koff, 16, 1024), id_mk64, j > 0);
-                }
-    #pragma unroll
-                for (int j = 0; j < 8; ++j)  // TdW^T = H (-TdU^T)^T... = -H TdU^T (R5): B = -TdU^T MN-major
-                    mma_bf16_ss(tmem + cR5, desc_sw128(sb + bHt + j * 2048, 16384, 1024),
-                                desc_sw128(sb + bWt + j * 2048, 8192, 1024), id_mm64, j > 0);
-    #pragma unroll
                 for (int j = 0; j < 8; ++j)  // dKd^T = dH U^T (R2): A = dH (MN-major view of dH^T)
                     mma_bf16_ss(tmem + cR2, desc_sw128(sb + bDHt + j * 2048, 16384, 1024),
                                 desc_sw128(sb + bUt + j * 2048, 8192, 1024), id_mm64, j > 0);
             }
-            if (!(ok = mma_sync_wait())) break;
+            if (tid == kIss2) {
+                tc_fence_after();
+    #pragma unroll
+                for (int j = 0; j < 8; ++j) {  // H [dO ; TdU]^T (R4 | R5, N = 128): A = H (MN-major view of
+                                               // H^T), B = the stacked [dO ; TdU] rows; R4 = H dO^T and
+                                               // R5 = H TdU^T = -TdW^T
+                    const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
+                    mma_bf16_ss(tmem + cR4, desc_sw128(sb + bHt + j * 2048, 16384, 1024),
+                                desc_sw128(sb + bDO + koff, 16, 1024), id_mk128, j > 0);
+                }
+            }
+            if (!(ok = mma_sync_wait(true, true))) break;
+            // the next chunk's dO and H image: this chunk's last reads of them were the products above
+            pre = c - 1 >= c0;
+            if (pre) load_do_h(c - 1, c - 1 < c1);
             {  // dP (lanes 0..63) and dA (lanes 64..127) rows, columns s in [32 hh, 32 hh + 32) in
                // four groups of eight: dgamma / dbeta terms, dP o E, G
                 const int r = m & 63;
@@ -664,12 +709,9 @@ __global__ void __launch_bounds__(kNT, 1)
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
+            if (pre) load_v(c - 1);  // G (over the v tile) has been read
             if (tid == 0) {
                 tc_fence_after();
-    #pragma unroll
-                for (int j = 0; j < 4; ++j)  // K^T (dP o E)^T (R3): A = K^T MN-major, B = dPE rows K-major
-                    mma_bf16_ss(tmem + cR3, desc_sw128(sb + bQK + 8192 + j * 2048, 16384, 1024),
-                                desc_sw128(sb + bP + j * 32, 16, 1024), id_mk64, j > 0);
     #pragma unroll
                 for (int j = 0; j < 4; ++j)  // dk^T main (R1): Q^T (dP o E) + K^T S^T
                     mma_bf16_ss(tmem + cR1, desc_sw128(sb + bQK + j * 2048, 16384, 1024),
@@ -679,7 +721,14 @@ __global__ void __launch_bounds__(kNT, 1)
                     mma_bf16_ss(tmem + cR1, desc_sw128(sb + bQK + 8192 + j * 2048, 16384, 1024),
                                 desc_sw128(sb + bT + j * 32, 16, 1024), id_mk64, 1);
             }
-            if (!(ok = mma_sync_wait())) break;
+            if (tid == kIss2) {
+                tc_fence_after();
+    #pragma unroll
+                for (int j = 0; j < 4; ++j)  // K^T (dP o E)^T (R3): A = K^T MN-major, B = dPE rows K-major
+                    mma_bf16_ss(tmem + cR3, desc_sw128(sb + bQK + 8192 + j * 2048, 16384, 1024),
+                                desc_sw128(sb + bP + j * 32, 16, 1024), id_mk64, j > 0);
+            }
+            if (!(ok = mma_sync_wait(true, true))) break;
             {  // epilogue: thread i = dk index (TMEM lane), tokens [32 hh, 32 hh + 32) in four
                // groups of eight (a rolled loop: a short body keeps the instruction stream small)
                 const int i = m;
@@ -700,6 +749,8 @@ __global__ void __launch_bounds__(kNT, 1)
                     // H dO^T, K^T dPE^T, dk main, dKd^T, TdW^T for the group's 8 tokens
                     tmem_ld8x5(tl + cR4 + tb, hdo, tl + cR3 + tb, kpe, tl + cR1 + tb, dkm, tl + cR2 + tb, dkd,
                                tl + cR5 + tb, tdw);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) tdw[e] = -tdw[e];  // R5 holds H TdU^T = -TdW^T
                     float gam8[8], dec8[8], bg8[8];
 #pragma unroll
                     for (int h4 = 0; h4 < 2; ++h4) {
@@ -776,6 +827,10 @@ __global__ void __launch_bounds__(kNT, 1)
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+    }
+    if (!ok && pre) {  // fetches for the next chunk are in flight: let them land before the CTA exits
+        if (tid == 0) mbar_arrive(bar_ld);
+        (void)mbar_wait(bar_ld, ph_ld);
     }
     if (ok && b.dS0 && seg == 0) {
         float* dst = b.dS0 + ((int64_t)n * Hv + h) * dk * dv + m;
