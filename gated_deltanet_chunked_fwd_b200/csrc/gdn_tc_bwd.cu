@@ -392,6 +392,13 @@ __global__ void __launch_bounds__(kNT, 1)
         const bool emit = c < c1;  // own chunk (else: reverse warm-up, the dH chain only)
         const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
         const int64_t t0 = bos + (int64_t)c * kChunk;
+        // this chunk's inputs (first of all: their latency overlaps the copies and gates below)
+        if (!pre) {
+            load_do_h(c, emit);
+            load_v(c);
+        }
+        load_qk_wy(c);
+        pre = false;
         // bf16 copies of the exit adjoint dH_c: TMEM (A operand) and smem (MN-major A of dKd)
         {
             float v[64];
@@ -410,12 +417,6 @@ __global__ void __launch_bounds__(kNT, 1)
             acc_b[tid] = 0.f;
         }
         if (tid < 8) acc_s[tid] = 0.f;
-        if (!pre) {
-            load_do_h(c, emit);
-            load_v(c);
-        }
-        load_qk_wy(c);
-        pre = false;
         const bool fac = gates(c, lc);
         ok = __syncthreads_and(mbar_wait(bar_ld, ph_ld));
         ph_ld ^= 1;
