@@ -550,6 +550,26 @@ def run_ours(args, world, rank, local):
                        + (" + dq/dk group reduction" if bi["v"].shape[2] != bi["q"].shape[2] else ""),
                "launches": gdn.launch_count(*qs[:5], backward=True)}
         del bi, qs, wsb
+        if not args.no_extra:
+            # the long context with weak decay (g = -softplus(N(-7,1))): reverse warm-ups would be
+            # ~200 chunks long or fail, so segments take their exit adjoint from the adjoint scan;
+            # against one reverse walk per head
+            wb = make_workload(4, seed=rank, device=dev, B=1, T=65536, g_mu=-7.0)
+            qs = [wb[n] for n in ("q", "k", "v", "beta", "g", "do")]
+            wsb = torch.empty(max(gdn.gdn_chunk_bwd_workspace_size(*qs[:5]), 1), dtype=torch.uint8,
+                              device=dev)
+            wt = wb["q"].shape[1]
+            for label, flags in (("split_auto_scan", 0), ("split_off", GDN_FLAG_SPLIT_OFF)):
+                def wstep(flags=flags):
+                    gdn.gdn_chunk_bwd(*qs, dST=wb["dST"], workspace=wsb, flags=flags)
+
+                wms = measure(wstep, max(1, min(args.steps, 3)), warm=1)
+                bwd[f"bwd_bf16_T65536_H16_d128_weakdecay_{label}"] = {
+                    "ms": wms, "tokens_per_s": job_throughput(wt, world, wms),
+                    "launches": gdn.launch_count(*qs[:5], backward=True, flags=flags),
+                    "roofline": roofline(bd * wt * Hv, bwd_bytes(wt, wb["q"].shape[2], Hv, dk, dv, 1),
+                                         wms * 1e-3, hbm, bf16, src)}
+            del wb, qs, wsb
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu_base = None

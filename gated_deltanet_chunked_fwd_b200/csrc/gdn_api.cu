@@ -157,7 +157,7 @@ gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan) {
     if (plan->use_tc) {
         size_t o1, o2, o3, o4;
         plan->total = align_up(tc_bwd_workspace(p, plan->cu_host, plan->split_mode, &o1, &o2, &o3, &o4), kAlign);
-        plan->launches = tc_bwd_launches(p);
+        plan->launches = tc_bwd_launches(p, plan->cu_host, plan->split_mode);
         return GDN_OK;
     }
     size_t off = 0;

@@ -88,9 +88,10 @@ size_t wy_tc_workspace(const Problem& p);
 size_t wy_tc_summary_offset(const Problem& p);
 // WY + fused kernel in replay mode: bf16 H^T entry-state image (32 KB) of every chunk, by
 // (image slot, value head), into himg; `ws` holds the WY outputs (wy_tc_workspace bytes);
-// split_mode as in FwdPlan
+// split_mode as in FwdPlan; the WY launch also zeroes the nrflags int32 flags at rflags (the
+// backward's adjoint scan)
 gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, int split_mode, char* ws,
-                            uint8_t* himg, cudaStream_t s);
+                            uint8_t* himg, cudaStream_t s, int32_t* rflags, int nrflags);
 int tc_fwd_launches(const Problem& p);
 bool tc_fwd_supported(const Problem& p);
 
@@ -108,7 +109,7 @@ gdn_status launch_bwd_reduce(const BwdProblem& b, const float* dqw, const float*
 bool tc_bwd_supported(const Problem& p);
 size_t tc_bwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode, size_t* off_himg,
                         size_t* off_timg, size_t* off_dqw, size_t* off_dkw);
-int tc_bwd_launches(const Problem& p);
+int tc_bwd_launches(const Problem& p, const int32_t* cu_host, int split_mode);
 gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s);
 
 // shared SIMT pieces (also used by the backward's forward recompute)

@@ -2,19 +2,22 @@
 // sm_100a).  The backward of the GDN layer (FlashQLA pages: dothoosh.com article, opening
 // paragraph, "backward pass"; news.hamidun.com page, "large-scale pretraining" scenario).
 //
-// Four launches: the WY kernel (T, T diag(beta Gam), T diag(beta) images and per-chunk gate
-// summaries), the fused forward
-// kernel in replay mode (the bf16 entry state H^T of every chunk, as a ready-to-use
-// 128-byte-swizzled shared-memory image), this reverse kernel, and the reduction of dq / dk over
-// grouped value heads.  The reverse kernel runs one CTA per (sequence, value head, segment of
+// Three to five launches: the WY kernel (T, T diag(beta Gam), T diag(beta) images and per-chunk
+// gate summaries), the fused forward kernel in replay mode (the bf16 entry state H^T of every
+// chunk, as a ready-to-use 128-byte-swizzled shared-memory image), in sequences of at least four
+// segments the adjoint scan's pre-pass (this kernel with kPre), this reverse kernel, and with
+// grouped value heads the reduction of dq / dk over each group.  The reverse kernel runs one CTA per (sequence, value head, segment of
 // chunks), 256 threads: the two warps of each TMEM lane quarter share its lanes (thread <-> MMA
 // row) and split each row's columns, or tokens, in halves.  A segment walks its chunks
 // backwards with the state adjoint dH (fp32, TMEM).  Its exit adjoint comes from a reverse
 // warm-up: the adjoint map of a chunk, dH -> (Gam_n I - W^T Kd) dH, is the transpose of the
 // chunk's state map and has the same norm bound exp(sum g) while 0 <= beta |k|^2 <= 2, so a
 // segment that does not end its sequence starts from dH = 0 a few chunks later (until the summed
-// log decay reaches log eps) and runs only the dH chain there; otherwise, or when the decay stays
-// weak, it starts exactly from dS_T at the sequence end.  Per chunk (notation of
+// log decay reaches log eps) and runs only the dH chain there.  Where that warm-up fails, or
+// would be long, the segment starts exactly from the entry adjoint that the adjoint scan's
+// pre-pass recorded (in sequences of at least four segments), else from dS_T at the sequence
+// end.  Every chunk maps the adjoint affinely, dH_c = (Gam_n I - W^T Kd) dH_c+1 + b_c, so the
+// scan is the forward's affine scan run backwards over the segments.  Per chunk (notation of
 // gdn_internal.cuh; E, Gam, dec, beta from the gates; Kb = diag(beta Gam) K):
 //   U^T  = Ut^T - H^T W^T                         (recomputed, MMAs)
 //   dU^T = dO^T P + (dH^T K^T) diag(dec)
@@ -34,6 +37,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <type_traits>
 #include <vector>
 
 #include "gdn_internal.cuh"
@@ -79,6 +83,8 @@ constexpr uint32_t bBar = bRed + 2048;
 constexpr uint32_t kSmemB = bBar + 64 + 1024;
 
 constexpr uint32_t kHImg = 32768;  // bytes of one saved H^T image
+constexpr int kRevScanMinSegs = 4;  // the adjoint scan is used in sequences of at least four segments
+constexpr int kRevScanFoldAllowance = 16;  // fold products, in dH-chain chunk steps
 
 struct TcBwdArgs {
     BwdProblem b;
@@ -90,6 +96,11 @@ struct TcBwdArgs {
     int L;                // chunks per segment
     int fixed_segs;       // segments per sequence when cu_seqlens is absent
     int auto_warm;        // 1: reverse warm-up for segments that do not end their sequence
+    // adjoint affine scan for segments whose reverse warm-up cannot reach log_eps: per CTA a flag
+    // and three fp32 [dk][dv] records (exit adjoint, M, B); nullptr (no sequence has enough
+    // segments): such a segment replays the dH chain from dS_T at the sequence end instead
+    int32_t* scan_flags;
+    float* scan_rec;
     float log_eps;        // the warm-up stops once the summed log decay is <= log_eps
 };
 
@@ -111,11 +122,61 @@ __device__ __forceinline__ void warp_reduce_scatter(float* v, int lane) {
     }
 }
 
+// End (exclusive) of the reverse warm-up of the segment whose chunks end at c1: the smallest w > c1
+// whose chunks c1 .. w-1 sum to a log decay <= log_eps (the per-chunk sums of the WY step's
+// summaries); -1 when the sum does not get there before the sequence end, or when one of those
+// chunks breaks 0 <= beta |k|^2 <= 2.  A whole warp searches 32 chunks at a time; every lane returns
+// the same.
+__device__ __forceinline__ int rev_warmup_end(const float2* summ, int64_t bos, int n, int h, int Hv, int c1,
+                                              int nck, float log_eps, int lane) {
+    float cum = 0.f;
+    bool bad = false;
+    for (int bot = c1; bot < nck; bot += 32) {
+        const int w = bot + lane;  // lane l looks at chunk bot + l
+        const float2 cs = w < nck ? summ[img_slot(bos, n, w) * Hv + h] : make_float2(0.f, 0.f);
+        float x = cs.x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, w < nck && cum + x <= log_eps);
+        if (hit) {
+            const int first = __ffs(hit) - 1;
+            bad |= __any_sync(0xffffffffu, lane <= first && cs.y != 0.f);
+            return bad ? -1 : bot + first + 1;
+        }
+        bad |= __any_sync(0xffffffffu, w < nck && cs.y != 0.f);
+        cum += __shfl_sync(0xffffffffu, x, 31);
+    }
+    return -1;
+}
+
+// the adjoint scan's flags: 0 nothing yet, 1 the segment's fold (M, B) is published, 2 its exit
+// adjoint is
+__device__ __forceinline__ void rflag_release(int32_t* f, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ int rflag_acquire(const int32_t* f) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float bf(const uint8_t* tile, int row, int col) {  // bf16 element of a swizzled tile
     const uint8_t* p = tile + sw128_off(row, (col & 63) >> 3) + (col & 7) * 2;
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
 }
 
+// kPre: the adjoint scan's pre-pass, which runs before the reverse walk with the gradients on the
+// same grid and runs the dH chain only.  A segment that takes the scan walks its own chunks twice,
+// from dH = 0 (the fold B) and from dH = I with dO = 0 (the fold M), publishes the fold, looks
+// forward for the nearest later segment whose exit adjoint is published, combines the folds in
+// between (X <- M X + B, fp32) into its entry adjoint, which it records for its reverse walk, and
+// publishes its own exit adjoint M X + B.  A segment that does not take the scan but has an
+// earlier one that does walks to its exit adjoint from its usual start and publishes it.  Every
+// other segment leaves at once.
+template <bool kPre>
 __global__ void __launch_bounds__(kNT, 1)
     gdn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -141,14 +202,17 @@ __global__ void __launch_bounds__(kNT, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hv = p.Hv, dk = 128, dv = 128;
-    // ---- which (sequence, head, segment) this CTA owns (the forward's scheme)
+    // ---- which (sequence, head, segment) this CTA owns (the forward's scheme, except that the
+    // later segments of a sequence take the lower block indices: a segment that takes the adjoint
+    // scan waits for later ones, which are then scheduled no later than it)
     const int h = blockIdx.x % Hv;
     const int sidx = blockIdx.x / Hv;
-    int n = 0, seg = 0;
+    int n = 0, seg = 0, segs_n = 1;
     int64_t bos = 0, len = 0;
     if (!p.cu) {
         n = sidx / args.fixed_segs;
-        seg = sidx % args.fixed_segs;
+        segs_n = args.fixed_segs;
+        seg = segs_n - 1 - sidx % args.fixed_segs;
         bos = (int64_t)n * p.T;
         len = p.T;
     } else {
@@ -174,7 +238,8 @@ __global__ void __launch_bounds__(kNT, 1)
             if (bal) {
                 const int src = __ffs(bal) - 1;
                 n = __shfl_sync(0xffffffffu, m, src);
-                seg = sidx - (base + __shfl_sync(0xffffffffu, incl - s_m, src));
+                segs_n = __shfl_sync(0xffffffffu, s_m, src);
+                seg = segs_n - 1 - (sidx - (base + __shfl_sync(0xffffffffu, incl - s_m, src)));
                 bos = __shfl_sync(0xffffffffu, b_m, src);
                 len = __shfl_sync(0xffffffffu, l_m, src);
                 found = true;
@@ -191,21 +256,43 @@ __global__ void __launch_bounds__(kNT, 1)
     const int c0 = min(nck, seg * args.L);
     const int c1 = min(nck, (seg + 1) * args.L);
     // ---- reverse warm-up: walk later chunks from dH = 0 until their summed log decay is
-    // <= log eps (exact start from dS_T at the sequence end otherwise)
+    // <= log eps.  In a sequence of at least kRevScanMinSegs segments the adjoint scan takes over
+    // where that fails, or where the warm-up would be longer than the scan's two fold walks over
+    // the own chunks plus an allowance for the fold products (every such segment scans, so that
+    // earlier ones find folds, not replays, between them and a published exit adjoint); else a
+    // failed warm-up becomes a replay of the dH chain from dS_T at the sequence end.
+    const bool scan_ok = args.scan_rec != nullptr && segs_n >= kRevScanMinSegs;
+    auto takes_scan = [&](int c0j, int c1j, int wj) {
+        return scan_ok && (wj < 0 || wj - c1j > 2 * (c1j - c0j) + kRevScanFoldAllowance);
+    };
     int cend = nck;
+    bool scan = false;
     if (c1 < nck && args.auto_warm) {
-        float cum = 0.f;
-        int w = c1;
-        bool bad = false;
-        while (w < nck && cum > args.log_eps) {
-            const float2 cs = args.summ[img_slot(bos, n, w) * Hv + h];
-            cum += cs.x;
-            bad |= cs.y != 0.f;
-            ++w;
-        }
-        cend = (cum > args.log_eps || bad) ? nck : w;
+        const int w = rev_warmup_end(args.summ, bos, n, h, Hv, c1, nck, args.log_eps, lane);
+        scan = takes_scan(c0, c1, w);
+        if (w >= 0 && !scan) cend = w;
     }
-    const bool exact_end = (cend == nck);
+    const bool exact_end = (cend == nck) && !scan;  // the walk starts from dS_T
+    if constexpr (kPre) {
+        // This segment's exit adjoint is published when an earlier segment of the sequence takes
+        // the scan: the same decision, made here from the same summaries, one warp per earlier
+        // segment.
+        bool earlier_scans = false;
+        if (scan_ok && args.auto_warm) {
+            for (int j = seg - 1 - warp; j >= 0; j -= kNT / 32) {
+                const int c0j = min(nck, j * args.L), c1j = min(nck, (j + 1) * args.L);
+                if (c1j < nck &&
+                    takes_scan(c0j, c1j, rev_warmup_end(args.summ, bos, n, h, Hv, c1j, nck, args.log_eps, lane)))
+                    earlier_scans = true;
+            }
+        }
+        if (!__syncthreads_or(earlier_scans) && !scan) {  // nothing to do in the pre-pass
+            // (the pre-pass is a programmatic dependent of the state replay, which it does not read:
+            // it completes only after the replay has, so that the reverse walk finds both done)
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            return;
+        }
+    }
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
@@ -375,21 +462,41 @@ __global__ void __launch_bounds__(kNT, 1)
         }
     };
     bool pre = false;  // dO, H and v of this chunk were fetched during the previous one
+    // the scan's flag of segment j of this (sequence, value head), and its records
+    auto flag_of = [&](int j) { return args.scan_flags + blockIdx.x + (int64_t)(seg - j) * Hv; };
+    auto rec_of = [&](int j) {
+        return args.scan_rec + (int64_t)(blockIdx.x + (int64_t)(seg - j) * Hv) * 4 * dk * dv;
+    };
+    // this CTA's records: [exit adjoint, M, B, entry adjoint], each [dk][dv]
+    float* rec = args.scan_rec ? rec_of(seg) : nullptr;
 
     // ===================== reverse walk with the state adjoint =====================
-    {  // dH^T <- dS_T at the sequence end, zero at the start of a reverse warm-up
-        const float* dst = b.dST ? b.dST + ((int64_t)n * Hv + h) * dk * dv : nullptr;
+    // One walk over the chunks (from dS_T, or from zero at the start of a reverse warm-up), or the
+    // three walks of the adjoint scan over the own chunks: the fold B (from dH = 0), the fold M
+    // (from dH = I with dO = 0), then the walk with the gradients from the scanned exit adjoint.
+    {  // the walk's start: dS_T at the sequence end; for a segment that takes the scan, the entry
+       // adjoint that the pre-pass recorded; zero at the start of a reverse warm-up (or of a fold)
+        const float* src = nullptr;
+        if (exact_end && b.dST) src = b.dST + ((int64_t)n * Hv + h) * dk * dv;
+        if (!kPre && scan) src = rec + (int64_t)3 * dk * dv;
         float v[64];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) v[e] = (dst && exact_end) ? dst[(int64_t)(64 * hh + e) * dv + m] : 0.f;
+        for (int e = 0; e < 64; ++e) v[e] = src ? src[(int64_t)(64 * hh + e) * dv + m] : 0.f;
         tmem_st64(tl + cH + 64 * hh, v);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
-    prefetch_gates(cend - 1);
-    for (int c = cend - 1; c >= c0 && ok; --c) {
-        const bool emit = c < c1;  // own chunk (else: reverse warm-up, the dH chain only)
+    // Walks: the reverse walk with the gradients (one walk); in the pre-pass the walk to the exit
+    // adjoint (one walk, the dH chain only) or the two fold walks of the scan.
+    auto run_walks = [&](auto walks) {
+    constexpr int npass = decltype(walks)::value;
+    for (int walk = 0; walk < npass && ok; ++walk) {
+    const bool with_do = !(kPre && npass == 2 && walk == 1);  // the fold M has dO = 0
+    const int ctop = scan ? c1 : cend;  // a walk covers chunks ctop - 1 down to c0
+    prefetch_gates(ctop - 1);
+    for (int c = ctop - 1; c >= c0 && ok; --c) {
+        const bool emit = !kPre && c < c1;  // own chunk (else: warm-up or fold, the dH chain only)
         const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
         const int64_t t0 = bos + (int64_t)c * kChunk;
         // this chunk's inputs (first of all: their latency overlaps the copies and gates below)
@@ -454,10 +561,12 @@ __global__ void __launch_bounds__(kNT, 1)
         }
         if (tid == kIss2) {
             tc_fence_after();
+            if (with_do) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)  // dO^T P (R4): A = dO^T MN-major, B = P MN-major (N = s)
-                mma_bf16_ss(tmem + cR4, desc_sw128(sb + bDO + j * 2048, 16384, 1024),
-                            desc_sw128(sb + bP + j * 2048, 8192, 1024), id_mm64, j > 0);
+                for (int j = 0; j < 4; ++j)  // dO^T P (R4): A = dO^T MN-major, B = P MN-major (N = s)
+                    mma_bf16_ss(tmem + cR4, desc_sw128(sb + bDO + j * 2048, 16384, 1024),
+                                desc_sw128(sb + bP + j * 2048, 8192, 1024), id_mm64, j > 0);
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {  // dH^T K^T (R5): A = bf16 dH^T (TMEM), B = K rows
                 const uint32_t koff = (j >> 2) * 16384 + (j & 3) * 32;
@@ -496,6 +605,10 @@ __global__ void __launch_bounds__(kNT, 1)
                // half reads fp32 columns this half overwrites, hence the barrier
                 float w32[32];
                 tmem_ld32x2(tl + cR4 + 32 * hh, v, tl + cR5 + 32 * hh, w32);
+                if (!with_do) {  // the fold of the linear part: dO = 0 (R4 was not written)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                }
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -547,10 +660,12 @@ __global__ void __launch_bounds__(kNT, 1)
         }
         if (tid == kIss2) {
             tc_fence_after();
+            if (with_do) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)  // dH^T += dO^T Qg   (B = Qg MN-major, N = dk)
-                mma_bf16_ss(tmem + cH, desc_sw128(sb + bDO + j * 2048, 16384, 1024),
-                            desc_sw128(sb + bBw + j * 2048, 8192, 1024), id_mm128, 1);
+                for (int j = 0; j < 4; ++j)  // dH^T += dO^T Qg   (B = Qg MN-major, N = dk)
+                    mma_bf16_ss(tmem + cH, desc_sw128(sb + bDO + j * 2048, 16384, 1024),
+                                desc_sw128(sb + bBw + j * 2048, 8192, 1024), id_mm128, 1);
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j)  // dH^T += dU^T (-W)  (B = -W^T rows, K-major)
                 mma_bf16_ts(tmem + cH, tmem + cR5 + 8 * j, desc_sw128(sb + bWt + j * 32, 16, 1024),
@@ -829,11 +944,165 @@ __global__ void __launch_bounds__(kNT, 1)
         __syncthreads();
         tc_fence_after();
     }
+    if (kPre && npass == 2 && ok && walk == 0) {
+        // the fold B ended (from dH = 0): recorded [dk][dv] (thread (m, hh): dv column m, dk rows
+        // [64 hh, 64 hh + 64)); the fold M starts from dH = I
+        {
+            float* dst = rec + (int64_t)2 * dk * dv + m;
+            float v[64];
+            tmem_ld64(tl + cH + 64 * hh, v);
+#pragma unroll
+            for (int e = 0; e < 64; ++e) dst[(int64_t)(64 * hh + e) * dv] = v[e];
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e] = (64 * hh + e == m) ? 1.f : 0.f;
+            tmem_st64(tl + cH + 64 * hh, v);
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    }  // walks
+    };
+    if constexpr (kPre) {
+        if (!scan) {
+            run_walks(std::integral_constant<int, 1>{});  // to the exit adjoint, from the usual start
+            if (ok) {
+                float* ex = rec + m;
+                float v[64];
+                tmem_ld64(tl + cH + 64 * hh, v);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) ex[(int64_t)(64 * hh + e) * dv] = v[e];
+                __threadfence();
+                __syncthreads();
+                if (tid == 0) rflag_release(flag_of(seg), 2);
+            }
+        } else {
+            run_walks(std::integral_constant<int, 2>{});  // the folds B and M
+        }
+        if (scan && ok) {
+            // the fold M (from dH = I with dO = 0), recorded; the fold is published
+            {
+                float* dst = rec + (int64_t)dk * dv + m;
+                float v[64];
+                tmem_ld64(tl + cH + 64 * hh, v);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) dst[(int64_t)(64 * hh + e) * dv] = v[e];
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) rflag_release(flag_of(seg), 1);
+            // look forward: the nearest later segment whose exit adjoint is published (one that does
+            // not take the scan publishes it after its walk; one that does, after its combination)
+            int* lb = (int*)red;
+            if (tid == 0) {
+                int i = seg + 1;
+                bool okl = true;
+                const uint64_t tw = globaltimer();
+                while (true) {
+                    if (i >= segs_n) {  // no later segment published an exit adjoint
+                        okl = false;
+                        break;
+                    }
+                    const int f = rflag_acquire(flag_of(i));
+                    if (f == 2) break;
+                    if (f == 1) {
+                        ++i;
+                        continue;
+                    }
+                    if (globaltimer() - tw > kWaitTimeoutNs) {
+                        okl = false;
+                        break;
+                    }
+                    __nanosleep(128);
+                }
+                lb[0] = i;
+                lb[1] = okl ? 1 : 0;
+            }
+            __syncthreads();
+            ok = lb[1] != 0;
+            const int base = lb[0];
+            __syncthreads();  // lb has been read
+            // X = the exit adjoint of segment base carried through the folds of segments base - 1 ..
+            // seg, X <- M X + B, in fp32: before the own fold X is this segment's entry adjoint,
+            // recorded for its reverse walk; after it, its exit adjoint.  Thread (m, hh) forms rows
+            // [64 hh, 64 hh + 64) of column m from the whole column (both halves of TMEM lane m);
+            // the exit record holds the new rows until both threads of the lane have read the old
+            // column.
+            float v[64];
+            if (ok) {
+                (void)rflag_acquire(flag_of(base));  // this thread's own acquire of the records it reads
+                const float* ex = rec_of(base) + m;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) v[e] = ex[(int64_t)(64 * hh + e) * dv];
+            } else {  // the look-forward timed out (reported): a zero entry adjoint, not garbage
+#pragma unroll
+                for (int e = 0; e < 64; ++e) v[e] = 0.f;
+                float* st = rec + (int64_t)3 * dk * dv + m;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) st[(int64_t)(64 * hh + e) * dv] = 0.f;
+            }
+            tmem_st64(tl + cH + 64 * hh, v);
+            float* tmp = rec + m;
+            for (int t = base - 1; t >= seg && ok; --t) {
+                (void)rflag_acquire(flag_of(t));
+                tc_fence_before();
+                __syncthreads();  // the column is complete in TMEM
+                tc_fence_after();
+                if (t == seg) {  // the entry adjoint of this segment's reverse walk
+                    float* st = rec + (int64_t)3 * dk * dv + m;
+                    tmem_ld64(tl + cH + 64 * hh, v);
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) st[(int64_t)(64 * hh + e) * dv] = v[e];
+                }
+                const float* Mt = rec_of(t) + dk * dv;
+                const float* Bt = Mt + dk * dv;
+#pragma unroll 1
+                for (int ib = 0; ib < 2; ++ib) {  // rows 64 hh + 32 ib .. + 31 of the new column
+                    const int r0 = 64 * hh + 32 * ib;
+                    float acc[32];
+#pragma unroll
+                    for (int ii = 0; ii < 32; ++ii) acc[ii] = Bt[(int64_t)(r0 + ii) * dv + m];
+#pragma unroll 1
+                    for (int lb4 = 0; lb4 < 4; ++lb4) {  // times X rows 32 lb4 .. 32 lb4 + 31
+                        float x[32];
+                        tmem_ld32(tl + cH + 32 * lb4, x);
+#pragma unroll 4
+                        for (int ii = 0; ii < 32; ++ii) {
+                            const float4* mr = reinterpret_cast<const float4*>(Mt + (int64_t)(r0 + ii) * dk + 32 * lb4);
+                            float sacc = 0.f;
+#pragma unroll
+                            for (int l4 = 0; l4 < 8; ++l4) {
+                                const float4 mv = mr[l4];
+                                sacc += mv.x * x[4 * l4] + mv.y * x[4 * l4 + 1] + mv.z * x[4 * l4 + 2] +
+                                        mv.w * x[4 * l4 + 3];
+                            }
+                            acc[ii] += sacc;
+                        }
+                    }
+#pragma unroll
+                    for (int ii = 0; ii < 32; ++ii) tmp[(int64_t)(r0 + ii) * dv] = acc[ii];
+                }
+                tc_fence_before();
+                __syncthreads();  // both threads of every lane have read the old column
+                tc_fence_after();
+#pragma unroll
+                for (int e = 0; e < 64; ++e) v[e] = tmp[(int64_t)(64 * hh + e) * dv];
+                tmem_st64(tl + cH + 64 * hh, v);
+            }
+            if (ok) {  // the exit adjoint M X + B is in the exit record: published
+                __threadfence();
+                __syncthreads();
+                if (tid == 0) rflag_release(flag_of(seg), 2);
+            }
+        }
+    } else {
+        run_walks(std::integral_constant<int, 1>{});
+    }
     if (!ok && pre) {  // fetches for the next chunk are in flight: let them land before the CTA exits
         if (tid == 0) mbar_arrive(bar_ld);
         (void)mbar_wait(bar_ld, ph_ld);
     }
-    if (ok && b.dS0 && seg == 0) {
+    if (!kPre && ok && b.dS0 && seg == 0) {
         float* dst = b.dS0 + ((int64_t)n * Hv + h) * dk * dv + m;
         float v[64];
         tmem_ld64(tl + cH + 64 * hh, v);
@@ -847,46 +1116,101 @@ __global__ void __launch_bounds__(kNT, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemColsB);
     }
+    if constexpr (kPre) asm volatile("griddepcontrol.wait;" ::: "memory");  // see the early exit above
+}
+
+
+// The split of the reverse walks over CTAs, and whether some sequence has enough segments for the
+// adjoint scan.  A reverse warm-up chunk runs only the dH chain: about a third of a full chunk.
+struct RevSplit {
+    std::vector<int> nck;
+    SplitChoice sc;
+    bool scan;
+};
+
+RevSplit rev_split(const Problem& p, const int32_t* cu_host, int split_mode) {
+    RevSplit r;
+    r.nck = chunk_counts(p, cu_host);
+    r.sc = choose_split(r.nck, p.Hv, split_mode, sm_count(), 0.3);
+    r.scan = false;
+    for (int c : r.nck) r.scan |= segments_of(c, r.sc.L, 0) >= kRevScanMinSegs;
+    r.scan &= split_mode != 1;
+    return r;
+}
+
+// bytes of the adjoint scan's flags (one int32 per CTA, 256-aligned) and records (four fp32
+// [dk][dv] states per CTA: exit adjoint, M, B, entry adjoint)
+size_t rev_scan_flag_bytes(int64_t ctas) { return align_up((size_t)ctas * 4, 256); }
+size_t rev_scan_bytes(const RevSplit& r, const Problem& p) {
+    return r.scan ? rev_scan_flag_bytes(r.sc.ctas) + (size_t)r.sc.ctas * 4 * p.dk * p.dv * sizeof(float) : 0;
+}
+
+struct BwdLayout {
+    size_t timg, himg, dqw, dkw, scan, total;
+};
+
+// workspace: the WY outputs (T / Bw / Bu images, gate summaries, the forward scan's flags and
+// records), the replayed H^T images, (with grouped heads) fp32 dq and dk per value head, summed
+// over each group by the reduction, then the adjoint scan's flags and records
+BwdLayout bwd_layout(const Problem& p, const int32_t* cu_host, int split_mode) {
+    BwdLayout l;
+    size_t off = 0;
+    l.timg = off;
+    off = align_up(off + tc_fwd_workspace(p, cu_host, split_mode), 256);
+    l.himg = off;
+    off = align_up(off + (p.num_chunks > 0 ? (size_t)img_slots(p) * p.Hv * kHImg : 0), 256);
+    const size_t per = p.group > 1 ? sizeof(float) * (size_t)p.T_total * p.Hv * p.dk : 0;
+    l.dqw = off;
+    off = align_up(off + per, 256);
+    l.dkw = off;
+    off = align_up(off + per, 256);
+    l.scan = off;
+    off = align_up(off + (p.num_chunks > 0 ? rev_scan_bytes(rev_split(p, cu_host, split_mode), p) : 0), 256);
+    l.total = off;
+    return l;
 }
 
 }  // namespace
 
 bool tc_bwd_supported(const Problem& p) { return p.dtype == GDN_BF16 && p.dk == 128 && p.dv == 128; }
 
-// workspace: the WY outputs (T / Bw / Bu images, gate summaries), the replayed H^T images, then (with
-// grouped heads) fp32 dq and dk per value head, summed over each group by the reduction
 size_t tc_bwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode, size_t* off_himg,
                         size_t* off_timg, size_t* off_dqw, size_t* off_dkw) {
-    size_t off = 0;
-    *off_timg = off;  // the forward's workspace (WY images and summaries, the scan) for the replay
-    off = align_up(off + tc_fwd_workspace(p, cu_host, split_mode), 256);
-    *off_himg = off;
-    off = align_up(off + (p.num_chunks > 0 ? (size_t)img_slots(p) * p.Hv * kHImg : 0), 256);
-    const size_t per = p.group > 1 ? sizeof(float) * (size_t)p.T_total * p.Hv * p.dk : 0;
-    *off_dqw = off;
-    off = align_up(off + per, 256);
-    *off_dkw = off;
-    off = align_up(off + per, 256);
-    return off;
+    const BwdLayout l = bwd_layout(p, cu_host, split_mode);
+    *off_himg = l.himg;
+    *off_timg = l.timg;
+    *off_dqw = l.dqw;
+    *off_dkw = l.dkw;
+    return l.total;
 }
 
-int tc_bwd_launches(const Problem& p) { return p.num_chunks > 0 ? (p.group == 1 ? 3 : 4) : 1; }
+int tc_bwd_launches(const Problem& p, const int32_t* cu_host, int split_mode) {
+    if (p.num_chunks <= 0) return 1;
+    // WY, state replay, [adjoint scan pre-pass,] reverse walk, [dq / dk group reduction]
+    return 3 + (rev_split(p, cu_host, split_mode).scan ? 1 : 0) + (p.group > 1 ? 1 : 0);
+}
 
 gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     const BwdProblem& bp = plan.b;
     const Problem& p = bp.f;
     TcBwdArgs a;
     a.b = bp;
-    size_t oh, ot, oq, ok_;
-    tc_bwd_workspace(p, plan.cu_host, plan.split_mode, &oh, &ot, &oq, &ok_);
+    const BwdLayout l = bwd_layout(p, plan.cu_host, plan.split_mode);
+    const size_t oh = l.himg, ot = l.timg;
     a.himg = (const uint8_t*)(ws + oh);
     a.timg = (const uint8_t*)(ws + ot);
     a.summ = (const float2*)(ws + ot + wy_tc_summary_offset(p));
-    a.dqw = (float*)(ws + oq);
-    a.dkw = (float*)(ws + ok_);
-    const std::vector<int> nck = chunk_counts(p, plan.cu_host);
-    // a reverse warm-up chunk runs only the dH chain: about a third of a full chunk
-    const SplitChoice sc = choose_split(nck, p.Hv, plan.split_mode, sm_count(), 0.3);
+    a.dqw = (float*)(ws + l.dqw);
+    a.dkw = (float*)(ws + l.dkw);
+    const RevSplit rs = rev_split(p, plan.cu_host, plan.split_mode);
+    const std::vector<int>& nck = rs.nck;
+    const SplitChoice& sc = rs.sc;
+    a.scan_flags = nullptr;
+    a.scan_rec = nullptr;
+    if (rs.scan && p.num_chunks > 0) {
+        a.scan_flags = (int32_t*)(ws + l.scan);
+        a.scan_rec = (float*)(ws + l.scan + rev_scan_flag_bytes(sc.ctas));
+    }
     a.L = sc.L;
     a.fixed_segs = p.cu ? 0 : std::max(1, (nck.empty() ? 1 : (nck[0] + sc.L - 1) / sc.L));
     a.auto_warm = plan.split_mode == 1 ? 0 : 1;
@@ -896,15 +1220,37 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     if (!make_map(&mq, p.q, Tt, p.Hk) || !make_map(&mk, p.k, Tt, p.Hk) || !make_map(&mv, p.v, Tt, p.Hv) ||
         !make_map(&mdo, bp.dout, Tt, p.Hv))
         return GDN_ERR_CUDA;
-    if (cudaFuncSetAttribute(gdn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gdn_bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
+            cudaSuccess ||
+        (a.scan_rec &&
+         cudaFuncSetAttribute(gdn_bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
+             cudaSuccess))
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
     if (p.num_chunks > 0) {  // WY step + replay of the entry states
-        const gdn_status st = launch_replay_tc(p, plan.cu_host, plan.split_mode, ws + ot, (uint8_t*)(ws + oh), s);
+        // (its WY launch also clears the adjoint scan's flags)
+        const gdn_status st = launch_replay_tc(p, plan.cu_host, plan.split_mode, ws + ot, (uint8_t*)(ws + oh), s,
+                                               a.scan_flags, a.scan_flags ? (int)sc.ctas : 0);
         if (st) return st;
     }
-    gdn_bwd_tc_kernel<<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);
+    if (a.scan_rec) {
+        // the adjoint scan's pre-pass on the same grid, as a programmatic dependent of the state
+        // replay: it reads only the WY step's outputs (complete once every replay CTA has passed its
+        // own wait for them), so its CTAs may run on the SMs the replay leaves free
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)sc.ctas);
+        cfg.blockDim = dim3(kNT);
+        cfg.dynamicSmemBytes = kSmemB;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, gdn_bwd_tc_kernel<true>, mq, mk, mv, mdo, a) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    gdn_bwd_tc_kernel<false><<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     if (p.T_total > 0 && p.group > 1) return launch_bwd_reduce(bp, a.dqw, a.dkw, s);
     return GDN_OK;

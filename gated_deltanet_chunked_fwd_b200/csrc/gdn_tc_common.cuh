@@ -149,10 +149,11 @@ inline std::vector<int> chunk_counts(const Problem& p, const int32_t* cu_host) {
 
 // WY / UT step on its own: one bf16 T image per (chunk, value head), then per-chunk gate
 // summaries, into the workspace `ws`; tm_k is k's tensor map (make_map below).  It also zeroes
-// the nflags int32 flags of the state chain's affine scan (nullptr / 0: none).  The T image is
+// the nflags int32 flags of the state chain's affine scan and the nflags2 flags of the
+// backward's adjoint scan (nullptr / 0: none).  The T image is
 // written only when with_t (the backward reads it; the forward needs Bw and Bu).
 gdn_status launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, int32_t* flags, int nflags,
-                        bool with_t, cudaStream_t s);
+                        int32_t* flags2, int nflags2, bool with_t, cudaStream_t s);
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

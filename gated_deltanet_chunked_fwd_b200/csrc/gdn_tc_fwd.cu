@@ -348,6 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (known_exact && tid >= kThreadsP) load_state(true);
     // The WY step (the previous launch) must be complete before its images and summaries are read.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // A programmatic dependent launch (the backward's adjoint-scan pre-pass, which reads the WY
+    // step's outputs but not this grid's) may start once every CTA has passed the wait above.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- warm-up start (gate-driven); exact start from S0 when seg == 0.  The WY step left,
     // per chunk, its summed log decay and whether some token breaks 0 <= beta |k|^2 <= 2.
@@ -964,7 +967,7 @@ int tc_fwd_launches(const Problem& p) { return (p.num_chunks > 0 ? 1 : 0) + 1; }
 
 // The WY kernel, then the fused kernel (forward, or replay of the states when himg != nullptr)
 gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int split_mode, char* ws,
-                              uint8_t* himg, cudaStream_t s) {
+                              uint8_t* himg, cudaStream_t s, int32_t* rflags = nullptr, int nrflags = 0) {
     // all host-side preparation first, so that the two launches follow each other directly
     TcArgs a;
     a.p = p;
@@ -998,7 +1001,8 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
     const gdn_status st =
-        launch_wy_tc(p, mk, (uint8_t*)ws, a.scan_flags, a.scan_flags ? (int)sc.ctas : 0, himg != nullptr, s);
+        launch_wy_tc(p, mk, (uint8_t*)ws, a.scan_flags, a.scan_flags ? (int)sc.ctas : 0, rflags, nrflags,
+                     himg != nullptr, s);
     if (st) return st;
     // Programmatic dependent launch: the fused kernel may start while the WY kernel drains; it
     // sets up and loads S0 for exact segments, then waits (griddepcontrol.wait) for the WY
@@ -1023,11 +1027,11 @@ gdn_status launch_fwd_tc(const FwdPlan& plan, char* ws, cudaStream_t s) {
 }
 
 gdn_status launch_replay_tc(const Problem& p, const int32_t* cu_host, int split_mode, char* ws,
-                            uint8_t* himg, cudaStream_t s) {
+                            uint8_t* himg, cudaStream_t s, int32_t* rflags, int nrflags) {
     Problem q = p;  // states only: no o, no S_T
     q.o = nullptr;
     q.ST = nullptr;
-    return launch_fwd_tc_impl(q, cu_host, split_mode, ws, himg, s);
+    return launch_fwd_tc_impl(q, cu_host, split_mode, ws, himg, s, rflags, nrflags);
 }
 
 }  // namespace gdn

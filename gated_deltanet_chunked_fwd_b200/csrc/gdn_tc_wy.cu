@@ -91,7 +91,8 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
 template <bool kGrouped>
 __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : kWyMinBlocks)
     gdn_wy_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const Problem p, uint8_t* __restrict__ timg,
-                     float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags, int with_t) {
+                     float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags,
+                     int32_t* __restrict__ flags2, int nflags2, int with_t) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -101,9 +102,14 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
     const int hk = blockIdx.y, G = kGrouped ? p.group : 1, Hv = p.Hv;
     int n = 0, c = 0;
     int64_t bos = 0, len = 0;
-    // the state chain's scan flags start at zero (CTA (x, hk) clears flags x Hv + hk G + i; the
-    // chain's CTAs are fewer than the image slots times the value heads)
-    if (tid < G && (int64_t)blockIdx.x * Hv + hk * G + tid < nflags) flags[(int64_t)blockIdx.x * Hv + hk * G + tid] = 0;
+    // the scan flags of the state chain and of the backward's reverse walks start at zero (CTA
+    // (x, hk) clears entry x Hv + hk G + i of each; both have fewer CTAs than the image slots times
+    // the value heads)
+    if (tid < G) {
+        const int64_t fi = (int64_t)blockIdx.x * Hv + hk * G + tid;
+        if (fi < nflags) flags[fi] = 0;
+        if (fi < nflags2) flags2[fi] = 0;
+    }
     const bool live = locate_slot(p, blockIdx.x, &n, &c, &bos, &len);  // CTA-uniform
     uint64_t* bar = (uint64_t*)(sm + wBar);
     uint64_t* bar_mma = bar + 1;
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
 }  // namespace
 
 gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* ws, int32_t* flags, int nflags,
-                            bool with_t, cudaStream_t s) {
+                            int32_t* flags2, int nflags2, bool with_t, cudaStream_t s) {
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
@@ -343,9 +349,10 @@ gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     const dim3 grid((unsigned)slots, (unsigned)p.Hk);
-    if ((int64_t)nflags > slots * p.Hv) return GDN_ERR_DEVICE;  // every flag has a CTA to clear it
+    if ((int64_t)nflags > slots * p.Hv || (int64_t)nflags2 > slots * p.Hv)
+        return GDN_ERR_DEVICE;  // every flag has a CTA to clear it
     kern<<<grid, kWyThreads, wSmemBytes, s>>>(tm_k, p, ws, (float2*)(ws + wy_tc_summary_offset(p)), flags, nflags,
-                                              with_t ? 1 : 0);
+                                              flags2, nflags2, with_t ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -177,9 +177,21 @@ def test_aliased_state_gradient_is_rejected():
 
 
 def test_tensor_core_weak_decay_affine_scan_replay():
-    """The backward's state replay with weak decay on 8192 tokens x 16 heads: segments 3-8 of each
-    head take their entry state from the affine scan (see the forward test); all six gradients
-    against the oracle adjoint."""
+    """Weak decay on 8192 tokens x 16 heads: in the state replay segments 3-8 of each head take
+    their entry state from the affine scan (see the forward test), and in the reverse walks (nine
+    15-chunk segments per head) segments 0-7 take their exit adjoint from the adjoint scan while the
+    last one first walks its chunks without gradients to publish its exit adjoint; all six
+    gradients against the oracle adjoint."""
     inp = make_inputs(1, 8192, 16, 16, 128, 128, dtype="bf16", seed=29, s0_std=0.1, g_mu=-7.0,
                       backward=True, device=DEV)
     compare(run(inp), ref(inp), TOL[inp["q"].dtype], "weak decay scan")
+
+
+def test_tensor_core_weak_decay_adjoint_scan_long_fold_chain():
+    """Weak decay on 16384 tokens x 2 heads: the reverse walks split into 64 four-chunk segments per
+    head, no reverse warm-up reaches the 2^-30 bound, and the first 63 segments of each head take
+    their exit adjoint from the adjoint scan (folds of up to 62 later segments combined); all six
+    gradients against the oracle adjoint."""
+    inp = make_inputs(1, 16384, 2, 2, 128, 128, dtype="bf16", seed=30, s0_std=0.1, g_mu=-7.0,
+                      backward=True, device=DEV)
+    compare(run(inp), ref(inp), TOL[inp["q"].dtype], "adjoint scan, long fold chain")
