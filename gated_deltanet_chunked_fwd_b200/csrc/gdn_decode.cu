@@ -11,13 +11,16 @@
 //   H_new[:, j] = exp(g) H_old[:, j] + d_j k,   o_j = exp(g) b_j + (k . q) d_j.
 // The step is bound by HBM: each state (dk x dv fp32) is read once and written once.
 //
-// Kernel: one 256-thread CTA per (sequence, value head).  Thread t owns the four state columns
-// 4 (t % 32) .. + 3 and the rows t / 32, t / 32 + 8, ... (16 rows at dk = 128), so that warp w
-// reads and writes whole 512-byte rows with 16-byte accesses.  The state goes into registers
-// with all loads in flight at once (64 KB per CTA at d = 128), the two column dots are reduced
-// over the eight row groups in shared memory, and the new state is written back from registers:
-// no thread reads a state element after another thread wrote it, so the update in place is safe
-// within a CTA, and different CTAs own different states.
+// Kernel: one 256-thread CTA per (sequence, value head, 64 state columns): the columns of H never
+// meet, so the state splits over CTAs by columns with no exchange.  Thread t owns the four
+// columns 4 (t % 16) .. + 3 of its half and the rows t / 16, t / 16 + 16, ... (8 rows at
+// dk = 128), so that half a warp reads and writes a 256-byte row piece with 16-byte accesses.
+// The state piece goes into registers with all loads in flight at once (32 KB per CTA at
+// d = 128), the two column dots are reduced over the 16 row groups in shared memory, and the new
+// state is written back from registers: no thread reads a state element after another thread
+// wrote it, so the update in place is safe, and different CTAs own different columns.  With 32
+// state registers per thread several CTAs share an SM, so one CTA's loads overlap another's
+// arithmetic and stores.
 #include "gdn_dtype.cuh"
 #include "gdn_internal.cuh"
 
@@ -25,8 +28,10 @@ namespace gdn {
 namespace {
 
 constexpr int kDecThreads = 256;
-constexpr int kRowGroups = kDecThreads / 32;           // 8
-constexpr int kRowsPerThread = kMaxHead / kRowGroups;  // 16
+constexpr int kDecCols = 64;                           // state columns per CTA
+constexpr int kColGroups = kDecCols / 4;               // 16 (four columns per thread)
+constexpr int kRowGroups = kDecThreads / kColGroups;   // 16
+constexpr int kRowsPerThread = kMaxHead / kRowGroups;  // 8
 
 struct DecodeArgs {
     int N, Hk, Hv, dk, dv, group, num_slots;
@@ -43,25 +48,26 @@ struct DecodeArgs {
 
 template <typename Tin>
 __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArgs a) {
-    __shared__ float sk[kMaxHead], sq[kMaxHead], sv[kMaxHead];
-    __shared__ float4 pa[kRowGroups][32], pb[kRowGroups][32];  // partial column dots
-    __shared__ float colA[kMaxHead], colB[kMaxHead];
+    __shared__ float sk[kMaxHead], sq[kMaxHead], sv[kDecCols];
+    __shared__ float4 pa[kRowGroups][kColGroups], pb[kRowGroups][kColGroups];  // partial column dots
+    __shared__ float colA[kDecCols], colB[kDecCols];
     __shared__ float skq;
     const int h = blockIdx.x % a.Hv, n = blockIdx.x / a.Hv, hk = h / a.group;
-    const int t = threadIdx.x, cg = t & 31, rg = t >> 5;
+    const int t = threadIdx.x, cg = t % kColGroups, rg = t / kColGroups;
     const int dk = a.dk, dv = a.dv;
+    const int jb = kDecCols * blockIdx.y;  // this CTA's first state column
     const int slot = a.idx ? a.idx[n] : n;
-    Tin* o = (Tin*)a.o + ((int64_t)n * a.Hv + h) * dv;
+    Tin* o = (Tin*)a.o + ((int64_t)n * a.Hv + h) * dv + jb;
     if (slot < 0) {  // padding entry of a batch: no state, zero output
-        if (t < dv) store_as(o + t, 0.f);
+        if (t < kDecCols && jb + t < dv) store_as(o + t, 0.f);
         return;
     }
     if (slot >= a.num_slots) {
         if (t == 0) report(a.status, GDN_ERR_DEVICE);
         return;
     }
-    float* S = a.S + ((int64_t)slot * a.Hv + h) * dk * dv;
-    const bool col_ok = 4 * cg < dv;
+    float* S = a.S + ((int64_t)slot * a.Hv + h) * dk * dv + jb;
+    const bool col_ok = jb + 4 * cg < dv;
 
     // ---- the state into registers: every load issued before any is used
     float4 Hr[kRowsPerThread];
@@ -73,21 +79,21 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArg
     }
     const Tin* qp = (const Tin*)a.q + ((int64_t)n * a.Hk + hk) * dk;
     const Tin* kp = (const Tin*)a.k + ((int64_t)n * a.Hk + hk) * dk;
-    const Tin* vp = (const Tin*)a.v + ((int64_t)n * a.Hv + h) * dv;
+    const Tin* vp = (const Tin*)a.v + ((int64_t)n * a.Hv + h) * dv + jb;
     if (t < dk) {
         sk[t] = to_f(kp[t]);
         sq[t] = to_f(qp[t]);
     }
-    if (t < dv) sv[t] = to_f(vp[t]);
+    if (t < kDecCols && jb + t < dv) sv[t] = to_f(vp[t]);
     const float eg = expf(a.g[(int64_t)n * a.Hv + h]);
     const float bt = a.beta[(int64_t)n * a.Hv + h];
     __syncthreads();
-    if (rg == 0) {  // k . q by warp 0
+    if (t < 32) {  // k . q by warp 0
         float s = 0.f;
-        for (int i = cg; i < dk; i += 32) s += sk[i] * sq[i];
+        for (int i = t; i < dk; i += 32) s += sk[i] * sq[i];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (cg == 0) skq = s;
+        if (t == 0) skq = s;
     }
 
     // ---- column dots a_j = H[:, j] . k and b_j = H[:, j] . q over this thread's rows
@@ -102,16 +108,17 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArg
     pa[rg][cg] = da;
     pb[rg][cg] = db;
     __syncthreads();
-    if (t < 2 * 32) {  // sum the eight row groups: threads 0-31 for a, 32-63 for b
-        const int c = t & 31;
+    if (t < 2 * kColGroups) {  // sum the row groups: threads 0-15 for a, 16-31 for b
+        const int c = t % kColGroups;
+        const bool is_a = t < kColGroups;
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int g8 = 0; g8 < kRowGroups; ++g8) {
-            const float4 x = t < 32 ? pa[g8][c] : pb[g8][c];
+        for (int g = 0; g < kRowGroups; ++g) {
+            const float4 x = is_a ? pa[g][c] : pb[g][c];
             s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
         }
-        float* dst = t < 32 ? colA : colB;
-        if (4 * c < dv) *reinterpret_cast<float4*>(dst + 4 * c) = s;
+        float* dst = is_a ? colA : colB;
+        if (jb + 4 * c < dv) *reinterpret_cast<float4*>(dst + 4 * c) = s;
     }
     __syncthreads();
 
@@ -188,7 +195,7 @@ gdn_status launch_decode(const gdn_decode_args* a, cudaStream_t s) {
     d.idx = a->state_indices;
     d.o = a->o;
     d.status = a->dev_status;
-    const unsigned grid = (unsigned)((int64_t)a->N * a->Hv);
+    const dim3 grid((unsigned)((int64_t)a->N * a->Hv), (unsigned)((a->dv + kDecCols - 1) / kDecCols));
     if (a->dtype == GDN_BF16)
         gdn_decode_kernel<__nv_bfloat16><<<grid, kDecThreads, 0, s>>>(d);
     else
