@@ -195,3 +195,13 @@ def test_tensor_core_weak_decay_adjoint_scan_long_fold_chain():
     inp = make_inputs(1, 16384, 2, 2, 128, 128, dtype="bf16", seed=30, s0_std=0.1, g_mu=-7.0,
                       backward=True, device=DEV)
     compare(run(inp), ref(inp), TOL[inp["q"].dtype], "adjoint scan, long fold chain")
+
+
+def test_tensor_core_weak_decay_varlen_gqa_mixed_scan():
+    """Weak decay on a ragged batch with grouped heads (2 q/k heads, 4 value heads): the long
+    sequences split into enough reverse segments for the adjoint scan, the short ones replay or
+    run unsplit, and the empty and one-token sequences have no chunk to scan; all six gradients
+    against the oracle adjoint."""
+    inp = make_inputs(1, 0, 2, 4, 128, 128, dtype="bf16", seed=31, s0_std=0.1, g_mu=-7.0,
+                      backward=True, lengths=[3000, 200, 0, 9000, 64, 1, 2500], device=DEV)
+    compare(run(inp), ref(inp), TOL[inp["q"].dtype], "weak decay varlen GQA")

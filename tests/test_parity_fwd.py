@@ -241,3 +241,14 @@ def test_tensor_core_weak_decay_affine_scan():
     check_every_unit(inp, o, ST)
     o1, ST1 = run(inp, GDN_FLAG_SPLIT_OFF)
     assert rel_l2(o, o1) < 5e-3 and rel_l2(ST, ST1) < 5e-3
+
+
+def test_tensor_core_weak_decay_varlen_gqa_mixed_scan():
+    """Weak decay on a ragged batch with grouped heads (2 q/k heads, 4 value heads): sequences long
+    enough to split into several segments take the affine scan for their later segments, short
+    ones run unsplit, and the empty and one-token sequences have nothing to scan; every unit
+    against the oracle."""
+    inp = make_inputs(1, 0, 2, 4, 128, 128, dtype="bf16", seed=32, s0_std=0.1, g_mu=-7.0,
+                      lengths=[3000, 200, 0, 9000, 64, 1, 2500], device=DEV)
+    o, ST = run(inp)
+    check_every_unit(inp, o, ST)
