@@ -17,7 +17,9 @@ with states stored transposed, H = S^T of shape [dk, dv].
 
 Pins (``tests/test_oracle_pins.py``): invariants of the rule, closed forms,
 a hand-worked example (``tests/golden/``), torch autograd and finite
-differences for the backward.  No function here is "parity unpinned".
+differences for the backward; closed forms and central differences for the
+optional input preprocessing and its backward.  No function here is "parity
+unpinned".
 """
 from __future__ import annotations
 
@@ -97,13 +99,75 @@ def _pack(q, k, v, beta, g, cu_seqlens):
     return (B, T, cu) + tuple(flat(x) for x in (q, k, v, beta, g))
 
 
-def fwd(q, k, v, beta, g, cu_seqlens=None, initial_state=None, output_final_state=True):
+# ---- optional input preprocessing ------------------------------------------------------
+# Models usually feed the layer from raw projections: q and k are L2-normalised over the head
+# dimension, beta is a sigmoid of a logit and the log decay g is minus a softplus.  The pages
+# do not describe this step (it is a reading: the plainest form of each map, as the input
+# generator applies it); with qk_l2norm / gate_logits the layer takes the raw values and
+# applies the maps itself, and the backward returns gradients with respect to the raw values.
+
+L2_EPS = 1e-6  # x / max(||x||, L2_EPS)
+
+
+def _l2norm(x):
+    n = np.sqrt((x * x).sum(-1, keepdims=True))
+    return x / np.maximum(n, L2_EPS), n
+
+
+def _sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _neg_softplus(x):
+    """-log(1 + exp(x)), in the form that neither overflows nor loses small values."""
+    return -(np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x))))
+
+
+def preprocess(q, k, beta, g, qk_l2norm=False, gate_logits=False):
+    """(q, k, beta, g) as the rule consumes them, from raw inputs (float64):
+    q, k -> x / max(||x||_2, 1e-6) over the head dimension when qk_l2norm;
+    beta -> sigmoid(beta) and g -> -softplus(g) = -log(1 + exp(g)) when gate_logits."""
+    q, k, beta, g = (_f64(x) for x in (q, k, beta, g))
+    if qk_l2norm:
+        q, k = _l2norm(q)[0], _l2norm(k)[0]
+    if gate_logits:
+        beta, g = _sigmoid(beta), _neg_softplus(g)
+    return q, k, beta, g
+
+
+def preprocess_bwd(q, k, beta, g, dq, dk, dbeta, dg, qk_l2norm=False, gate_logits=False):
+    """Gradients with respect to the raw (q, k, beta, g) from those with respect to the
+    preprocessed values (chain rule of the maps above):
+      y = x / ||x||:             dx = (dy - y (y . dy)) / ||x||    (dx = dy / 1e-6 below the clamp)
+      beta = sigmoid(b):         db = dbeta beta (1 - beta)
+      g = -softplus(a):          da = -dg sigmoid(a)"""
+    q, k, beta, g, dq, dk, dbeta, dg = (_f64(x) for x in (q, k, beta, g, dq, dk, dbeta, dg))
+    if qk_l2norm:
+        out = []
+        for x, dy in ((q, dq), (k, dk)):
+            y, n = _l2norm(x)
+            c = np.maximum(n, L2_EPS)
+            proj = dy - y * (y * dy).sum(-1, keepdims=True)
+            out.append(np.where(n > L2_EPS, proj, dy) / c)
+        dq, dk = out
+    if gate_logits:
+        s = _sigmoid(beta)
+        dbeta = dbeta * s * (1.0 - s)
+        dg = -dg * _sigmoid(g)
+    return dq, dk, dbeta, dg
+
+
+def fwd(q, k, v, beta, g, cu_seqlens=None, initial_state=None, output_final_state=True,
+        qk_l2norm=False, gate_logits=False):
     """o, S_T = rule applied token by token (float64).
 
     q, k: [B, T, Hk, dk]; v: [B, T, Hv, dv]; beta, g: [B, T, Hv];
     cu_seqlens: optional [N+1] offsets (B must be 1); initial_state: [N, Hv, dk, dv]
     (the transposed state H = S^T).  Returns numpy float64 (o [B,T,Hv,dv], S_T or None).
+    qk_l2norm / gate_logits: the inputs are raw and go through `preprocess` first.
     """
+    if qk_l2norm or gate_logits:
+        q, k, beta, g = preprocess(q, k, beta, g, qk_l2norm, gate_logits)
     B, T, cu, qf, kf, vf, bf, gf = _pack(q, k, v, beta, g, cu_seqlens)
     N = cu.shape[0] - 1
     Hk, dk = qf.shape[1], qf.shape[2]
@@ -121,12 +185,20 @@ def fwd(q, k, v, beta, g, cu_seqlens=None, initial_state=None, output_final_stat
     return o.reshape(B, T, Hv, dv), ST
 
 
-def bwd(q, k, v, beta, g, do, cu_seqlens=None, initial_state=None, dST=None):
+def bwd(q, k, v, beta, g, do, cu_seqlens=None, initial_state=None, dST=None, qk_l2norm=False,
+        gate_logits=False):
     """Gradients of <do, o> + <dST, S_T> w.r.t. (q, k, v, beta, g, S0), float64.
 
     Returns numpy arrays (dq, dk, dv, dbeta, dg, dS0) with the input shapes;
-    dq/dk are summed over the value heads that share a q/k head.
+    dq/dk are summed over the value heads that share a q/k head.  With qk_l2norm /
+    gate_logits the inputs are raw and the gradients are with respect to them.
     """
+    if qk_l2norm or gate_logits:
+        raw = (q, k, beta, g)
+        q, k, beta, g = preprocess(q, k, beta, g, qk_l2norm, gate_logits)
+        res = bwd(q, k, v, beta, g, do, cu_seqlens, initial_state, dST)
+        dq, dk_, db, dg_ = preprocess_bwd(*raw, res[0], res[1], res[3], res[4], qk_l2norm, gate_logits)
+        return dq, dk_, res[2], db, dg_, res[5]
     B, T, cu, qf, kf, vf, bf, gf = _pack(q, k, v, beta, g, cu_seqlens)
     N = cu.shape[0] - 1
     Hk, dk = qf.shape[1], qf.shape[2]

@@ -258,3 +258,93 @@ def test_backward_central_differences():
             fd = (L(plus) - L(minus)) / (2 * h)
             an = float((grads[i] * d).sum())
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (i, fd, an)
+
+
+# ---- optional input preprocessing (q / k L2-normalisation, beta and g from logits) ----
+
+def test_preprocess_closed_forms():
+    """sigmoid(0) = 1/2, -softplus(0) = -log 2, -softplus tends to -a for large a and to -e^a for
+    very negative a; normalised vectors have unit norm, and a vector below the clamp is divided
+    by 1e-6."""
+    q = np.array([[[[3.0, 4.0]], [[1e-8, 0.0]]]])        # [B=1, T=2, H=1, d=2]
+    k = np.array([[[[0.0, -2.0]], [[6.0, 8.0]]]])
+    b = np.array([[[0.0], [np.log(3.0)]]])                  # sigmoid: 1/2, 3/4
+    a = np.array([[[0.0], [40.0]]])
+    qh, kh, bt, g = oracle.preprocess(q, k, b, a, qk_l2norm=True, gate_logits=True)
+    np.testing.assert_allclose(qh[0, 0, 0], [0.6, 0.8], rtol=1e-15)
+    np.testing.assert_allclose(qh[0, 1, 0], [1e-2, 0.0], rtol=1e-12)
+    np.testing.assert_allclose(kh[0, :, 0], [[0.0, -1.0], [0.6, 0.8]], rtol=1e-15)
+    np.testing.assert_allclose(bt[0, :, 0], [0.5, 0.75], rtol=1e-15)
+    assert g[0, 0, 0] == pytest.approx(-np.log(2.0), rel=1e-15)
+    assert g[0, 1, 0] == pytest.approx(-40.0 - np.exp(-40.0), rel=1e-15)
+    assert oracle.preprocess(q, k, b, np.array([[[-50.0], [0.0]]]), gate_logits=True)[3][0, 0, 0] == \
+        pytest.approx(-np.exp(-50.0), rel=1e-12)
+    # flags off: the inputs come back unchanged
+    for x, y in zip(oracle.preprocess(q, k, b, a), (q, k, b, a)):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_preprocess_backward_central_differences():
+    """The chain rule of the preprocessing maps against central differences of a random linear
+    functional of their outputs (a dropped projection term, a sign or a sigmoid' slip fails)."""
+    rs = np.random.default_rng(21)
+    q = rnd((1, 7, 2, 5), rs)
+    k = rnd((1, 7, 2, 5), rs)
+    q[0, 3, 1] *= 1e-9  # one vector below the clamp
+    b = rnd((1, 7, 3), rs) * 3
+    a = rnd((1, 7, 3), rs) * 3
+    w = [rnd(x.shape, rs) for x in (q, k, b, a)]
+
+    def L(xs):
+        ys = oracle.preprocess(*xs, qk_l2norm=True, gate_logits=True)
+        return float(sum((y * wi).sum() for y, wi in zip(ys, w)))
+
+    an = oracle.preprocess_bwd(q, k, b, a, *w, qk_l2norm=True, gate_logits=True)
+    base = [q, k, b, a]
+    for i in range(4):
+        for _ in range(3):
+            d = rnd(base[i].shape, rs)
+            h = 1e-7 if i < 2 else 1e-6
+            plus = [x.copy() for x in base]
+            minus = [x.copy() for x in base]
+            plus[i] += h * d
+            minus[i] -= h * d
+            if i == 0:  # keep the clamped vector clamped: perturb it within its size
+                plus[0][0, 3, 1] = q[0, 3, 1] * (1 + 1e-3 * d[0, 3, 1, 0])
+                minus[0][0, 3, 1] = q[0, 3, 1] * (1 - 1e-3 * d[0, 3, 1, 0])
+                dd = d.copy()
+                dd[0, 3, 1] = q[0, 3, 1] * 1e-3 * d[0, 3, 1, 0] / h
+            else:
+                dd = d
+            fd = (L(plus) - L(minus)) / (2 * h)
+            val = float((an[i] * dd).sum())
+            assert abs(fd - val) <= 1e-5 * max(1.0, abs(val)), (i, fd, val)
+
+
+def test_layer_with_preprocessing_central_differences():
+    """bwd(..., qk_l2norm, gate_logits) is the gradient of fwd(..., qk_l2norm, gate_logits) with
+    respect to the raw q, k, beta and g (directional central differences through the layer)."""
+    rs = np.random.default_rng(22)
+    q, k, v, beta, g, S0 = small_case(rs, T=9, Hk=1, Hv=2, dk=4, dv=3)
+    q, k = q * 3, k * 0.5              # raw, not unit vectors
+    beta, g = beta * 4 - 2, g * 3 + 1  # logits of either sign
+    do = rnd((1, 9, 2, 3), rs)
+    dST = rnd((1, 2, 4, 3), rs)
+    kw = dict(qk_l2norm=True, gate_logits=True)
+    grads = oracle.bwd(q, k, v, beta, g, do, initial_state=S0, dST=dST, **kw)
+
+    def L(xs):
+        o, ST = oracle.fwd(*xs[:5], initial_state=xs[5], **kw)
+        return float((o * do).sum() + (ST * dST).sum())
+
+    base = [q, k, v, beta, g, S0]
+    h = 1e-6
+    for i in range(6):
+        d = rnd(base[i].shape, rs)
+        plus = [x.copy() for x in base]
+        minus = [x.copy() for x in base]
+        plus[i] += h * d
+        minus[i] -= h * d
+        fd = (L(plus) - L(minus)) / (2 * h)
+        an = float((grads[i] * d).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (i, fd, an)
