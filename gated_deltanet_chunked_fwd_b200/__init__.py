@@ -19,12 +19,13 @@ from typing import Optional
 import torch
 
 from . import _abi
-from ._abi import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE, GDN_FLAG_SPLIT_OFF, GdnBwdArgs,
-                   GdnDecodeArgs, GdnError, GdnFwdArgs)
+from ._abi import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE, GDN_FLAG_SPLIT_OFF,
+                   GdnBwdArgs, GdnDecodeArgs, GdnError, GdnFwdArgs)
 
 __all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_size",
            "gdn_chunk_bwd_workspace_size", "chunk_fwd", "chunk_bwd", "GdnError",
-           "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE", "decode_step"]
+           "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE", "GDN_FLAG_GATE_LOGITS",
+           "decode_step"]
 
 _DT = {torch.float32: _abi.GDN_F32, torch.bfloat16: _abi.GDN_BF16}
 
@@ -177,7 +178,7 @@ def gdn_chunk_bwd(q, k, v, beta, g, do, cu_seqlens=None, initial_state=None, dST
     return dq, dk, dv, dbeta, dg, dS0
 
 
-def _decode_args(q, k, v, beta, g, state, state_indices, o):
+def _decode_args(q, k, v, beta, g, state, state_indices, o, flags=0):
     if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[0] != q.shape[0]:
         raise ValueError("q, k must be [N, Hk, dk] and v [N, Hv, dv]")
     if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
@@ -201,20 +202,21 @@ def _decode_args(q, k, v, beta, g, state, state_indices, o):
         raise ValueError(f"state must be float32 [slots, {Hv}, {dk}, {dv}]")
     a.q, a.k, a.v, a.beta, a.g = _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g)
     a.S, a.state_indices, a.o = _ptr(state), _ptr(state_indices), _ptr(o)
+    a.flags = flags
     return a
 
 
-def gdn_decode_step(q, k, v, beta, g, state, state_indices=None, *, out=None,
+def gdn_decode_step(q, k, v, beta, g, state, state_indices=None, *, out=None, flags: int = 0,
                     check_device_status: bool = False):
     """One decode token per sequence; updates ``state`` in place and returns o [N, Hv, dv].
 
     q, k: [N, Hk, dk]; v: [N, Hv, dv] (one dtype, fp32 or bf16); beta, g: [N, Hv] fp32;
     state: fp32 [N, Hv, dk, dv] (H = S^T, as S_T of gdn_chunk_fwd), or a pool of slots
     [num_slots, Hv, dk, dv] indexed by ``state_indices`` (int32 [N] on the device; negative
-    = skip that sequence).
+    = skip that sequence).  flags: GDN_FLAG_GATE_LOGITS (beta, g as logits) or 0.
     """
     o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
-    a = _decode_args(q, k, v, beta, g, state, state_indices, o)
+    a = _decode_args(q, k, v, beta, g, state, state_indices, o, flags)
     st = _dev_status(q.device, check_device_status)
     a.dev_status = _ptr(st)
     _check("gdn_decode_step", _abi.lib().gdn_decode_step(ctypes.byref(a), _stream(q.device)))

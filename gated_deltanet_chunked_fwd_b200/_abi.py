@@ -18,6 +18,7 @@ GDN_F32, GDN_BF16 = 0, 1
 GDN_FLAG_SPLIT_OFF = 1 << 0
 GDN_FLAG_SPLIT_FORCE = 1 << 1
 GDN_FLAG_PORTABLE = 1 << 2
+GDN_FLAG_GATE_LOGITS = 1 << 3
 
 STATUS = {
     0: "GDN_OK",

@@ -44,6 +44,7 @@ struct DecodeArgs {
     const int32_t* idx;
     void* o;
     int32_t* status;
+    int gate_logits;  // GDN_FLAG_GATE_LOGITS
 };
 
 template <typename Tin>
@@ -85,8 +86,8 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArg
         sq[t] = to_f(qp[t]);
     }
     if (t < kDecCols && jb + t < dv) sv[t] = to_f(vp[t]);
-    const float eg = expf(a.g[(int64_t)n * a.Hv + h]);
-    const float bt = a.beta[(int64_t)n * a.Hv + h];
+    const float eg = expf(gate_g(a.g[(int64_t)n * a.Hv + h], a.gate_logits));
+    const float bt = gate_beta(a.beta[(int64_t)n * a.Hv + h], a.gate_logits);
     __syncthreads();
     if (t < 32) {  // k . q by warp 0
         float s = 0.f;
@@ -195,6 +196,7 @@ gdn_status launch_decode(const gdn_decode_args* a, cudaStream_t s) {
     d.idx = a->state_indices;
     d.o = a->o;
     d.status = a->dev_status;
+    d.gate_logits = (a->flags & GDN_FLAG_GATE_LOGITS) ? 1 : 0;
     const dim3 grid((unsigned)((int64_t)a->N * a->Hv), (unsigned)((a->dv + kDecCols - 1) / kDecCols));
     if (a->dtype == GDN_BF16)
         gdn_decode_kernel<__nv_bfloat16><<<grid, kDecThreads, 0, s>>>(d);

@@ -41,7 +41,25 @@ struct Problem {
     float* ST;
     int32_t* status;
     int64_t num_chunks;  // sum over sequences of ceil(len / 64)
+    int gate_logits;     // GDN_FLAG_GATE_LOGITS: beta and g hold logits / pre-activations
 };
+
+// Raw gates (GDN_FLAG_GATE_LOGITS): beta = sigmoid(b) and g = -softplus(a) = -log(1 + e^a), the
+// latter as -(max(a, 0) + log1p(e^-|a|)), which neither overflows nor loses small values; the
+// identity maps otherwise.  Padding tokens keep their plain zeros (callers apply the maps to
+// loaded values only).
+__device__ __forceinline__ float gate_beta(float b, int logits) { return logits ? 1.f / (1.f + expf(-b)) : b; }
+__device__ __forceinline__ float gate_g(float a, int logits) {
+    return logits ? -(fmaxf(a, 0.f) + log1pf(expf(-fabsf(a)))) : a;
+}
+// Chain rule back to the raw gates: d/db sigmoid(b) = beta (1 - beta) (from the mapped beta),
+// d/da -softplus(a) = -sigmoid(a).
+__device__ __forceinline__ float gate_beta_grad(float dbeta, float beta, int logits) {
+    return logits ? dbeta * beta * (1.f - beta) : dbeta;
+}
+__device__ __forceinline__ float gate_g_grad(float dg, float a, int logits) {
+    return logits ? -dg / (1.f + expf(-a)) : dg;
+}
 
 // Per-chunk lookup built on the device from cu_seqlens (or arithmetic).
 struct ChunkTable {

@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(256) simt_bwd_chunk_kernel(BwdProblem b, Chunk
     }
     if (threadIdx.x < kChunk) {
         const int r = threadIdx.x;
-        bs[r] = r < n ? p.beta[(int64_t)(t0 + r) * p.Hv + h] : 0.f;
+        bs[r] = r < n ? gate_beta(p.beta[(int64_t)(t0 + r) * p.Hv + h], p.gate_logits) : 0.f;
         gs[r] = gam[ch * kChunk + r];
         dgam[r] = 0.f;
     }
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(256) simt_bwd_chunk_kernel(BwdProblem b, Chunk
         acc3 = warp_sum(acc3);
         acc4 = warp_sum(acc4);
         if (lane == 0) {
-            b.dbeta[(int64_t)(t0 + r) * p.Hv + h] = acc1 + Gs[r] * acc2 + acc3;
+            b.dbeta[(int64_t)(t0 + r) * p.Hv + h] = gate_beta_grad(acc1 + Gs[r] * acc2 + acc3, bs[r], p.gate_logits);
             dgam[r] += bG[r] * acc2 + acc4;
         }
     }
@@ -377,7 +377,8 @@ __global__ void __launch_bounds__(256) simt_bwd_chunk_kernel(BwdProblem b, Chunk
         float run = 0.f;
         for (int r = n - 1; r >= 0; --r) {  // dg = reverse in-chunk cumsum
             run += dgam[r];
-            b.dg[(int64_t)(t0 + r) * p.Hv + h] = run;
+            b.dg[(int64_t)(t0 + r) * p.Hv + h] =
+                gate_g_grad(run, p.gate_logits ? p.g[(int64_t)(t0 + r) * p.Hv + h] : 0.f, p.gate_logits);
         }
     }
 }

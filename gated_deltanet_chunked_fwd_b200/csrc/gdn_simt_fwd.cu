@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(256) simt_wy_kernel(Problem p, ChunkTable ct, 
     }
     if (threadIdx.x < kChunk) {
         const int r = threadIdx.x;
-        bs[r] = r < n ? p.beta[(int64_t)(t0 + r) * p.Hv + h] : 0.f;
-        gs[r] = r < n ? p.g[(int64_t)(t0 + r) * p.Hv + h] : 0.f;  // padding: g = 0
+        bs[r] = r < n ? gate_beta(p.beta[(int64_t)(t0 + r) * p.Hv + h], p.gate_logits) : 0.f;
+        gs[r] = r < n ? gate_g(p.g[(int64_t)(t0 + r) * p.Hv + h], p.gate_logits) : 0.f;  // padding: g = 0
     }
     __syncthreads();
     if (threadIdx.x == 0) {

@@ -355,8 +355,8 @@ __global__ void __launch_bounds__(kNT, 1)
         if (tid < 64 && c >= c0) {
             const int64_t t0 = bos + (int64_t)c * kChunk;
             const int lcc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-            nxt_g = tid < lcc ? p.g[(t0 + tid) * Hv + h] : 0.f;  // padding: g = 0, beta = 0
-            nxt_b = tid < lcc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
+            nxt_g = tid < lcc ? gate_g(p.g[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;  // padding: g = 0,
+            nxt_b = tid < lcc ? gate_beta(p.beta[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;  // beta = 0
         }
     };
     auto gates = [&](int c, int lc) -> bool {
@@ -935,10 +935,12 @@ __global__ void __launch_bounds__(kNT, 1)
                     const float y = __shfl_down_sync(0xffffffffu, suf, o);
                     if (lane + o < 32) suf += y;
                 }
-                if (r0 < lc) b.dg[(t0 + r0) * Hv + h] = suf;
-                if (r0 + 1 < lc) b.dg[(t0 + r0 + 1) * Hv + h] = suf - x0;
+                if (r0 < lc) b.dg[(t0 + r0) * Hv + h] = gate_g_grad(suf, p.gate_logits ? p.g[(t0 + r0) * Hv + h] : 0.f, p.gate_logits);
+                if (r0 + 1 < lc)
+                    b.dg[(t0 + r0 + 1) * Hv + h] =
+                        gate_g_grad(suf - x0, p.gate_logits ? p.g[(t0 + r0 + 1) * Hv + h] : 0.f, p.gate_logits);
             }
-            if (tid < lc) b.dbeta[(t0 + tid) * Hv + h] = acc_b[tid];
+            if (tid < lc) b.dbeta[(t0 + tid) * Hv + h] = gate_beta_grad(acc_b[tid], vbeta[tid], p.gate_logits);
         }
         tc_fence_before();
         __syncthreads();

@@ -441,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lcc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
             const int r0 = 2 * lane;
-            gx0 = r0 < lcc ? p.g[(t0 + r0) * Hv + h] : 0.f;  // padding: g = 0
-            gx1 = r0 + 1 < lcc ? p.g[(t0 + r0 + 1) * Hv + h] : 0.f;
+            gx0 = r0 < lcc ? gate_g(p.g[(t0 + r0) * Hv + h], p.gate_logits) : 0.f;  // padding: g = 0
+            gx1 = r0 + 1 < lcc ? gate_g(p.g[(t0 + r0 + 1) * Hv + h], p.gate_logits) : 0.f;
         };
         // vectors of chunk kk (buffer kk mod 4; beta enters through the Bw / Bu images): gamma =
         // cumsum g, Gam = exp(gamma), decay to the chunk end exp(gamma_n - gamma), the E factors

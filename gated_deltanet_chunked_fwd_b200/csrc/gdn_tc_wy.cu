@@ -137,8 +137,8 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
     }
     float xg = 0.f, bt = 0.f;
     auto load_gates = [&](int h) {
-        xg = tid < lc ? p.g[(t0 + tid) * Hv + h] : 0.f;  // lc <= 64
-        bt = tid < lc ? p.beta[(t0 + tid) * Hv + h] : 0.f;
+        xg = tid < lc ? gate_g(p.g[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;  // lc <= 64
+        bt = tid < lc ? gate_beta(p.beta[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;
     };
     load_gates(hk * G);
     tc_fence_before();

@@ -84,6 +84,11 @@ typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
                                           kernels cover on the CUDA-core kernels instead
                                           (fp32 arithmetic), to cross-check the two; not
                                           a second backend for production use          */
+#define GDN_FLAG_GATE_LOGITS (1u << 3) /* raw gates: beta holds logits b, beta =
+                                          sigmoid(b); g holds pre-activations a, g =
+                                          -softplus(a) = -log(1 + e^a); the backward's
+                                          dbeta and dg are then gradients with respect to
+                                          b and a.  Forward, backward and decode step.  */
 
 /* Arguments of the forward.  struct_size = sizeof(gdn_fwd_args),
  * abi_version = GDN_ABI_VERSION. */
@@ -218,7 +223,7 @@ typedef struct gdn_decode_args {
     int32_t Hk, Hv;    /* q/k heads, value heads (Hv % Hk == 0, contiguous groups)   */
     int32_t dk, dv;    /* head dims, 1..128, dv a multiple of 4                      */
     int32_t num_slots; /* states in S when state_indices != NULL (else N)            */
-    uint32_t flags;    /* reserved, 0                                                */
+    uint32_t flags;    /* GDN_FLAG_GATE_LOGITS or 0; other bits are ignored         */
     const void* q;     /* [N, Hk, dk] dtype                                          */
     const void* k;     /* [N, Hk, dk] dtype                                          */
     const void* v;     /* [N, Hv, dv] dtype                                          */

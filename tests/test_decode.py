@@ -109,3 +109,24 @@ def test_decode_workload_every_unit():
     inp1 = {"q": x["q"], "v": x["v"]}
     assert_every_unit(o[:, None], o_ref, inp1, "tok", 1e-2, "o")
     assert_every_unit(S, S_ref, inp1, "state", 1e-5, "S")
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_gate_logits(dt):
+    """GDN_FLAG_GATE_LOGITS in the decode step: beta and g as logits / pre-activations."""
+    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_GATE_LOGITS
+
+    x = decode_inputs(6, 2, 4, 128, 128, dt, seed=37)
+    gen = torch.Generator().manual_seed(38)
+    x["beta"] = (2.0 * torch.randn(x["beta"].shape, generator=gen)).to(DEV)
+    x["g"] = (torch.randn(x["g"].shape, generator=gen) + 1.0).to(DEV)
+    S = x["initial_state"].clone()
+    c = cpu(x)
+    o_ref, S_ref = oracle.fwd(c["q"], c["k"], c["v"], c["beta"], c["g"], initial_state=S.cpu(),
+                              gate_logits=True)
+    c0 = {n: x[n][:, 0].contiguous() for n in ("q", "k", "v", "beta", "g")}
+    o = gdn_decode_step(c0["q"], c0["k"], c0["v"], c0["beta"], c0["g"], S, flags=GDN_FLAG_GATE_LOGITS,
+                        check_device_status=True)
+    torch.cuda.synchronize()
+    assert rel_l2(o, o_ref[:, 0]) < TOL[x["q"].dtype]
+    assert rel_l2(S, S_ref) < 1e-5

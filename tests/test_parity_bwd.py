@@ -205,3 +205,19 @@ def test_tensor_core_weak_decay_varlen_gqa_mixed_scan():
     inp = make_inputs(1, 0, 2, 4, 128, 128, dtype="bf16", seed=31, s0_std=0.1, g_mu=-7.0,
                       backward=True, lengths=[3000, 200, 0, 9000, 64, 1, 2500], device=DEV)
     compare(run(inp), ref(inp), TOL[inp["q"].dtype], "weak decay varlen GQA")
+
+
+@pytest.mark.parametrize("dt,flags", [("bf16", 0), ("fp32", 0)], ids=["tensor-core", "cuda-core-fp32"])
+def test_gate_logits(dt, flags):
+    """GDN_FLAG_GATE_LOGITS: dbeta and dg are gradients with respect to the raw logits /
+    pre-activations; all six gradients against the oracle's chain rule, ragged, grouped heads."""
+    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_GATE_LOGITS
+    from tests.test_parity_fwd import with_raw_gates
+
+    d = 128 if dt == "bf16" else 64
+    inp = with_raw_gates(make_inputs(1, 0, 2, 4, d, d, dtype=dt, seed=35, s0_std=0.1, backward=True,
+                                     lengths=[300, 1, 0, 129], device=DEV), 36)
+    x = cpu(inp)
+    refs = oracle.bwd(x["q"], x["k"], x["v"], x["beta"], x["g"], x["do"], cu_seqlens=x["cu_seqlens"],
+                      initial_state=x["initial_state"], dST=x["dST"], gate_logits=True)
+    compare(run(inp, flags | GDN_FLAG_GATE_LOGITS), refs, TOL[inp["q"].dtype], "gate logits")

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE,
+from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE,
                                              GDN_FLAG_SPLIT_OFF, gdn_chunk_fwd)
 from gated_deltanet_chunked_fwd_b200.inputs import make_inputs, make_workload
 from tests._helpers import TOL, assert_every_unit, cpu, rel_l2
@@ -252,3 +252,30 @@ def test_tensor_core_weak_decay_varlen_gqa_mixed_scan():
                       lengths=[3000, 200, 0, 9000, 64, 1, 2500], device=DEV)
     o, ST = run(inp)
     check_every_unit(inp, o, ST)
+
+
+def with_raw_gates(inp, seed):
+    """Replace beta and g by raw values for GDN_FLAG_GATE_LOGITS: logits of either sign for beta
+    and pre-activations around +1 for g (the layer applies sigmoid and -softplus itself)."""
+    gen = torch.Generator().manual_seed(seed)
+    shape = inp["beta"].shape
+    inp = dict(inp)
+    inp["beta"] = (2.0 * torch.randn(shape, generator=gen)).to(inp["beta"].device)
+    inp["g"] = (torch.randn(shape, generator=gen) + 1.0).to(inp["g"].device)
+    return inp
+
+
+@pytest.mark.parametrize("dt,flags", [("bf16", 0), ("fp32", 0), ("bf16", GDN_FLAG_PORTABLE)],
+                         ids=["tensor-core", "cuda-core-fp32", "cuda-core-bf16"])
+def test_gate_logits(dt, flags):
+    """GDN_FLAG_GATE_LOGITS: beta and g arrive as logits / pre-activations, ragged sequences,
+    grouped heads; o and S_T against the oracle applying sigmoid and -softplus in float64."""
+    d = 128 if dt == "bf16" else 64
+    inp = with_raw_gates(make_inputs(1, 0, 2, 4, d, d, dtype=dt, seed=33, s0_std=0.1,
+                                     lengths=[300, 1, 0, 129], device=DEV), 34)
+    o, ST = run(inp, flags | GDN_FLAG_GATE_LOGITS)
+    x = cpu(inp)
+    o_ref, ST_ref = oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["g"], cu_seqlens=x["cu_seqlens"],
+                               initial_state=x["initial_state"], gate_logits=True)
+    tol = TOL[inp["q"].dtype]
+    assert rel_l2(o, o_ref) < tol and rel_l2(ST, ST_ref) < tol, (rel_l2(o, o_ref), rel_l2(ST, ST_ref))
