@@ -19,12 +19,13 @@ from typing import Optional
 import torch
 
 from . import _abi
-from ._abi import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE, GDN_FLAG_SPLIT_OFF,
-                   GdnBwdArgs, GdnDecodeArgs, GdnError, GdnFwdArgs)
+from ._abi import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_QK_L2NORM, GDN_FLAG_SPLIT_FORCE,
+                   GDN_FLAG_SPLIT_OFF, GdnBwdArgs, GdnDecodeArgs, GdnError, GdnFwdArgs)
 
 __all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_size",
            "gdn_chunk_bwd_workspace_size", "chunk_fwd", "chunk_bwd", "GdnError",
            "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE", "GDN_FLAG_GATE_LOGITS",
+           "GDN_FLAG_QK_L2NORM",
            "decode_step"]
 
 _DT = {torch.float32: _abi.GDN_F32, torch.bfloat16: _abi.GDN_BF16}
@@ -213,7 +214,8 @@ def gdn_decode_step(q, k, v, beta, g, state, state_indices=None, *, out=None, fl
     q, k: [N, Hk, dk]; v: [N, Hv, dv] (one dtype, fp32 or bf16); beta, g: [N, Hv] fp32;
     state: fp32 [N, Hv, dk, dv] (H = S^T, as S_T of gdn_chunk_fwd), or a pool of slots
     [num_slots, Hv, dk, dv] indexed by ``state_indices`` (int32 [N] on the device; negative
-    = skip that sequence).  flags: GDN_FLAG_GATE_LOGITS (beta, g as logits) or 0.
+    = skip that sequence).  flags: GDN_FLAG_GATE_LOGITS (beta, g as logits), GDN_FLAG_QK_L2NORM
+    (raw q, k normalised inside) or 0.
     """
     o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
     a = _decode_args(q, k, v, beta, g, state, state_indices, o, flags)

@@ -19,6 +19,7 @@ GDN_FLAG_SPLIT_OFF = 1 << 0
 GDN_FLAG_SPLIT_FORCE = 1 << 1
 GDN_FLAG_PORTABLE = 1 << 2
 GDN_FLAG_GATE_LOGITS = 1 << 3
+GDN_FLAG_QK_L2NORM = 1 << 4
 
 STATUS = {
     0: "GDN_OK",

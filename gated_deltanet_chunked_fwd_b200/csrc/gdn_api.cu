@@ -86,6 +86,7 @@ gdn_status plan_fwd(const gdn_fwd_args* a, FwdPlan* plan) {
     p.ST = a->ST;
     p.status = a->dev_status;
     p.gate_logits = (a->flags & GDN_FLAG_GATE_LOGITS) ? 1 : 0;
+    p.qk_norm = (a->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     plan->cu_host = a->cu_seqlens ? a->cu_seqlens_host : nullptr;
     plan->split_mode = (a->flags & GDN_FLAG_SPLIT_OFF) ? 1 : (a->flags & GDN_FLAG_SPLIT_FORCE) ? 2 : 0;
     plan->use_tc = !(a->flags & GDN_FLAG_PORTABLE) && tc_fwd_supported(p);
@@ -143,6 +144,7 @@ gdn_status plan_bwd(const gdn_bwd_args* a, BwdPlan* plan) {
     p.S0 = a->S0;
     p.status = a->dev_status;
     p.gate_logits = (a->flags & GDN_FLAG_GATE_LOGITS) ? 1 : 0;
+    p.qk_norm = (a->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     BwdProblem& b = plan->b;
     b.dout = a->dout;
     b.dST = a->dST;

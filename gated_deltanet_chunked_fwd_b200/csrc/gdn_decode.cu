@@ -45,6 +45,7 @@ struct DecodeArgs {
     void* o;
     int32_t* status;
     int gate_logits;  // GDN_FLAG_GATE_LOGITS
+    int qk_norm;      // GDN_FLAG_QK_L2NORM
 };
 
 template <typename Tin>
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArg
     __shared__ float sk[kMaxHead], sq[kMaxHead], sv[kDecCols];
     __shared__ float4 pa[kRowGroups][kColGroups], pb[kRowGroups][kColGroups];  // partial column dots
     __shared__ float colA[kDecCols], colB[kDecCols];
-    __shared__ float skq;
+    __shared__ float skq, sinv[2];
     const int h = blockIdx.x % a.Hv, n = blockIdx.x / a.Hv, hk = h / a.group;
     const int t = threadIdx.x, cg = t % kColGroups, rg = t / kColGroups;
     const int dk = a.dk, dv = a.dv;
@@ -89,6 +90,22 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArg
     const float eg = expf(gate_g(a.g[(int64_t)n * a.Hv + h], a.gate_logits));
     const float bt = gate_beta(a.beta[(int64_t)n * a.Hv + h], a.gate_logits);
     __syncthreads();
+    if (a.qk_norm) {  // raw k and q: x / max(|x|, eps), norms by warps 0 (k) and 1 (q)
+        if (t < 64) {
+            const float* x = t < 32 ? sk : sq;
+            float ss = 0.f;
+            for (int i = t & 31; i < dk; i += 32) ss += x[i] * x[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            if ((t & 31) == 0) sinv[t >> 5] = 1.f / fmaxf(sqrtf(ss), kL2Eps);
+        }
+        __syncthreads();
+        if (t < dk) {
+            sk[t] *= sinv[0];
+            sq[t] *= sinv[1];
+        }
+        __syncthreads();
+    }
     if (t < 32) {  // k . q by warp 0
         float s = 0.f;
         for (int i = t; i < dk; i += 32) s += sk[i] * sq[i];
@@ -197,6 +214,7 @@ gdn_status launch_decode(const gdn_decode_args* a, cudaStream_t s) {
     d.o = a->o;
     d.status = a->dev_status;
     d.gate_logits = (a->flags & GDN_FLAG_GATE_LOGITS) ? 1 : 0;
+    d.qk_norm = (a->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     const dim3 grid((unsigned)((int64_t)a->N * a->Hv), (unsigned)((a->dv + kDecCols - 1) / kDecCols));
     if (a->dtype == GDN_BF16)
         gdn_decode_kernel<__nv_bfloat16><<<grid, kDecThreads, 0, s>>>(d);

@@ -42,7 +42,24 @@ struct Problem {
     int32_t* status;
     int64_t num_chunks;  // sum over sequences of ceil(len / 64)
     int gate_logits;     // GDN_FLAG_GATE_LOGITS: beta and g hold logits / pre-activations
+    int qk_norm;         // GDN_FLAG_QK_L2NORM: q and k rows are normalised before use
 };
+
+constexpr float kL2Eps = 1e-6f;  // GDN_FLAG_QK_L2NORM: x / max(|x|_2, kL2Eps)
+
+// GDN_FLAG_QK_L2NORM on rows held in shared memory as fp32: X[r][0, dk) <- X[r] / max(|X[r]|_2,
+// kL2Eps) for r < rows, one warp per row; the caller synchronises before and after.
+__device__ __forceinline__ void l2norm_rows_smem(float* X, int rows, int dk) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int r = warp; r < rows; r += nw) {
+        float ss = 0.f;
+        for (int i = lane; i < dk; i += 32) ss += X[r * dk + i] * X[r * dk + i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = 1.f / fmaxf(sqrtf(ss), kL2Eps);
+        for (int i = lane; i < dk; i += 32) X[r * dk + i] *= inv;
+    }
+}
 
 // Raw gates (GDN_FLAG_GATE_LOGITS): beta = sigmoid(b) and g = -softplus(a) = -log(1 + e^a), the
 // latter as -(max(a, 0) + log1p(e^-|a|)), which neither overflows nor loses small values; the

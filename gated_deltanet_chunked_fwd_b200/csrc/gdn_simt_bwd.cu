@@ -74,6 +74,11 @@ __global__ void __launch_bounds__(256) simt_bwd_dstate_kernel(BwdProblem b, Chun
             Qs[idx] = r < len ? to_f(qp[off]) : 0.f;
             Ks[idx] = r < len ? to_f(kp[off]) : 0.f;
         }
+        if (p.qk_norm) {  // raw q and k rows: normalised before use
+            __syncthreads();
+            l2norm_rows_smem(Qs, kChunk, dk);
+            l2norm_rows_smem(Ks, kChunk, dk);
+        }
         for (int idx = threadIdx.x; idx < kChunk * kSliceB; idx += blockDim.x) {
             const int r = idx / kSliceB, jj = idx % kSliceB;
             dOs[idx] = (r < len && jj < sw) ? to_f(dop[((int64_t)(t0 + r) * p.Hv + h) * dv + j0 + jj])
@@ -193,6 +198,11 @@ __global__ void __launch_bounds__(256) simt_bwd_chunk_kernel(BwdProblem b, Chunk
         dgam[r] = 0.f;
     }
     __syncthreads();
+    if (p.qk_norm) {  // raw q and k rows: normalised before use
+        l2norm_rows_smem(Qs, kChunk, dk);
+        l2norm_rows_smem(Ks, kChunk, dk);
+        __syncthreads();
+    }
     const float gl = gs[kChunk - 1];
     if (threadIdx.x < kChunk) {
         const int r = threadIdx.x;
@@ -405,6 +415,68 @@ __global__ void simt_bwd_reduce_kernel(BwdProblem b, const float* dqw, const flo
     }
 }
 
+// GDN_FLAG_QK_L2NORM: one warp per (token, q/k head) row sums the per-value-head gradients of
+// the normalised row y = x / max(|x|, eps) over the group, then takes them back to the raw row x:
+// dx = (dy - y (y . dy)) / max(|x|, eps), or dy / eps where the clamp holds (dk <= 128: four
+// elements per lane).
+template <typename Tin>
+__global__ void simt_bwd_reduce_l2norm_kernel(BwdProblem b, const float* dqw, const float* dkw) {
+    const Problem& p = b.f;
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = p.T_total * p.Hk;
+    const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t row = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; row < rows; row += wstride) {
+        const int hk = (int)(row % p.Hk);
+        const int64_t t = row / p.Hk;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            const float* w = which ? dkw : dqw;
+            const Tin* x = (const Tin*)(which ? p.k : p.q) + row * p.dk;
+            Tin* out = (Tin*)(which ? b.dk : b.dq) + row * p.dk;
+            float dy[4], xv[4], ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = lane + 32 * e;
+                float acc = 0.f, xi = 0.f;
+                if (i < p.dk) {
+                    for (int gg = 0; gg < p.group; ++gg) acc += w[(t * p.Hv + hk * p.group + gg) * p.dk + i];
+                    xi = to_f(x[i]);
+                }
+                dy[e] = acc;
+                xv[e] = xi;
+                ss += xi * xi;
+            }
+            ss = warp_sum(ss);
+            const float nrm = sqrtf(ss), inv = 1.f / fmaxf(nrm, kL2Eps);
+            float dot = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dot += xv[e] * inv * dy[e];
+            dot = warp_sum(dot);
+            const bool clamped = !(nrm > kL2Eps);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = lane + 32 * e;
+                if (i < p.dk) store_as(out + i, clamped ? dy[e] * inv : (dy[e] - xv[e] * inv * dot) * inv);
+            }
+        }
+    }
+}
+
+template <typename Tin>
+static gdn_status launch_reduce_t(const BwdProblem& b, const float* dqw, const float* dkw, cudaStream_t s) {
+    const Problem& p = b.f;
+    if (p.qk_norm) {
+        const int64_t rows = p.T_total * p.Hk;
+        const int blocks = (int)std::min<int64_t>((rows + 7) / 8, 148 * 16);  // 8 rows per block
+        simt_bwd_reduce_l2norm_kernel<Tin><<<blocks, 256, 0, s>>>(b, dqw, dkw);
+    } else {
+        const int64_t total = p.T_total * p.Hk * p.dk;
+        const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
+        simt_bwd_reduce_kernel<Tin><<<blocks, 256, 0, s>>>(b, dqw, dkw);
+    }
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 template <typename K>
 static gdn_status set_smem_b(K kernel, size_t bytes) {
     if (bytes > 48 * 1024 &&
@@ -453,23 +525,15 @@ static gdn_status launch_bwd_typed(const BwdPlan& plan, char* ws, cudaStream_t s
         dim3 grid((unsigned)nc, p.Hv);
         simt_bwd_chunk_kernel<Tin><<<grid, 256, smem, s>>>(b, ct, U, gam, Hc, dHc, dU, dqw, dkw);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-        const int64_t total = p.T_total * p.Hk * p.dk;
-        const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
-        simt_bwd_reduce_kernel<Tin><<<blocks, 256, 0, s>>>(b, dqw, dkw);
-        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+        const gdn_status st = launch_reduce_t<Tin>(b, dqw, dkw, s);
+        if (st) return st;
     }
     return GDN_OK;
 }
 
 gdn_status launch_bwd_reduce(const BwdProblem& b, const float* dqw, const float* dkw, cudaStream_t s) {
-    const Problem& p = b.f;
-    const int64_t total = p.T_total * p.Hk * p.dk;
-    const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
-    if (p.dtype == GDN_BF16)
-        simt_bwd_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(b, dqw, dkw);
-    else
-        simt_bwd_reduce_kernel<float><<<blocks, 256, 0, s>>>(b, dqw, dkw);
-    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return b.f.dtype == GDN_BF16 ? launch_reduce_t<__nv_bfloat16>(b, dqw, dkw, s)
+                                 : launch_reduce_t<float>(b, dqw, dkw, s);
 }
 
 gdn_status launch_bwd_simt(const BwdPlan& plan, char* ws, cudaStream_t s) {

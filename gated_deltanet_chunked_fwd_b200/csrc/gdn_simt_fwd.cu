@@ -97,6 +97,10 @@ __global__ void __launch_bounds__(256) simt_wy_kernel(Problem p, ChunkTable ct, 
         gs[r] = r < n ? gate_g(p.g[(int64_t)(t0 + r) * p.Hv + h], p.gate_logits) : 0.f;  // padding: g = 0
     }
     __syncthreads();
+    if (p.qk_norm) {  // raw k rows: normalised before use
+        l2norm_rows_smem(Ks, kChunk, dk);
+        __syncthreads();
+    }
     if (threadIdx.x == 0) {
         float acc = 0.f;
         for (int r = 0; r < kChunk; ++r) {
@@ -182,10 +186,24 @@ __global__ void __launch_bounds__(256) simt_state_kernel(Problem p, ChunkTable c
         if (threadIdx.x < kChunk) gs[threadIdx.x] = gam[ch * kChunk + threadIdx.x];
         __syncthreads();
         const float gl = gs[kChunk - 1];
-        for (int idx = threadIdx.x; idx < kChunk * dk; idx += blockDim.x) {
-            const int r = idx / dk, i = idx % dk;
-            Kd[idx] = r < len ? to_f(kp[((int64_t)(t0 + r) * p.Hk + hk) * dk + i]) * expf(gl - gs[r])
-                              : 0.f;
+        if (!p.qk_norm) {
+            for (int idx = threadIdx.x; idx < kChunk * dk; idx += blockDim.x) {
+                const int r = idx / dk, i = idx % dk;
+                Kd[idx] = r < len ? to_f(kp[((int64_t)(t0 + r) * p.Hk + hk) * dk + i]) * expf(gl - gs[r])
+                                  : 0.f;
+            }
+        } else {  // raw k rows: normalised, then scaled by the decay
+            for (int idx = threadIdx.x; idx < kChunk * dk; idx += blockDim.x) {
+                const int r = idx / dk, i = idx % dk;
+                Kd[idx] = r < len ? to_f(kp[((int64_t)(t0 + r) * p.Hk + hk) * dk + i]) : 0.f;
+            }
+            __syncthreads();
+            l2norm_rows_smem(Kd, kChunk, dk);
+            __syncthreads();
+            for (int idx = threadIdx.x; idx < kChunk * dk; idx += blockDim.x) {
+                const int r = idx / dk;
+                Kd[idx] *= r < len ? expf(gl - gs[r]) : 0.f;
+            }
         }
         float* Hcc = Hc + ch * dk * dv;
         for (int idx = threadIdx.x; idx < dk * kSlice; idx += blockDim.x) {
@@ -248,6 +266,11 @@ __global__ void __launch_bounds__(256) simt_output_kernel(Problem p, ChunkTable 
     const int64_t ch = (int64_t)c * p.Hv + h;
     if (threadIdx.x < kChunk) gs[threadIdx.x] = gam[ch * kChunk + threadIdx.x];
     __syncthreads();
+    if (p.qk_norm) {  // raw q and k rows: normalised before use
+        l2norm_rows_smem(Qs, kChunk, dk);
+        l2norm_rows_smem(Ks, kChunk, dk);
+        __syncthreads();
+    }
     for (int idx = threadIdx.x; idx < kChunk * kChunk; idx += blockDim.x) {
         const int r = idx / kChunk, s = idx % kChunk;
         float v = 0.f;

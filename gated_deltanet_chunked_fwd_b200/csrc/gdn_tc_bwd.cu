@@ -6,7 +6,8 @@
 // gate summaries), the fused forward kernel in replay mode (the bf16 entry state H^T of every
 // chunk, as a ready-to-use 128-byte-swizzled shared-memory image), in sequences of at least four
 // segments the adjoint scan's pre-pass (this kernel with kPre), this reverse kernel, and with
-// grouped value heads the reduction of dq / dk over each group.  The reverse kernel runs one CTA per (sequence, value head, segment of
+// grouped value heads (or GDN_FLAG_QK_L2NORM) the reduction of dq / dk over each group (and the
+// chain rule of the q / k normalisation).  The reverse kernel runs one CTA per (sequence, value head, segment of
 // chunks), 256 threads: the two warps of each TMEM lane quarter share its lanes (thread <-> MMA
 // row) and split each row's columns, or tokens, in halves.  A segment walks its chunks
 // backwards with the state adjoint dH (fp32, TMEM).  Its exit adjoint comes from a reverse
@@ -528,6 +529,8 @@ __global__ void __launch_bounds__(kNT, 1)
         ok = __syncthreads_and(mbar_wait(bar_ld, ph_ld));
         ph_ld ^= 1;
         if (!ok) break;
+        if (p.qk_norm)  // raw q and k rows (0-63 q, 64-127 k): normalised in place first
+            l2norm_row_sw128(sm + bQK, 16384, tid >> 1, tid & 1);
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
@@ -852,7 +855,7 @@ __global__ void __launch_bounds__(kNT, 1)
                 const uint8_t* qtile = sm + bQK + (i >> 6) * 16384;
                 // without grouped heads dq / dk go out directly (bf16); else per value head (fp32)
                 // for the reduction over the group
-                const bool direct = p.group == 1;
+                const bool direct = p.group == 1 && !p.qk_norm;
                 float* dqp = args.dqw + (t0 * Hv + h) * dk + i;
                 float* dkp = args.dkw + (t0 * Hv + h) * dk + i;
                 __nv_bfloat16* dqb = (__nv_bfloat16*)b.dq + (t0 * Hv + h) * dk + i;
@@ -1161,7 +1164,9 @@ BwdLayout bwd_layout(const Problem& p, const int32_t* cu_host, int split_mode) {
     off = align_up(off + tc_fwd_workspace(p, cu_host, split_mode), 256);
     l.himg = off;
     off = align_up(off + (p.num_chunks > 0 ? (size_t)img_slots(p) * p.Hv * kHImg : 0), 256);
-    const size_t per = p.group > 1 ? sizeof(float) * (size_t)p.T_total * p.Hv * p.dk : 0;
+    // per-value-head fp32 dq / dk: summed over grouped heads, or taken through the chain rule of
+    // the q / k normalisation, by the reduction kernel
+    const size_t per = (p.group > 1 || p.qk_norm) ? sizeof(float) * (size_t)p.T_total * p.Hv * p.dk : 0;
     l.dqw = off;
     off = align_up(off + per, 256);
     l.dkw = off;
@@ -1189,7 +1194,7 @@ size_t tc_bwd_workspace(const Problem& p, const int32_t* cu_host, int split_mode
 int tc_bwd_launches(const Problem& p, const int32_t* cu_host, int split_mode) {
     if (p.num_chunks <= 0) return 1;
     // WY, state replay, [adjoint scan pre-pass,] reverse walk, [dq / dk group reduction]
-    return 3 + (rev_split(p, cu_host, split_mode).scan ? 1 : 0) + (p.group > 1 ? 1 : 0);
+    return 3 + (rev_split(p, cu_host, split_mode).scan ? 1 : 0) + ((p.group > 1 || p.qk_norm) ? 1 : 0);
 }
 
 gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
@@ -1254,7 +1259,7 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     }
     gdn_bwd_tc_kernel<false><<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    if (p.T_total > 0 && p.group > 1) return launch_bwd_reduce(bp, a.dqw, a.dkw, s);
+    if (p.T_total > 0 && (p.group > 1 || p.qk_norm)) return launch_bwd_reduce(bp, a.dqw, a.dkw, s);
     return GDN_OK;
 }
 

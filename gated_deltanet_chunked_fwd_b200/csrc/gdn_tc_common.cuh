@@ -87,6 +87,40 @@ __device__ __forceinline__ int as_idx(int r, int s) { return r * 64 + ((((s >> 2
 // Multi-SM split of the chunk chains (host side): chunks per sequence, and the segment length L
 // that minimises the estimated makespan (waves of CTAs x chunk steps per CTA, a warm-up chunk
 // counted as warm_cost steps).  split_mode: 0 auto, 1 off (one segment per sequence), 2 force (L = 2).
+// GDN_FLAG_QK_L2NORM on a bf16 tile of 128-wide rows stored as two 64-column halves
+// `half_bytes` apart, each row 128 bytes of 16-byte chunks swizzled by sw128_off: row `row` <-
+// row / max(|row|_2, kL2Eps), with the sum of squares in fp32 and the result rounded to bf16 in
+// place.  Two threads per row, adjacent lanes of one warp (`half` = 0 / 1, the lane's lowest
+// bit): each reads, scales and writes its half; the two partial sums meet by one shuffle.  The
+// caller orders the writes before the tensor core reads the tile (fence.proxy.async + barrier).
+__device__ __forceinline__ void l2norm_row_sw128(uint8_t* tile, uint32_t half_bytes, int row, int half) {
+    uint8_t* base = tile + half * half_bytes;
+    float ss = 0.f;  // first pass: the sum of squares (the row is read twice to keep registers low)
+#pragma unroll 2
+    for (int c = 0; c < 8; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4*>(base + sm100::sw128_off(row, c));
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(b2[e]);
+            ss += f.x * f.x + f.y * f.y;
+        }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    const float inv = 1.f / fmaxf(sqrtf(ss), kL2Eps);
+#pragma unroll 2
+    for (int c = 0; c < 8; ++c) {
+        uint4 u = *reinterpret_cast<const uint4*>(base + sm100::sw128_off(row, c));
+        __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(b2[e]);
+            b2[e] = __floats2bfloat162_rn(f.x * inv, f.y * inv);
+        }
+        *reinterpret_cast<uint4*>(base + sm100::sw128_off(row, c)) = u;
+    }
+}
+
 inline int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)

@@ -546,6 +546,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = wg_and(1, kThreadsP, mbar_wait(&bar_tma[stage], (k >> 1) & 1));
             if (!ok) break;
+            if (p.qk_norm) {  // raw q and k rows (0-63 q, 64-127 k): normalised in place first
+                l2norm_row_sw128(sm + kStageQK + stage * 32768, 16384, t >> 1, t & 1);
+                fence_proxy_async();
+                wg_sync(1, kThreadsP);
+            }
             if (t == 0) {  // MMA1: [Q;K] K^T -> Q K^T (lanes 0-63; lanes 64-127 are unused)
                 tc_fence_after();
 #pragma unroll

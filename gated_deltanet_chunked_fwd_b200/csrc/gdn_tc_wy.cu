@@ -162,6 +162,11 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
     // the Gram block; rows 64-127 come from the bytes after the tile and are not read), N = 64,
     // bf16 in, fp32 out in TMEM lanes 0-63 (one K row per lane)
     bool ok = __syncthreads_and(mbar_wait(bar, 0));  // the K tile has landed
+    if (p.qk_norm) {  // raw k rows: normalised in place before the Gram (thread pair per row)
+        l2norm_row_sw128(sm + wK, 8192, tid >> 1, tid & 1);
+        fence_proxy_async();
+        __syncthreads();
+    }
     if (ok && tid == 0) {
         const uint64_t dK = desc_sw128(smem_u32(sm + wK), 16, 1024);
         tc_fence_after();

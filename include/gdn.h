@@ -89,6 +89,11 @@ typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
                                           -softplus(a) = -log(1 + e^a); the backward's
                                           dbeta and dg are then gradients with respect to
                                           b and a.  Forward, backward and decode step.  */
+#define GDN_FLAG_QK_L2NORM (1u << 4)   /* raw q and k: each (token, head) row is
+                                          normalised over the head dimension,
+                                          x / max(|x|_2, 1e-6) in fp32, before use; dq
+                                          and dk are then gradients with respect to the
+                                          raw rows.  Forward, backward and decode step. */
 
 /* Arguments of the forward.  struct_size = sizeof(gdn_fwd_args),
  * abi_version = GDN_ABI_VERSION. */
@@ -223,7 +228,7 @@ typedef struct gdn_decode_args {
     int32_t Hk, Hv;    /* q/k heads, value heads (Hv % Hk == 0, contiguous groups)   */
     int32_t dk, dv;    /* head dims, 1..128, dv a multiple of 4                      */
     int32_t num_slots; /* states in S when state_indices != NULL (else N)            */
-    uint32_t flags;    /* GDN_FLAG_GATE_LOGITS or 0; other bits are ignored         */
+    uint32_t flags;    /* GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM; others ignored  */
     const void* q;     /* [N, Hk, dk] dtype                                          */
     const void* k;     /* [N, Hk, dk] dtype                                          */
     const void* v;     /* [N, Hv, dv] dtype                                          */

@@ -130,3 +130,27 @@ def test_gate_logits(dt):
     torch.cuda.synchronize()
     assert rel_l2(o, o_ref[:, 0]) < TOL[x["q"].dtype]
     assert rel_l2(S, S_ref) < 1e-5
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_qk_l2norm(dt):
+    """GDN_FLAG_QK_L2NORM (with GDN_FLAG_GATE_LOGITS) in the decode step: raw q, k rows."""
+    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM
+
+    x = decode_inputs(6, 2, 4, 128, 128, dt, seed=47)
+    gen = torch.Generator().manual_seed(48)
+    for name in ("q", "k"):
+        y = x[name].float().cpu() * (0.3 + 2.7 * torch.rand(x[name].shape[:-1] + (1,), generator=gen))
+        x[name] = y.to(x[name].dtype).to(DEV)
+    x["beta"] = (2.0 * torch.randn(x["beta"].shape, generator=gen)).to(DEV)
+    x["g"] = (torch.randn(x["g"].shape, generator=gen) + 1.0).to(DEV)
+    S = x["initial_state"].clone()
+    c = cpu(x)
+    o_ref, S_ref = oracle.fwd(c["q"], c["k"], c["v"], c["beta"], c["g"], initial_state=S.cpu(),
+                              qk_l2norm=True, gate_logits=True)
+    c0 = {n: x[n][:, 0].contiguous() for n in ("q", "k", "v", "beta", "g")}
+    o = gdn_decode_step(c0["q"], c0["k"], c0["v"], c0["beta"], c0["g"], S,
+                        flags=GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS, check_device_status=True)
+    torch.cuda.synchronize()
+    assert rel_l2(o, o_ref[:, 0]) < TOL[x["q"].dtype]
+    assert rel_l2(S, S_ref) < TOL[x["q"].dtype]

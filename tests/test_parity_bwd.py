@@ -221,3 +221,38 @@ def test_gate_logits(dt, flags):
     refs = oracle.bwd(x["q"], x["k"], x["v"], x["beta"], x["g"], x["do"], cu_seqlens=x["cu_seqlens"],
                       initial_state=x["initial_state"], dST=x["dST"], gate_logits=True)
     compare(run(inp, flags | GDN_FLAG_GATE_LOGITS), refs, TOL[inp["q"].dtype], "gate logits")
+
+
+@pytest.mark.parametrize("dt,flags", [("bf16", 0), ("fp32", 0)], ids=["tensor-core", "cuda-core-fp32"])
+@pytest.mark.parametrize("gates", [False, True], ids=["qk-norm", "qk-norm+gate-logits"])
+def test_qk_l2norm(dt, flags, gates):
+    """GDN_FLAG_QK_L2NORM: dq and dk are gradients with respect to the raw rows (the reduction
+    kernel applies the normalisation's chain rule after the group sum), alone and with
+    GDN_FLAG_GATE_LOGITS; all six gradients against the oracle, ragged, grouped heads."""
+    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM
+    from tests.test_parity_fwd import with_raw_gates, with_raw_qk
+
+    d = 128 if dt == "bf16" else 64
+    inp = with_raw_qk(make_inputs(1, 0, 2, 4, d, d, dtype=dt, seed=42, s0_std=0.1, backward=True,
+                                  lengths=[300, 1, 0, 129], device=DEV), 43)
+    if gates:
+        inp = with_raw_gates(inp, 44)
+    x = cpu(inp)
+    refs = oracle.bwd(x["q"], x["k"], x["v"], x["beta"], x["g"], x["do"], cu_seqlens=x["cu_seqlens"],
+                      initial_state=x["initial_state"], dST=x["dST"], qk_l2norm=True, gate_logits=gates)
+    f = flags | GDN_FLAG_QK_L2NORM | (GDN_FLAG_GATE_LOGITS if gates else 0)
+    compare(run(inp, f), refs, TOL[inp["q"].dtype], f"qk norm gates={gates}")
+
+
+def test_qk_l2norm_ungrouped_tensor_core():
+    """GDN_FLAG_QK_L2NORM without grouped heads: dq / dk go through the fp32 per-head buffers and
+    the reduction kernel instead of the direct bf16 stores."""
+    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_QK_L2NORM
+    from tests.test_parity_fwd import with_raw_qk
+
+    inp = with_raw_qk(make_inputs(2, 200, 2, 2, 128, 128, dtype="bf16", seed=45, s0_std=0.1,
+                                  backward=True, device=DEV), 46)
+    x = cpu(inp)
+    refs = oracle.bwd(x["q"], x["k"], x["v"], x["beta"], x["g"], x["do"], initial_state=x["initial_state"],
+                      dST=x["dST"], qk_l2norm=True)
+    compare(run(inp, GDN_FLAG_QK_L2NORM), refs, TOL[inp["q"].dtype], "qk norm ungrouped")

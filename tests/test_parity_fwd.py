@@ -10,7 +10,8 @@ import pytest
 import torch
 
 import oracle
-from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_SPLIT_FORCE,
+from gated_deltanet_chunked_fwd_b200 import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_QK_L2NORM,
+                                             GDN_FLAG_SPLIT_FORCE,
                                              GDN_FLAG_SPLIT_OFF, gdn_chunk_fwd)
 from gated_deltanet_chunked_fwd_b200.inputs import make_inputs, make_workload
 from tests._helpers import TOL, assert_every_unit, cpu, rel_l2
@@ -277,5 +278,41 @@ def test_gate_logits(dt, flags):
     x = cpu(inp)
     o_ref, ST_ref = oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["g"], cu_seqlens=x["cu_seqlens"],
                                initial_state=x["initial_state"], gate_logits=True)
+    tol = TOL[inp["q"].dtype]
+    assert rel_l2(o, o_ref) < tol and rel_l2(ST, ST_ref) < tol, (rel_l2(o, o_ref), rel_l2(ST, ST_ref))
+
+
+def with_raw_qk(inp, seed):
+    """Raw q and k rows for GDN_FLAG_QK_L2NORM: the generator's unit rows times random scales in
+    [0.3, 3] (and one exactly zero k row), rounded to the tensor dtype again."""
+    gen = torch.Generator().manual_seed(seed)
+    inp = dict(inp)
+    for name in ("q", "k"):
+        x = inp[name].float().cpu()
+        scale = 0.3 + 2.7 * torch.rand(x.shape[:-1] + (1,), generator=gen)
+        x = x * scale
+        if name == "k" and x.shape[1] > 5:
+            x[0, 5] = 0.0
+        inp[name] = x.to(inp[name].dtype).to(inp[name].device)
+    return inp
+
+
+@pytest.mark.parametrize("dt,flags", [("bf16", 0), ("fp32", 0), ("bf16", GDN_FLAG_PORTABLE)],
+                         ids=["tensor-core", "cuda-core-fp32", "cuda-core-bf16"])
+@pytest.mark.parametrize("gates", [False, True], ids=["qk-norm", "qk-norm+gate-logits"])
+def test_qk_l2norm(dt, flags, gates):
+    """GDN_FLAG_QK_L2NORM: raw q and k rows (scales 0.3-3, one zero row), ragged sequences,
+    grouped heads, alone and with GDN_FLAG_GATE_LOGITS; o and S_T against the oracle
+    normalising in float64."""
+    d = 128 if dt == "bf16" else 64
+    inp = with_raw_qk(make_inputs(1, 0, 2, 4, d, d, dtype=dt, seed=39, s0_std=0.1,
+                                  lengths=[300, 1, 0, 129], device=DEV), 40)
+    if gates:
+        inp = with_raw_gates(inp, 41)
+    f = flags | GDN_FLAG_QK_L2NORM | (GDN_FLAG_GATE_LOGITS if gates else 0)
+    o, ST = run(inp, f)
+    x = cpu(inp)
+    o_ref, ST_ref = oracle.fwd(x["q"], x["k"], x["v"], x["beta"], x["g"], cu_seqlens=x["cu_seqlens"],
+                               initial_state=x["initial_state"], qk_l2norm=True, gate_logits=gates)
     tol = TOL[inp["q"].dtype]
     assert rel_l2(o, o_ref) < tol and rel_l2(ST, ST_ref) < tol, (rel_l2(o, o_ref), rel_l2(ST, ST_ref))
