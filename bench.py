@@ -424,7 +424,7 @@ def e2e_leg(inp, dev, stream, measure, steps, tokens, world):
 
 def run_ours(args, world, rank, local):
     import gated_deltanet_chunked_fwd_b200 as gdn
-    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_SPLIT_OFF
+    from gated_deltanet_chunked_fwd_b200 import GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM, GDN_FLAG_SPLIT_OFF
     from gated_deltanet_chunked_fwd_b200.inputs import WORKLOADS, make_workload
 
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -524,6 +524,25 @@ def run_ours(args, world, rank, local):
                 "roofline": roofline(dense * tokens * Hv, c.bytes(), m * 1e-3, hbm, bf16, src)}
             del c
         del wk
+        # the headline fed raw inputs: q, k rows at random scales and beta, g as logits /
+        # pre-activations, normalised and mapped inside (GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS);
+        # the logits are drawn so that the mapped beta and g follow the headline's distributions
+        # (beta = sigmoid(N(0,1)), g = -softplus(N(g_mu,1)))
+        wr = make_workload(HEADLINE, seed=rank, device=dev)
+        gen = torch.Generator().manual_seed(rank)
+        for name in ("q", "k"):
+            x = wr[name].float().cpu()
+            wr[name] = (x * (0.3 + 2.7 * torch.rand(x.shape[:-1] + (1,), generator=gen))).to(
+                wr[name].dtype).to(dev)
+        wr["beta"] = torch.randn(wr["beta"].shape, generator=gen).to(dev)
+        wr["g"] = (torch.randn(wr["g"].shape, generator=gen) + WORKLOADS[HEADLINE].g_mu).to(dev)
+        c = FwdCall(wr, dev, stream, flags=GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS)
+        m = measure(c, max(2, min(args.steps, 5)))
+        extra["fwd_bf16_T65536_H16_d128_raw_inputs_fused_preprocessing"] = {
+            "ms": m, "tokens_per_s": job_throughput(tokens, world, m), "tokens": tokens,
+            "launches": c.launches,
+            "roofline": roofline(dense * tokens * Hv, c.bytes(), m * 1e-3, hbm, bf16, src)}
+        del c, wr
 
     # ---- backward on its own workload
     bwd = None

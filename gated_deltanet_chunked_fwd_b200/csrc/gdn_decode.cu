@@ -48,7 +48,8 @@ struct DecodeArgs {
     int qk_norm;      // GDN_FLAG_QK_L2NORM
 };
 
-template <typename Tin>
+// kPrep: the input preprocessing flags (GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM) are compiled in
+template <typename Tin, bool kPrep>
 __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArgs a) {
     __shared__ float sk[kMaxHead], sq[kMaxHead], sv[kDecCols];
     __shared__ float4 pa[kRowGroups][kColGroups], pb[kRowGroups][kColGroups];  // partial column dots
@@ -87,10 +88,11 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArg
         sq[t] = to_f(qp[t]);
     }
     if (t < kDecCols && jb + t < dv) sv[t] = to_f(vp[t]);
-    const float eg = expf(gate_g(a.g[(int64_t)n * a.Hv + h], a.gate_logits));
-    const float bt = gate_beta(a.beta[(int64_t)n * a.Hv + h], a.gate_logits);
+    const int glog = kPrep ? a.gate_logits : 0;
+    const float eg = expf(gate_g(a.g[(int64_t)n * a.Hv + h], glog));
+    const float bt = gate_beta(a.beta[(int64_t)n * a.Hv + h], glog);
     __syncthreads();
-    if (a.qk_norm) {  // raw k and q: x / max(|x|, eps), norms by warps 0 (k) and 1 (q)
+    if (kPrep && a.qk_norm) {  // raw k and q: x / max(|x|, eps), norms by warps 0 (k) and 1 (q)
         if (t < 64) {
             const float* x = t < 32 ? sk : sq;
             float ss = 0.f;
@@ -216,10 +218,14 @@ gdn_status launch_decode(const gdn_decode_args* a, cudaStream_t s) {
     d.gate_logits = (a->flags & GDN_FLAG_GATE_LOGITS) ? 1 : 0;
     d.qk_norm = (a->flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     const dim3 grid((unsigned)((int64_t)a->N * a->Hv), (unsigned)((a->dv + kDecCols - 1) / kDecCols));
-    if (a->dtype == GDN_BF16)
-        gdn_decode_kernel<__nv_bfloat16><<<grid, kDecThreads, 0, s>>>(d);
-    else
-        gdn_decode_kernel<float><<<grid, kDecThreads, 0, s>>>(d);
+    const bool prep = d.gate_logits || d.qk_norm;
+    if (a->dtype == GDN_BF16) {
+        if (prep) gdn_decode_kernel<__nv_bfloat16, true><<<grid, kDecThreads, 0, s>>>(d);
+        else gdn_decode_kernel<__nv_bfloat16, false><<<grid, kDecThreads, 0, s>>>(d);
+    } else {
+        if (prep) gdn_decode_kernel<float, true><<<grid, kDecThreads, 0, s>>>(d);
+        else gdn_decode_kernel<float, false><<<grid, kDecThreads, 0, s>>>(d);
+    }
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

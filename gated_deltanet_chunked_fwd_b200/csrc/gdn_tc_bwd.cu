@@ -177,7 +177,8 @@ __device__ __forceinline__ float bf(const uint8_t* tile, int row, int col) {  //
 // publishes its own exit adjoint M X + B.  A segment that does not take the scan but has an
 // earlier one that does walks to its exit adjoint from its usual start and publishes it.  Every
 // other segment leaves at once.
-template <bool kPre>
+// kPrep: the input preprocessing flags (GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM) are compiled in.
+template <bool kPre, bool kPrep>
 __global__ void __launch_bounds__(kNT, 1)
     gdn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(kNT, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hv = p.Hv, dk = 128, dv = 128;
+    const int glog = kPrep ? p.gate_logits : 0;  // GDN_FLAG_GATE_LOGITS, when compiled in
     // ---- which (sequence, head, segment) this CTA owns (the forward's scheme, except that the
     // later segments of a sequence take the lower block indices: a segment that takes the adjoint
     // scan waits for later ones, which are then scheduled no later than it)
@@ -356,15 +358,18 @@ __global__ void __launch_bounds__(kNT, 1)
         if (tid < 64 && c >= c0) {
             const int64_t t0 = bos + (int64_t)c * kChunk;
             const int lcc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
-            nxt_g = tid < lcc ? gate_g(p.g[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;  // padding: g = 0,
-            nxt_b = tid < lcc ? gate_beta(p.beta[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;  // beta = 0
+            // padding: g = beta = 0 (as raw gates: -inf, which the maps take to 0); raw gates are
+            // mapped where they are used, a chunk later
+            const float pad = glog ? -INFINITY : 0.f;
+            nxt_g = tid < lcc ? p.g[(t0 + tid) * Hv + h] : pad;
+            nxt_b = tid < lcc ? p.beta[(t0 + tid) * Hv + h] : pad;
         }
     };
     auto gates = [&](int c, int lc) -> bool {
         float gr = 0.f, gm = 0.f;
         if (tid < 64) {
-            float x = nxt_g;
-            const float bt = nxt_b;
+            float x = gate_g(nxt_g, glog);
+            const float bt = gate_beta(nxt_b, glog);
             prefetch_gates(c - 1);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kNT, 1)
         ok = __syncthreads_and(mbar_wait(bar_ld, ph_ld));
         ph_ld ^= 1;
         if (!ok) break;
-        if (p.qk_norm)  // raw q and k rows (0-63 q, 64-127 k): normalised in place first
+        if (kPrep && p.qk_norm)  // raw q and k rows (0-63 q, 64-127 k): normalised in place first
             l2norm_row_sw128(sm + bQK, 16384, tid >> 1, tid & 1);
         fence_proxy_async();
         tc_fence_before();
@@ -855,7 +860,7 @@ __global__ void __launch_bounds__(kNT, 1)
                 const uint8_t* qtile = sm + bQK + (i >> 6) * 16384;
                 // without grouped heads dq / dk go out directly (bf16); else per value head (fp32)
                 // for the reduction over the group
-                const bool direct = p.group == 1 && !p.qk_norm;
+                const bool direct = p.group == 1 && !(kPrep && p.qk_norm);
                 float* dqp = args.dqw + (t0 * Hv + h) * dk + i;
                 float* dkp = args.dkw + (t0 * Hv + h) * dk + i;
                 __nv_bfloat16* dqb = (__nv_bfloat16*)b.dq + (t0 * Hv + h) * dk + i;
@@ -938,12 +943,11 @@ __global__ void __launch_bounds__(kNT, 1)
                     const float y = __shfl_down_sync(0xffffffffu, suf, o);
                     if (lane + o < 32) suf += y;
                 }
-                if (r0 < lc) b.dg[(t0 + r0) * Hv + h] = gate_g_grad(suf, p.gate_logits ? p.g[(t0 + r0) * Hv + h] : 0.f, p.gate_logits);
+                if (r0 < lc) b.dg[(t0 + r0) * Hv + h] = gate_g_grad(suf, glog ? p.g[(t0 + r0) * Hv + h] : 0.f, glog);
                 if (r0 + 1 < lc)
-                    b.dg[(t0 + r0 + 1) * Hv + h] =
-                        gate_g_grad(suf - x0, p.gate_logits ? p.g[(t0 + r0 + 1) * Hv + h] : 0.f, p.gate_logits);
+                    b.dg[(t0 + r0 + 1) * Hv + h] = gate_g_grad(suf - x0, glog ? p.g[(t0 + r0 + 1) * Hv + h] : 0.f, glog);
             }
-            if (tid < lc) b.dbeta[(t0 + tid) * Hv + h] = gate_beta_grad(acc_b[tid], vbeta[tid], p.gate_logits);
+            if (tid < lc) b.dbeta[(t0 + tid) * Hv + h] = gate_beta_grad(acc_b[tid], vbeta[tid], glog);
         }
         tc_fence_before();
         __syncthreads();
@@ -1227,10 +1231,13 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
     if (!make_map(&mq, p.q, Tt, p.Hk) || !make_map(&mk, p.k, Tt, p.Hk) || !make_map(&mv, p.v, Tt, p.Hv) ||
         !make_map(&mdo, bp.dout, Tt, p.Hv))
         return GDN_ERR_CUDA;
-    if (cudaFuncSetAttribute(gdn_bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
+    const bool prep = p.gate_logits || p.qk_norm;
+    auto main_k = prep ? gdn_bwd_tc_kernel<false, true> : gdn_bwd_tc_kernel<false, false>;
+    auto pre_k = prep ? gdn_bwd_tc_kernel<true, true> : gdn_bwd_tc_kernel<true, false>;
+    if (cudaFuncSetAttribute(main_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
             cudaSuccess ||
         (a.scan_rec &&
-         cudaFuncSetAttribute(gdn_bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
+         cudaFuncSetAttribute(pre_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemB) !=
              cudaSuccess))
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
@@ -1254,10 +1261,10 @@ gdn_status launch_bwd_tc(const BwdPlan& plan, char* ws, cudaStream_t s) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, gdn_bwd_tc_kernel<true>, mq, mk, mv, mdo, a) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, pre_k, mq, mk, mv, mdo, a) != cudaSuccess)
             return GDN_ERR_CUDA;
     }
-    gdn_bwd_tc_kernel<false><<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);
+    main_k<<<(unsigned)sc.ctas, kNT, kSmemB, s>>>(mq, mk, mv, mdo, a);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     if (p.T_total > 0 && (p.group > 1 || p.qk_norm)) return launch_bwd_reduce(bp, a.dqw, a.dkw, s);
     return GDN_OK;

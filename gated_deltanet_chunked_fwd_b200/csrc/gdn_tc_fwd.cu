@@ -232,6 +232,9 @@ __device__ __forceinline__ void scan_start_state(uint32_t tl, int m, const int32
     }
 }
 
+// kPrep: the input preprocessing flags (GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM) are compiled in;
+// without them the kernel is the plain form.
+template <bool kPrep>
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -436,13 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // are in shared memory before chunk k is handed to group S.  g / beta of the chunk after
         // that are prefetched into registers.
         float gx0 = 0.f, gx1 = 0.f;
+        const int glog = kPrep ? p.gate_logits : 0;  // GDN_FLAG_GATE_LOGITS, when compiled in
         auto load_gates = [&](int kk) {
             const int cc = chunk_ofn(kk);
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lcc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
             const int r0 = 2 * lane;
-            gx0 = r0 < lcc ? gate_g(p.g[(t0 + r0) * Hv + h], p.gate_logits) : 0.f;  // padding: g = 0
-            gx1 = r0 + 1 < lcc ? gate_g(p.g[(t0 + r0 + 1) * Hv + h], p.gate_logits) : 0.f;
+            // padding: g = 0 (as a raw gate: -inf, which -softplus maps to 0); raw gates are mapped
+            // where they are used, a chunk later, so that the prefetch does not wait here
+            const float pad = glog ? -INFINITY : 0.f;
+            gx0 = r0 < lcc ? p.g[(t0 + r0) * Hv + h] : pad;
+            gx1 = r0 + 1 < lcc ? p.g[(t0 + r0 + 1) * Hv + h] : pad;
         };
         // vectors of chunk kk (buffer kk mod 4; beta enters through the Bw / Bu images): gamma =
         // cumsum g, Gam = exp(gamma), decay to the chunk end exp(gamma_n - gamma), the E factors
@@ -450,13 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // exp2(a_r - b_s)
         auto gates = [&](int kk) {
             float* vec = (float*)(sm + kVec) + (kk & 3) * kVecStride;
-            float incl = gx0 + gx1;
+            const float m0 = gate_g(gx0, glog), m1 = gate_g(gx1, glog);
+            float incl = m0 + m1;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += y;
             }
-            const float g1 = incl, g0 = incl - gx1;
+            const float g1 = incl, g0 = incl - m1;
             const float gm = __shfl_sync(0xffffffffu, g1, 15);  // gamma_31
             const float gl = __shfl_sync(0xffffffffu, g1, 31);  // gamma_63 (= gamma of the last token)
             const bool fac = __all_sync(0xffffffffu, fabsf(g0 - gm) < 80.f && fabsf(g1 - gm) < 80.f);
@@ -546,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = wg_and(1, kThreadsP, mbar_wait(&bar_tma[stage], (k >> 1) & 1));
             if (!ok) break;
-            if (p.qk_norm) {  // raw q and k rows (0-63 q, 64-127 k): normalised in place first
+            if (kPrep && p.qk_norm) {  // raw q and k rows (0-63 q, 64-127 k): normalised in place first
                 l2norm_row_sw128(sm + kStageQK + stage * 32768, 16384, t >> 1, t & 1);
                 fence_proxy_async();
                 wg_sync(1, kThreadsP);
@@ -1001,7 +1009,8 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
         return GDN_ERR_CUDA;
     // o (replay mode writes no o: the map is then never used)
     if (!make_map(&mo, p.o ? p.o : p.v, Tt, p.Hv)) return GDN_ERR_CUDA;
-    if (cudaFuncSetAttribute(gdn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = (p.gate_logits || p.qk_norm) ? gdn_fwd_tc_kernel<true> : gdn_fwd_tc_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (sc.ctas > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
@@ -1023,7 +1032,7 @@ gdn_status launch_fwd_tc_impl(const Problem& p, const int32_t* cu_host, int spli
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = p.num_chunks > 0 ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, gdn_fwd_tc_kernel, mq, mk, mv, mo, a) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, a) != cudaSuccess) return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -87,8 +87,9 @@ __device__ __forceinline__ bool locate_slot(const Problem& p, int64_t x, int* n_
 }
 
 // kGrouped: value heads share q/k heads (p.group > 1); the CTA loops over the group.  Without
-// grouping the loop has one pass and compiles away.
-template <bool kGrouped>
+// grouping the loop has one pass and compiles away.  kPrep: the input preprocessing flags
+// (GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM) are compiled in.
+template <bool kGrouped, bool kPrep>
 __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : kWyMinBlocks)
     gdn_wy_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const Problem p, uint8_t* __restrict__ timg,
                      float2* __restrict__ summ, int32_t* __restrict__ flags, int nflags,
@@ -136,9 +137,13 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
         fence_barrier_init();
     }
     float xg = 0.f, bt = 0.f;
+    const int glog = kPrep ? p.gate_logits : 0;  // GDN_FLAG_GATE_LOGITS, when compiled in
     auto load_gates = [&](int h) {
-        xg = tid < lc ? gate_g(p.g[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;  // lc <= 64
-        bt = tid < lc ? gate_beta(p.beta[(t0 + tid) * Hv + h], p.gate_logits) : 0.f;
+        // padding: g = beta = 0 (as raw gates: -inf, which the maps take to 0); raw gates are mapped
+        // where they are used
+        const float pad = glog ? -INFINITY : 0.f;
+        xg = tid < lc ? p.g[(t0 + tid) * Hv + h] : pad;  // lc <= 64
+        bt = tid < lc ? p.beta[(t0 + tid) * Hv + h] : pad;
     };
     load_gates(hk * G);
     tc_fence_before();
@@ -162,7 +167,7 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
     // the Gram block; rows 64-127 come from the bytes after the tile and are not read), N = 64,
     // bf16 in, fp32 out in TMEM lanes 0-63 (one K row per lane)
     bool ok = __syncthreads_and(mbar_wait(bar, 0));  // the K tile has landed
-    if (p.qk_norm) {  // raw k rows: normalised in place before the Gram (thread pair per row)
+    if (kPrep && p.qk_norm) {  // raw k rows: normalised in place before the Gram (thread pair per row)
         l2norm_row_sw128(sm + wK, 8192, tid >> 1, tid & 1);
         fence_proxy_async();
         __syncthreads();
@@ -182,14 +187,15 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
     const int h = hk * G + gi;  // the value head of this pass
     // ---- gates: gamma = cumsum g (two warp scans), E_rs = a_r b_s when factorable
     float gr = 0.f;
+    const float btm = gate_beta(bt, glog);  // the mapped beta of this thread's token
     if (tid < 64) {
-        float x = xg;
+        float x = gate_g(xg, glog);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
-        vbeta[tid] = bt;
+        vbeta[tid] = btm;
         vgam[tid] = x;
     }
     __syncthreads();
@@ -202,7 +208,7 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
         const float LOG2E = 1.4426950408889634f;
         va[tid] = fac ? expf(gr - gm) : gr * LOG2E;
         vb[tid] = fac ? expf(gm - gr) : gr * LOG2E;
-        vbG[tid] = bt * expf(gr);
+        vbG[tid] = btm * expf(gr);
     }
     if (gi + 1 < G) load_gates(h + 1);  // the next value head's gates, while this one runs
     // the Gram block is in TMEM (the first pass waits for it) and the vectors are written
@@ -350,7 +356,9 @@ gdn_status tc::launch_wy_tc(const Problem& p, const CUtensorMap& tm_k, uint8_t* 
     if (p.num_chunks <= 0) return GDN_OK;
     const int64_t slots = img_slots(p);
     if (slots > 0x7fffffff || p.Hv > 65535) return GDN_ERR_UNSUPPORTED;
-    auto kern = p.group > 1 ? gdn_wy_tc_kernel<true> : gdn_wy_tc_kernel<false>;
+    const bool prep = p.gate_logits || p.qk_norm;
+    auto kern = p.group > 1 ? (prep ? gdn_wy_tc_kernel<true, true> : gdn_wy_tc_kernel<true, false>)
+                            : (prep ? gdn_wy_tc_kernel<false, true> : gdn_wy_tc_kernel<false, false>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wSmemBytes) != cudaSuccess)
         return GDN_ERR_CUDA;
     const dim3 grid((unsigned)slots, (unsigned)p.Hk);
