@@ -198,3 +198,33 @@ def test_decode_argument_checks():
     assert call(dargs(q=None)) == INVALID
     assert call(dargs(state_indices=FAKE, num_slots=0)) == INVALID
     assert call(dargs(N=0)) == OK
+
+
+def test_preprocessing_flags_reach_the_plan():
+    """GDN_FLAG_QK_L2NORM routes the tensor-core backward's dq / dk through the fp32 per-head
+    buffers and the reduction kernel even without grouped heads: one more launch and a larger
+    workspace; GDN_FLAG_GATE_LOGITS changes neither (the maps run inside the existing kernels)."""
+    L = _abi.lib()
+
+    def bwd(flags, Hv=2):
+        a = GdnBwdArgs()
+        a.struct_size = ctypes.sizeof(a)
+        a.abi_version = 1
+        a.dtype = _abi.GDN_BF16
+        a.B, a.T, a.Hk, a.Hv, a.dk, a.dv = 1, 512, 2, Hv, 128, 128
+        a.flags = flags
+        for f in ("q", "k", "v", "beta", "g", "dout", "dq", "dk_out", "dv_out", "dbeta", "dg"):
+            setattr(a, f, FAKE)
+        n = ctypes.c_size_t(0)
+        assert L.gdn_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
+        return L.gdn_chunk_bwd_launch_count(ctypes.byref(a)), n.value
+
+    plain, gates, norm = bwd(0), bwd(_abi.GDN_FLAG_GATE_LOGITS), bwd(_abi.GDN_FLAG_QK_L2NORM)
+    assert gates == plain
+    assert norm[0] == plain[0] + 1 and norm[1] > plain[1]
+    # with grouped heads the reduction runs anyway
+    assert bwd(_abi.GDN_FLAG_QK_L2NORM, Hv=4)[0] == bwd(0, Hv=4)[0]
+    # the forward keeps its two launches with either flag
+    for f in (_abi.GDN_FLAG_GATE_LOGITS, _abi.GDN_FLAG_QK_L2NORM):
+        assert L.gdn_chunk_fwd_launch_count(ctypes.byref(fwd_args(flags=f))) == \
+            L.gdn_chunk_fwd_launch_count(ctypes.byref(fwd_args()))
