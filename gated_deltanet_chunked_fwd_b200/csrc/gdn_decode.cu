@@ -19,8 +19,8 @@
 // d = 128), the two column dots are reduced over the 16 row groups in shared memory, and the new
 // state is written back from registers: no thread reads a state element after another thread
 // wrote it, so the update in place is safe, and different CTAs own different columns.  With 32
-// state registers per thread several CTAs share an SM, so one CTA's loads overlap another's
-// arithmetic and stores.
+// state registers per thread (64 in all) four CTAs share an SM, so one CTA's loads overlap
+// another's arithmetic and stores.
 #include "gdn_dtype.cuh"
 #include "gdn_internal.cuh"
 
@@ -32,6 +32,7 @@ constexpr int kDecCols = 64;                           // state columns per CTA
 constexpr int kColGroups = kDecCols / 4;               // 16 (four columns per thread)
 constexpr int kRowGroups = kDecThreads / kColGroups;   // 16
 constexpr int kRowsPerThread = kMaxHead / kRowGroups;  // 8
+constexpr int kDecMinBlocks = 4;  // CTAs per SM the registers are sized for (64 per thread)
 
 struct DecodeArgs {
     int N, Hk, Hv, dk, dv, group, num_slots;
@@ -50,7 +51,7 @@ struct DecodeArgs {
 
 // kPrep: the input preprocessing flags (GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM) are compiled in
 template <typename Tin, bool kPrep>
-__global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks) gdn_decode_kernel(const DecodeArgs a) {
     __shared__ float sk[kMaxHead], sq[kMaxHead], sv[kDecCols];
     __shared__ float4 pa[kRowGroups][kColGroups], pb[kRowGroups][kColGroups];  // partial column dots
     __shared__ float colA[kDecCols], colB[kDecCols];
