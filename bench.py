@@ -447,6 +447,13 @@ def run_ours(args, world, rank, local):
         barrier(world)
         return max_over_ranks(sum(ms) / len(ms), world)
 
+    if args.decode_only:
+        # the decode workload by itself, so that a profiler sees its launches alone
+        r = decode_bench(dev, stream, rank, measure, world, hbm, bf16, src, args.steps)
+        if rank == 0:
+            print(json.dumps({"workload": "decode_bf16_N64_Hk16_Hv32_d128", **r}), flush=True)
+        return
+
     # ---- headline: one 65,536-token call (fewer with --tokens, to profile a small case)
     inp = make_workload(HEADLINE, seed=rank, device=dev, **({"T": args.tokens} if args.tokens else {}))
     call = FwdCall(inp, dev, stream)
@@ -648,6 +655,8 @@ def main():
                     help="headline shape with this many tokens (profiling a small case; 0 = 65,536)")
     ap.add_argument("--bwd-batch", type=int, default=4,
                     help="sequences in the backward workload (4 = the backward workload; fewer for a small profile)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time the decode workload by itself and print its line (profiling)")
     args = ap.parse_args()
     if args.impl == "reference":
         # the oracle arm runs on rank 0's host cores only; no process group
