@@ -65,13 +65,16 @@ namespace {
 //                                       images of the WY step as B operands), W^T -> smem
 //   group S (threads 256-383, 4 warps)  the state chain of chunk k: U^T = Ut^T - H^T W^T,
 //                                       O^T, H^T <- Gam_n H^T + (U^T diag(decay)) K, bf16 H
-// Each group has one tcgen05 issuer (threads 0 and 256) and its own commit
-// barrier; they hand chunks over through mbarriers (full / empty pairs).  Warp w
+// Each group has a tcgen05 issuer (threads 0 and 256) and its own commit barrier; group P
+// issues Ut^T from a second thread (kUIssuer, own barrier) at the same time as Q K^T, so that
+// the two run together and only W^T waits for P.  The groups hand chunks over through
+// mbarriers (full / empty pairs).  Warp w
 // reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so group P's two warps per lane
 // quarter split the columns.
 constexpr int kThreads = 384;
 constexpr int kThreadsP = 256;
 constexpr int kThreadsS = 128;
+constexpr int kUIssuer = 96;  // group P's second MMA issuer (warp 3; thread 0 is the first)
 constexpr int kTmemCols = 512;
 // TMEM column map (lane = row of the M = 128 MMA)
 constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk     [0, 128)
@@ -249,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bar_wt_full = bars + 4;  // W^T of chunk k in smem, Ut^T of chunk k in TMEM
     uint64_t* bar_wt_empty = bars + 5; // MMA_HW of chunk k has read W^T
     uint64_t* bar_s_done = bars + 6;   // [2] group S finished chunk k (parity buffers free)
+    uint64_t* bar_mma_u = bars + 8;    // MMA_U completions (group P's second issuer)
     uint32_t* tmem_slot = (uint32_t*)(bars + 9);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -427,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = tid;
         const int hf = t >> 7;                       // which 32-column half of a TMEM row
         const int row = ((warp & 3) << 5) | lane;    // TMEM lane (= MMA row) this thread reads
-        uint32_t ph = 0;  // parity of bar_mma_p
+        uint32_t ph = 0;   // parity of bar_mma_p
+        uint32_t phu = 0;  // parity of bar_mma_u
         // The loops come in two compiled forms: one walk over the chunks (every segment that does
         // not take the scan), or the three walks of the scan.
         auto run_p = [&](auto walks) {
@@ -536,6 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = chunk_ofn(k);
             const int stage = k & 1;
             const bool emit = emits(k);
+            const bool with_v = v_onn(k);  // walk 1 of a scan (the M fold) has v = 0: no Ut
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)c * kChunk);
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t sV = sbase + kStageV + stage * 16384;
@@ -559,7 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async();
                 wg_sync(1, kThreadsP);
             }
-            if (t == 0) {  // MMA1: [Q;K] K^T -> Q K^T (lanes 0-63; lanes 64-127 are unused)
+            if (emit && t == 0) {  // MMA1: [Q;K] K^T -> Q K^T (lanes 0-63; lanes 64-127 are unused);
+                                   // a chunk without outputs (warm-up, fold walk, replay) needs none
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -569,13 +576,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(bar_mma_p);
             }
+            if (with_v && t == kUIssuer) {  // MMA_U: Ut^T = V^T Bu^T (R2[stage]) from a second issuer,
+                                            // on its own barrier, while MMA1 runs
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
+                                desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
+                mma_commit(bar_mma_u);
+            }
             if (warp == 2 && k + 1 < nk) {  // the next chunk's gates, while MMA1 runs
                 gates(k + 1);
                 if (k + 2 < nk) load_gates(k + 2);
             }
-            ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
-            ph ^= 1;
-            if (!ok) break;
+            if (emit) {
+                ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
+                ph ^= 1;
+                if (!ok) break;
+            }
             tc_fence_after();
             const bool fac = vec[448] != 0.f;
 
@@ -636,26 +654,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             wg_sync(1, kThreadsP);
 
-            if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1);  MMA_U: Ut^T = V^T Bu^T (R2[stage]), unless the
-                           // walk has v = 0 (the M fold of a scan: U = -W H)
-                const bool with_v = v_onn(k);
+            if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1, once P has read Q K^T from it)
                 tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 4; ++j)
                     mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
                                 desc_sw128(sBwu + j * 32, 16, 1024), id_mn_n64, j > 0);
-                    if (with_v)
-                        mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
-                                    desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
-                }
                 mma_commit(bar_mma_p);
             }
-            ok = wg_and(1, kThreadsP, mbar_wait(bar_mma_p, ph));
-            ph ^= 1;
-            if (!ok) break;
-            // Wt is free once MMA_HW of chunk k-1 has read it
-            if (k >= 1) {
-                ok = wg_and(1, kThreadsP, mbar_wait(bar_wt_empty, (k - 1) & 1));
+            {  // W^T and Ut^T are in TMEM, and Wt is free once MMA_HW of chunk k-1 has read it
+                bool w = mbar_wait(bar_mma_p, ph);
+                if (with_v) w = w && mbar_wait(bar_mma_u, phu);
+                if (k >= 1) w = w && mbar_wait(bar_wt_empty, (k - 1) & 1);
+                ok = wg_and(1, kThreadsP, w);
+                ph ^= 1;
+                if (with_v) phu ^= 1;
                 if (!ok) break;
             }
             tc_fence_after();

@@ -1,5 +1,5 @@
 // gdn_tc_inverse.cuh -- the blocked unit-lower-triangular inverse T = (I + A)^-1 of one chunk
-// (64 x 64, A strictly lower), shared by the WY kernel and the fused forward kernel.
+// (64 x 64, A strictly lower), used by the WY kernel.
 //
 // A and T share one fp32 64 x 64 array X (row stride kXs floats): A is strictly lower and T
 // unit lower-triangular, so A sits below the diagonal and T (off its unit diagonal) above it,
@@ -7,7 +7,9 @@
 // blocks are solved by fp32 forward substitution (threads 0..63 of the 128 that run it), then
 // three merge levels run as warp-level tf32 MMAs (four warps).  Every X entry that feeds a
 // merge is stored already rounded to tf32 (round to nearest, ties away), so the merges issue no
-// conversions; the diagonal blocks of A stay fp32 for the substitution.
+// conversions; the diagonal blocks of A stay fp32 for the substitution.  Once solved, a diagonal
+// block of X holds its block of T^T whole (the unit diagonal, and zeros where A was), so every
+// read of a diagonal T block, here and in the caller, takes X as it stands.
 #pragma once
 
 #include <stdint.h>
@@ -41,13 +43,11 @@ __device__ __forceinline__ void mma_tf32(float* d, float a0, float a1, float a2,
           "r"(__float_as_uint(a3)), "r"(__float_as_uint(b0)), "r"(__float_as_uint(b1)));
 }
 
-// T[r][s] given x = X[s][r] (the stored value when r > s): 1 on the diagonal, 0 above it
-__device__ __forceinline__ float t_sel(float x, int r, int s) { return r > s ? x : (r == s ? 1.f : 0.f); }
-
 // The four 16 x 16 diagonal blocks of T (threads 0..63: block t / 16, column t % 16): unit
 // lower-triangular inverse by forward substitution, reading each A row as 16-byte vectors.
-// Column cc of block b is T[16 b + r][16 b + cc] = x[r]; it is written to row 16 b + cc of X
-// once every thread has read its A block (the caller's barrier sits in between).
+// Column cc of block b is T[16 b + r][16 b + cc] = x[r] (x[r] = 0 for r < cc, x[cc] = 1); it is
+// written whole to row 16 b + cc of X once every thread has read its A block (the caller's
+// barrier sits in between).
 __device__ __forceinline__ void diag_solve(const float* X, int t, float* x) {
     const int b = t >> 4, cc = t & 15;
     const float* a = X + 16 * b * (kXs + 1);
@@ -105,11 +105,7 @@ __device__ __forceinline__ void merge_level(float* X, float* ysw, int warp, int 
                 const int kc = 16 * (j0 + kb) + 8 * ks + 2 * t;
                 const float2 a0 = *reinterpret_cast<const float2*>(X + r0 * kXs + kc);
                 const float2 a1 = *reinterpret_cast<const float2*>(X + (r0 + 8) * kXs + kc);
-                float2 bv = *reinterpret_cast<const float2*>(X + (col + g) * kXs + kc);
-                if (kb == 0) {  // T block (j0, j0) is the diagonal one
-                    bv.x = t_sel(bv.x, kc, col + g);
-                    bv.y = t_sel(bv.y, kc + 1, col + g);
-                }
+                const float2 bv = *reinterpret_cast<const float2*>(X + (col + g) * kXs + kc);
                 mma_tf32(y, a0.x, a1.x, a0.y, a1.y, bv.x, bv.y);
             }
         }
@@ -125,8 +121,7 @@ __device__ __forceinline__ void merge_level(float* X, float* ysw, int warp, int 
             const int kc = 16 * i + 8 * ks + t;
             const float2 p0 = *reinterpret_cast<const float2*>(X + kc * kXs + rr);
             const float2 p1 = *reinterpret_cast<const float2*>(X + (kc + 4) * kXs + rr);
-            mma_tf32(r, t_sel(p0.x, rr, kc), t_sel(p0.y, rr + 1, kc), t_sel(p1.x, rr, kc + 4),
-                     t_sel(p1.y, rr + 1, kc + 4), ysw[(8 * ks + t) * 9 + g], ysw[(8 * ks + t + 4) * 9 + g]);
+            mma_tf32(r, p0.x, p0.y, p1.x, p1.y, ysw[(8 * ks + t) * 9 + g], ysw[(8 * ks + t + 4) * 9 + g]);
         }
         __syncwarp();  // the scratch is rewritten by this warp's next unit
         // T block (i, j0), transposed into X above the diagonal

@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
         float* X = (float*)(sm + wK);
         if (warp < 2) {
             const int r = tid;
-            const float br = vbeta[r], ar = va[r];
+            const float br = r < lc ? vbeta[r] : 0.f;  // rows past the chunk's end are zero
+            const float ar = va[r], bra = br * ar;  // beta_r a_r
             float* xr = X + r * kXs;
             const int qn = warp == 0 ? 2 : 4;  // warp-uniform: the TMEM load is warp-collective
 #pragma unroll 1
@@ -245,18 +246,18 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
                     for (int e = 0; e < 16; ++e) dg = (e == (r & 15)) ? v[e] : dg;
                     vnrm[r] = dg;
                 }
-                // E_rs = a_r b_s, or exp2(a_r - b_s) when the chunk's decay range is too wide
-                // (block-uniform branch: one loop per form); E is used only under the mask:
-                // above the diagonal it may overflow.  Entries below the diagonal 16 x 16 blocks
+                // beta_r E_rs with E_rs = a_r b_s, or exp2(a_r - b_s) when the chunk's decay range
+                // is too wide (block-uniform branch: one loop per form); E is used only under the
+                // mask: above the diagonal it may overflow.  Entries below the diagonal 16 x 16 blocks
                 // (q < r / 16) are merge operands only: stored rounded to tf32.
                 const bool below = q < (r >> 4);
                 const bool store = q <= (r >> 4);
                 if (fac) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] *= ar * vb[16 * q + e];
+                    for (int e = 0; e < 16; ++e) v[e] *= bra * vb[16 * q + e];
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] *= exp2f(ar - vb[16 * q + e]);
+                    for (int e = 0; e < 16; ++e) v[e] *= br * exp2f(ar - vb[16 * q + e]);
                 }
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int s = 16 * q + 4 * e4 + e;
-                        const float x = (s < r && r < lc) ? br * v[4 * e4 + e] : 0.f;
+                        const float x = s < r ? v[4 * e4 + e] : 0.f;
                         o[e] = below ? tf32r(x) : x;
                     }
                     if (store) *reinterpret_cast<float4*>(xr + 16 * q + 4 * e4) = make_float4(o[0], o[1], o[2], o[3]);
@@ -297,12 +298,14 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
     __syncthreads();
 
     // ---- bf16 images T (for the backward only), Bw, Bu: thread = rows nr4 .. nr4 + 3, columns
-    // s0 .. s0 + 7 (one 16-byte chunk of each row), from T[r][s] = X[s][r] for r > s
+    // s0 .. s0 + 7 (one 16-byte chunk of each row, all in one 16 x 16 block of T), from
+    // T[r][s] = X[s][r].  X holds T^T in every block on or above its diagonal (the diagonal
+    // blocks exactly, with their ones and zeros); blocks of T above the diagonal are zero.
     {
         const int nr4 = 4 * (tid & 15), ch = tid >> 4, s0 = 8 * ch;
         uint8_t* img = timg + (img_slot(bos, n, c) * Hv + h) * (int64_t)kWyImgBytes;
         float v[4][8];
-        if (s0 > nr4 + 3) {  // the block lies above the diagonal
+        if ((s0 >> 4) > (nr4 >> 4)) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -311,10 +314,10 @@ __global__ void __launch_bounds__(kWyThreads, kGrouped ? kWyMinBlocksGrouped : k
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float4 col = *reinterpret_cast<const float4*>(X + (s0 + e) * kXs + nr4);
-                v[0][e] = t_sel(col.x, nr4, s0 + e);
-                v[1][e] = t_sel(col.y, nr4 + 1, s0 + e);
-                v[2][e] = t_sel(col.z, nr4 + 2, s0 + e);
-                v[3][e] = t_sel(col.w, nr4 + 3, s0 + e);
+                v[0][e] = col.x;
+                v[1][e] = col.y;
+                v[2][e] = col.z;
+                v[3][e] = col.w;
             }
         }
         float sw[8], su[8];
