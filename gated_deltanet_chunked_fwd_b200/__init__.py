@@ -20,13 +20,14 @@ import torch
 
 from . import _abi
 from ._abi import (GDN_FLAG_GATE_LOGITS, GDN_FLAG_PORTABLE, GDN_FLAG_QK_L2NORM, GDN_FLAG_SPLIT_FORCE,
-                   GDN_FLAG_SPLIT_OFF, GdnBwdArgs, GdnDecodeArgs, GdnError, GdnFwdArgs)
+                   GDN_FLAG_SPLIT_OFF, GdnBwdArgs, GdnCombineArgs, GdnDecodeArgs, GdnError, GdnFwdArgs,
+                   GdnHaloArgs)
 
 __all__ = ["gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_size",
            "gdn_chunk_bwd_workspace_size", "chunk_fwd", "chunk_bwd", "GdnError",
            "GDN_FLAG_SPLIT_OFF", "GDN_FLAG_SPLIT_FORCE", "GDN_FLAG_PORTABLE", "GDN_FLAG_GATE_LOGITS",
            "GDN_FLAG_QK_L2NORM",
-           "decode_step"]
+           "decode_step", "gdn_affine_combine", "gdn_halo_check"]
 
 _DT = {torch.float32: _abi.GDN_F32, torch.bfloat16: _abi.GDN_BF16}
 
@@ -224,6 +225,55 @@ def gdn_decode_step(q, k, v, beta, g, state, state_indices=None, *, out=None, fl
     _check("gdn_decode_step", _abi.lib().gdn_decode_step(ctypes.byref(a), _stream(q.device)))
     _raise_dev_status("gdn_decode_step", st)
     return o
+
+
+def gdn_affine_combine(M, X, B=None):
+    """X <- M X + B in place for every (sequence, value head); returns X.
+
+    M: fp32 [N, Hv, dk, dk]; X, B: fp32 [N, Hv, dk, dv] (B None = zero); X must not share
+    memory with M or B.  One step of the fold that gives a shard of a long sequence its entry
+    state (``cp_chunk_fwd``).
+    """
+    if M.dtype != torch.float32 or X.dtype != torch.float32 or (B is not None and B.dtype != torch.float32):
+        raise ValueError("M, X and B must be float32")
+    if M.dim() != 4 or X.dim() != 4 or M.shape[:2] != X.shape[:2] or M.shape[2] != M.shape[3] or \
+            M.shape[2] != X.shape[2] or (B is not None and B.shape != X.shape):
+        raise ValueError("M must be [N, Hv, dk, dk], X and B [N, Hv, dk, dv]")
+    a = GdnCombineArgs()
+    a.struct_size = ctypes.sizeof(a)
+    a.abi_version = _abi.GDN_ABI_VERSION
+    a.N, a.Hv, a.dk, a.dv = X.shape
+    a.M, a.B, a.X = _ptr(M), _ptr(B), _ptr(X)
+    _check("gdn_affine_combine", _abi.lib().gdn_affine_combine(ctypes.byref(a), _stream(X.device)))
+    return X
+
+
+def gdn_halo_check(k, beta, g, log_eps: float, *, flags: int = 0, log_decay: bool = False):
+    """Per value head, whether the tokens of k, beta, g (a halo) can stand in for everything
+    before them: int32 [Hv] (1 = yes), and with ``log_decay`` also their summed log decay.
+
+    k: [T, Hk, dk] (fp32 or bf16); beta, g: [T, Hv] fp32; flags: GDN_FLAG_GATE_LOGITS,
+    GDN_FLAG_QK_L2NORM as in the forward.
+    """
+    if k.dim() != 3 or beta.dim() != 2 or g.shape != beta.shape or beta.shape[0] != k.shape[0]:
+        raise ValueError("k must be [T, Hk, dk], beta and g [T, Hv]")
+    if k.dtype not in _DT or beta.dtype != torch.float32 or g.dtype != torch.float32:
+        raise ValueError("k must be float32 or bfloat16, beta and g float32")
+    T, Hk, dk = k.shape
+    Hv = beta.shape[1]
+    ok = torch.empty(Hv, dtype=torch.int32, device=k.device)
+    ld = torch.empty(Hv, dtype=torch.float32, device=k.device) if log_decay else None
+    a = GdnHaloArgs()
+    a.struct_size = ctypes.sizeof(a)
+    a.abi_version = _abi.GDN_ABI_VERSION
+    a.dtype = _DT[k.dtype]
+    a.T, a.Hk, a.Hv, a.dk = T, Hk, Hv, dk
+    a.flags = flags
+    a.log_eps = float(log_eps)
+    a.k, a.beta, a.g = (_ptr(k), _ptr(beta), _ptr(g)) if T > 0 else (None, None, None)
+    a.ok, a.log_decay = _ptr(ok), _ptr(ld)
+    _check("gdn_halo_check", _abi.lib().gdn_halo_check(ctypes.byref(a), _stream(k.device)))
+    return (ok, ld) if log_decay else ok
 
 
 def launch_count(q, k, v, beta, g, cu_seqlens=None, cu_seqlens_host=None, initial_state=None,

@@ -63,10 +63,26 @@ class GdnDecodeArgs(ctypes.Structure):
     ]
 
 
+class GdnCombineArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _u32), ("abi_version", _u32), ("N", _i32), ("Hv", _i32), ("dk", _i32),
+        ("dv", _i32), ("M", _p), ("B", _p), ("X", _p),
+    ]
+
+
+class GdnHaloArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _u32), ("abi_version", _u32), ("dtype", _i32), ("T", _i32), ("Hk", _i32),
+        ("Hv", _i32), ("dk", _i32), ("flags", _u32), ("log_eps", ctypes.c_float), ("k", _p),
+        ("beta", _p), ("g", _p), ("ok", _p), ("log_decay", _p),
+    ]
+
+
 EXPORTS = [
     "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_launch_count",
     "gdn_chunk_bwd_workspace_size", "gdn_chunk_bwd", "gdn_chunk_bwd_launch_count",
-    "gdn_status_string", "gdn_chunk_fwd_noalloc", "gdn_decode_step",
+    "gdn_status_string", "gdn_chunk_fwd_noalloc", "gdn_decode_step", "gdn_affine_combine",
+    "gdn_halo_check",
 ]
 
 _lib = None
@@ -99,6 +115,10 @@ def lib() -> ctypes.CDLL:
             getattr(L, fn).restype = ctypes.c_int
         L.gdn_decode_step.argtypes = [ctypes.POINTER(GdnDecodeArgs), _p]
         L.gdn_decode_step.restype = ctypes.c_int
+        L.gdn_affine_combine.argtypes = [ctypes.POINTER(GdnCombineArgs), _p]
+        L.gdn_affine_combine.restype = ctypes.c_int
+        L.gdn_halo_check.argtypes = [ctypes.POINTER(GdnHaloArgs), _p]
+        L.gdn_halo_check.restype = ctypes.c_int
         L.gdn_chunk_fwd_noalloc.argtypes = [F, _p]
         L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]

@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 #include "gdn_internal.cuh"
@@ -194,15 +195,24 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder.  Calls may come from several host threads at once: the entry
+// point is resolved once per process under std::call_once, and each calling thread first binds
+// its device's primary context (once per thread), so that the driver call has a current context
+// even in a thread whose first CUDA call this is.
 inline EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;  // resolved once per process (a driver entry point)
-    if (!fn) {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = (EncodeTiledFn)ptr;
+    });
+    thread_local bool bound = false;
+    if (!bound) {
+        int d = 0;
+        bound = cudaGetDevice(&d) == cudaSuccess && cudaSetDevice(d) == cudaSuccess;
     }
     return fn;
 }

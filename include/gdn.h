@@ -257,6 +257,65 @@ typedef struct gdn_decode_args {
  * argument errors return before anything is enqueued.  Needs no workspace. */
 GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, void* stream);
 
+/* ---- Context parallelism across GPUs (one long sequence, token shards on several
+ * GPUs).  The dothoosh.com FlashQLA article (first innovation: gate-driven context
+ * parallelism; its million-token paragraph) splits one long sequence automatically
+ * among processing units; across GPUs a shard needs the state its sequence carries
+ * into it.  Two ways to get it, both per (sequence, value head):
+ *  - the gate-driven way: start the shard a few chunks early (a halo of the previous
+ *    shard's last tokens) from a zero state; valid when the halo's summed log decay
+ *    is at most log(eps) and every halo token keeps 0 <= beta |k|^2 <= 2 (each
+ *    token's state map then has norm <= exp(g_t)), gdn_halo_check below;
+ *  - the exact way: every shard's tokens map its entry state affinely,
+ *    H_exit = M H_entry + B (M = the product of the tokens' maps, dk x dk; B = the
+ *    exit state from a zero entry), and the entry state of shard r is the fold of
+ *    shards 0..r-1 applied to S0, X <- M_j X + B_j in order: gdn_affine_combine below.
+ * The shards' folds (M from a forward with v = 0 and S0 = [I | 0], B from a forward
+ * with S0 = 0) and the collectives belong to the caller (the Python package's
+ * cp_chunk_fwd). */
+
+/* One step of the affine fold, per (sequence n, value head h):
+ *     X <- M X + B      (M [dk][dk], X and B [dk][dv], fp32, row-major).
+ * struct_size = sizeof(gdn_combine_args), abi_version = GDN_ABI_VERSION. */
+typedef struct gdn_combine_args {
+    uint32_t struct_size;
+    uint32_t abi_version;
+    int32_t N, Hv;    /* sequences and value heads (N * Hv states); 0 is a no-op      */
+    int32_t dk, dv;   /* 1..128                                                      */
+    const float* M;   /* [N, Hv, dk, dk]                                             */
+    const float* B;   /* [N, Hv, dk, dv] or NULL (zero)                              */
+    float* X;         /* in / out [N, Hv, dk, dv]; must overlap neither M nor B
+                         (GDN_ERR_INVALID_ARG); X, M and B 16-byte aligned            */
+} gdn_combine_args;
+/* One launch; asynchronous on `stream`; argument errors return before anything is
+ * enqueued.  fp32 arithmetic (fused multiply-adds in row order j = 0..dk-1). */
+GDN_API gdn_status gdn_affine_combine(const gdn_combine_args* args, void* stream);
+
+/* Whether a halo of tokens can stand in for everything before it, per value head:
+ * ok[h] = 1 when sum_t g[t][h] <= log_eps and 0 <= beta[t][h] |k[t][h / G]|^2 <= 2 for
+ * every halo token t (G = Hv / Hk; with GDN_FLAG_GATE_LOGITS g and beta are mapped
+ * first, with GDN_FLAG_QK_L2NORM k is normalised first, as in the forward), else 0.
+ * The gate-driven split of a sequence (dothoosh.com FlashQLA article, first
+ * innovation) takes this test for its warm-up across SMs; across GPUs the halo is
+ * the previous shard's last tokens.  struct_size = sizeof(gdn_halo_args). */
+typedef struct gdn_halo_args {
+    uint32_t struct_size;
+    uint32_t abi_version;
+    int32_t dtype;       /* gdn_dtype of k                                             */
+    int32_t T;           /* halo tokens (0: every head fails, no halo to stand in)     */
+    int32_t Hk, Hv, dk;  /* heads as in the forward, dk 1..128                         */
+    uint32_t flags;      /* GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM; others ignored  */
+    float log_eps;       /* bound on the summed log decay (the forward uses -30 ln 2) */
+    const void* k;       /* [T, Hk, dk] dtype                                          */
+    const float* beta;   /* [T, Hv]                                                    */
+    const float* g;      /* [T, Hv]                                                    */
+    int32_t* ok;         /* out [Hv]                                                   */
+    float* log_decay;    /* out [Hv] (the summed log decay) or NULL                    */
+} gdn_halo_args;
+/* One launch; asynchronous on `stream`; argument errors return before anything is
+ * enqueued. */
+GDN_API gdn_status gdn_halo_check(const gdn_halo_args* args, void* stream);
+
 /* Number of kernel launches gdn_chunk_fwd / gdn_chunk_bwd enqueue for these
  * arguments (a pure function of the arguments; -1 on an argument error).  The
  * FlashQLA pages describe no interface; this is for launch accounting. */
