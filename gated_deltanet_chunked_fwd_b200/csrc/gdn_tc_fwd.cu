@@ -759,17 +759,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (args.himg && c >= c0 && fin) {
                 // replay mode: the chunk's entry state, as the bf16 H^T image [dk half][128 dv
                 // rows][128 B] (128-byte swizzled) that the backward loads; the bf16 copy in TMEM
-                // holds it (dk pairs per column)
+                // holds it (dk pairs per column).  Staged in the two 16 KB tiles that replay mode
+                // leaves unused (P's tile and the output tile), then written by two bulk copies:
+                // a thread per row writing 16 bytes into each of 128 rows straight to global
+                // memory used only half of every sector it touched.
                 uint8_t* img = args.himg + (img_slot(bos, n, c) * Hv + h) * (int64_t)32768;
+                if (m == 0) bulk_wait_read0();  // the previous image's copies have read the tiles
+                wg_sync(2, kThreadsS);
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     float w[32];
                     tmem_ld32(tl + kColHb + 32 * a, w);
+                    uint8_t* tile = sm + (a == 0 ? kPt : kOst);
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc)
-                        *reinterpret_cast<uint4*>(img + a * 16384 + sw128_off(m, cc)) =
+                        *reinterpret_cast<uint4*>(tile + sw128_off(m, cc)) =
                             make_uint4(__float_as_uint(w[4 * cc]), __float_as_uint(w[4 * cc + 1]),
                                        __float_as_uint(w[4 * cc + 2]), __float_as_uint(w[4 * cc + 3]));
+                }
+                fence_proxy_async();  // the tiles are read by the bulk copies
+                wg_sync(2, kThreadsS);
+                if (m == 0) {
+                    bulk_store(img, sm + kPt, 16384);
+                    bulk_store(img + 16384, sm + kOst, 16384);
+                    bulk_commit();
                 }
             }
             ok = wg_and(2, kThreadsS, mbar_wait(bar_mma_s, ph));
@@ -937,6 +950,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (!ok && (tid == 0 || tid == kThreadsP)) report(p.status, GDN_ERR_TIMEOUT);
+    if (args.himg && tid == kThreadsP) bulk_wait0();  // the entry-state images have been written
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
