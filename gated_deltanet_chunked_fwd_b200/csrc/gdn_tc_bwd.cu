@@ -683,7 +683,8 @@ __global__ void __launch_bounds__(kNT, 1)
         if (emit) {  // the chunk's gradients (own chunks only)
             {  // U^T -> Ut;  TdU: dv out, rows 64..127 of the dO tile, dbeta part;
                // this thread: row m of U^T and of TdU^T, tokens [32 hh, 32 hh + 32) in groups of 8
-                __nv_bfloat16* dvp = (__nv_bfloat16*)b.dv + (t0 * Hv + h) * dv + m;
+                __nv_bfloat16* dvp = (__nv_bfloat16*)b.dv + (t0 * Hv + h) * dv + (m & ~1);  // bf16 pairs
+                const bool odd = m & 1;
 #pragma unroll 1
                 for (int g = 0; g < 4; ++g) {
                     const int tb = 32 * hh + 8 * g;  // first token of the group
@@ -695,13 +696,22 @@ __global__ void __launch_bounds__(kNT, 1)
                     const float btv[8] = {bt0.x, bt0.y, bt0.z, bt0.w, bt1.x, bt1.y, bt1.z, bt1.w};
                     float bvals[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int r = tb + e;
-                        if (r < lc) dvp[(int64_t)r * Hv * dv] = __float2bfloat16_rn(btv[e] * t8[e]);
-                        bvals[e] = t8[e] * bf(sm + bV + (m >> 6) * 8192, r, m & 63);  // TdU[r][m] v[r][m]
-                        // TdU row r of the stacked [dO ; TdU] tile: element (64 + r, m)
-                        *reinterpret_cast<__nv_bfloat16*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
-                                                          (m & 7) * 2) = __float2bfloat16_rn(t8[e]);
+                    for (int e = 0; e < 8; ++e)  // TdU[r][m] v[r][m]
+                        bvals[e] = t8[e] * bf(sm + bV + (m >> 6) * 8192, tb + e, m & 63);
+                    // dv = beta TdU, and TdU into rows 64 + r of the stacked [dO ; TdU] tile, as bf16
+                    // pairs (m & ~1, m | 1): lanes m, m^1 swap one value per two tokens, the even
+                    // lane writes token tb + e, the odd one token tb + e + 1
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const float d0 = btv[e] * t8[e], d1 = btv[e + 1] * t8[e + 1];
+                        const float rd = __shfl_xor_sync(0xffffffffu, odd ? d0 : d1, 1);
+                        const float rt = __shfl_xor_sync(0xffffffffu, odd ? t8[e] : t8[e + 1], 1);
+                        const int r = tb + e + (odd ? 1 : 0);
+                        if (r < lc)
+                            *reinterpret_cast<uint32_t*>(dvp + (int64_t)r * Hv * dv) =
+                                odd ? pack_bf16(rd, d1) : pack_bf16(d0, rd);
+                        *reinterpret_cast<uint32_t*>(sm + bDO + (m >> 6) * 16384 + sw128_off(64 + r, (m & 63) >> 3) +
+                                                     (m & 6) * 2) = odd ? pack_bf16(rt, t8[e + 1]) : pack_bf16(t8[e], rt);
                     }
                     // sums over this warp's 32 m for each token: lane l ends with token tb + l / 4
                     warp_reduce_scatter<8>(bvals, lane);
@@ -863,8 +873,9 @@ __global__ void __launch_bounds__(kNT, 1)
                 const bool direct = p.group == 1 && !(kPrep && p.qk_norm);
                 float* dqp = args.dqw + (t0 * Hv + h) * dk + i;
                 float* dkp = args.dkw + (t0 * Hv + h) * dk + i;
-                __nv_bfloat16* dqb = (__nv_bfloat16*)b.dq + (t0 * Hv + h) * dk + i;
-                __nv_bfloat16* dkb = (__nv_bfloat16*)b.dk + (t0 * Hv + h) * dk + i;
+                __nv_bfloat16* dqb = (__nv_bfloat16*)b.dq + (t0 * Hv + h) * dk + (i & ~1);  // bf16 pairs
+                __nv_bfloat16* dkb = (__nv_bfloat16*)b.dk + (t0 * Hv + h) * dk + (i & ~1);
+                const bool odd = i & 1;
                 float* red2 = (float*)(sm + bBw);  // [8 warps][32]: the Gam-scaled Q is no longer read
 #pragma unroll 1
                 for (int g = 0; g < 4; ++g) {
@@ -885,7 +896,7 @@ __global__ void __launch_bounds__(kNT, 1)
                         dec8[4 * h4] = x2.x; dec8[4 * h4 + 1] = x2.y; dec8[4 * h4 + 2] = x2.z; dec8[4 * h4 + 3] = x2.w;
                         bg8[4 * h4] = x3.x; bg8[4 * h4 + 1] = x3.y; bg8[4 * h4 + 2] = x3.z; bg8[4 * h4 + 3] = x3.w;
                     }
-                    float gv[8], bv[8];
+                    float gv[8], bv[8], dq8[8], dk8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int r = tb + e;
@@ -893,19 +904,30 @@ __global__ void __launch_bounds__(kNT, 1)
                         const float dqv = qs + kpe[e];
                         const float kv = bf(qtile, 64 + r, i & 63);
                         const float dkv = dkm[e] + dec8[e] * dkd[e] + bg8[e] * tdw[e];
-                        if (r < lc) {
-                            if (direct) {
-                                dqb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(dqv);
-                                dkb[(int64_t)r * Hv * dk] = __float2bfloat16_rn(dkv);
-                            } else {
-                                dqp[(int64_t)r * Hv * dk] = dqv;
-                                dkp[(int64_t)r * Hv * dk] = dkv;
-                            }
+                        dq8[e] = dqv;
+                        dk8[e] = dkv;
+                        if (!direct && r < lc) {
+                            dqp[(int64_t)r * Hv * dk] = dqv;
+                            dkp[(int64_t)r * Hv * dk] = dkv;
                         }
                         const float kdterm = dec8[e] * kv * dkd[e];
                         gv[e] = bf(qtile, r, i & 63) * qs + bg8[e] * tdw[e] * kv - kdterm;
                         bv[e] = gam8[e] * tdw[e] * kv;
                         kdk += kdterm;
+                    }
+                    if (direct) {  // bf16 pairs (i & ~1, i | 1): lanes i, i^1 swap one value per two tokens
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            const float sq = __shfl_xor_sync(0xffffffffu, odd ? dq8[e] : dq8[e + 1], 1);
+                            const float sk = __shfl_xor_sync(0xffffffffu, odd ? dk8[e] : dk8[e + 1], 1);
+                            const int r = tb + e + (odd ? 1 : 0);
+                            if (r < lc) {
+                                *reinterpret_cast<uint32_t*>(dqb + (int64_t)r * Hv * dk) =
+                                    odd ? pack_bf16(sq, dq8[e + 1]) : pack_bf16(dq8[e], sq);
+                                *reinterpret_cast<uint32_t*>(dkb + (int64_t)r * Hv * dk) =
+                                    odd ? pack_bf16(sk, dk8[e + 1]) : pack_bf16(dk8[e], sk);
+                            }
+                        }
                     }
                     // sums over this warp's 32 i for each of the 8 tokens: lane l ends with token l / 4
                     warp_reduce_scatter<8>(gv, lane);
