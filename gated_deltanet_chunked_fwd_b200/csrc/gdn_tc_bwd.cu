@@ -829,16 +829,22 @@ __global__ void __launch_bounds__(kNT, 1)
                 }
             }
             __syncthreads();
-            if (tid < 128) {  // S = G + G^T, row s = tid % 64, columns [32 (tid / 64), + 32)
-                const int s = tid & 63, hs = tid >> 6;
+            {  // S = G + G^T, row s = tid % 64, columns [16 (tid / 64), + 16): G's rows as 16-byte
+               // groups (as_idx keeps four columns together), its columns element by element
+                const int s = tid & 63, qs = tid >> 6;
                 const float* G = (const float*)(sm + bV);
-                float v[32];
+                float v[16];
     #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = 32 * hs + jj;
-                    v[jj] = G[as_idx(s, j)] + G[as_idx(j, s)];
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    const int j0 = 16 * qs + 4 * j4;
+                    const float4 a = *reinterpret_cast<const float4*>(G + as_idx(s, j0));
+                    v[4 * j4] = a.x + G[as_idx(j0, s)];
+                    v[4 * j4 + 1] = a.y + G[as_idx(j0 + 1, s)];
+                    v[4 * j4 + 2] = a.z + G[as_idx(j0 + 2, s)];
+                    v[4 * j4 + 3] = a.w + G[as_idx(j0 + 3, s)];
                 }
-                store_row32(sm + bT, s, 4 * hs, v);
+                *reinterpret_cast<uint4*>(sm + bT + sw128_off(s, 2 * qs)) = pack8(v);
+                *reinterpret_cast<uint4*>(sm + bT + sw128_off(s, 2 * qs + 1)) = pack8(v + 8);
             }
             fence_proxy_async();
             tc_fence_before();
