@@ -309,6 +309,31 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, float* va, uint32_t tb,
         : "memory");
 }
 
+// One 16x256b.x4 load (16 TMEM lanes from the address x 32 columns); waits.  Per 8-column block b,
+// thread t gets (lane t/4, columns 8b + 2 (t%4) + {0, 1}) in registers 4b, 4b+1 and (lane t/4 + 8,
+// the same columns) in 4b+2, 4b+3: the fragment layout of 8 x 8 matrices (rows = lanes, columns =
+// TMEM columns) that stmatrix stores.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t ta, float* va) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(va);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(ta)
+        : "memory");
+}
+
+// stmatrix, four 8 x 8 b16 matrices, transposed: register j holds matrix j's fragment element pair
+// (row t/4, columns 2 (t%4), 2 (t%4) + 1); thread 8j + i gives the shared address of the stored row
+// i of matrix j, which is the matrix's column i (16 bytes).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t q0, uint32_t q1, uint32_t q2,
+                                                  uint32_t q3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(q0),
+                 "r"(q1), "r"(q2), "r"(q3)
+                 : "memory");
+}
+
 // 64 registers -> 64 consecutive TMEM columns of this warp's lanes; waits.
 __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* v) {
     const uint32_t* r = reinterpret_cast<const uint32_t*>(v);

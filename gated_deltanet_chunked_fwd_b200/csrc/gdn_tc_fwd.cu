@@ -491,34 +491,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nk > 1) load_gates(1);
         }
         // Outputs of chunk kk (once group S has finished it): o[t0+n][h][m] = O^T[m][n] from the
-        // O^T buffer of parity kk; this thread holds dv row m = `row`, tokens [32 hf, 32 hf + 32).
-        // A whole chunk goes through a shared-memory tile and one TMA store per 64-column half:
-        // lanes m, m^1 swap one value so that each thread writes bf16 pairs (columns m & ~1,
-        // m | 1) of one token.  A chunk cut short by its sequence's end is stored element by
-        // element, masked to its tokens.
+        // O^T buffer of parity kk; this warp covers dv rows 32 (warp & 3) .. + 31 and tokens
+        // [32 hf, 32 hf + 32).  A whole chunk goes through a shared-memory tile and one TMA store
+        // per 64-column half: the block is loaded in the 16x256b layout, whose registers form 8 x 8
+        // matrix fragments (dv rows x tokens), and stmatrix stores them transposed, one 16-byte row
+        // of 8 dv values per token.  A chunk cut short by its sequence's end is stored element by
+        // element (this thread: dv row `row`), masked to its tokens.
         auto emits = [&](int kk) { return final_walkn(kk) && chunk_ofn(kk) >= c0 && !args.himg; };
         auto epilogue = [&](int kk) {
             const int cc = chunk_ofn(kk);
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
-            const int m = row;
-            float ov[32];
+            const uint32_t colo = kColO + 64 * (kk & 1) + 32 * hf;
             tc_fence_after();
-            tmem_ld32(tl + kColO + 64 * (kk & 1) + 32 * hf, ov);
             if (lc == kChunk) {
-                if (t == 0) bulk_wait_read0();  // the previous chunk's store has read the tile
-                wg_sync(1, kThreadsP);
-                const bool odd = m & 1;
-                const int c = m & ~1, cin = c & 63;
-                uint8_t* tile = sm + kOst + (c >> 6) * 8192;
+                const int j = lane >> 3, i = lane & 7;  // this lane addresses stored row i of matrix j
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int nn = 32 * hf + e;
-                    const float x0 = ov[e], x1 = ov[e + 1];
-                    const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
-                    const uint32_t w = odd ? pack_bf16(recv, x1) : pack_bf16(x0, recv);
-                    const int orow = nn + (odd ? 1 : 0);
-                    *reinterpret_cast<uint32_t*>(tile + sw128_off(orow, cin >> 3) + (cin & 7) * 2) = w;
+                for (int lh = 0; lh < 2; ++lh) {  // lane halves 0-15 and 16-31 of this warp's quarter
+                    float f[16];
+                    tmem_ld16x256b_x4(tl + ((uint32_t)(16 * lh) << 16) + colo, f);
+                    if (lh == 0) {
+                        if (t == 0) bulk_wait_read0();  // the previous chunk's store has read the tile
+                        wg_sync(1, kThreadsP);
+                    }
+                    const int mrow = 32 * (warp & 3) + 16 * lh + 8 * (j & 1);  // first dv of its matrix
+                    uint8_t* tile = sm + kOst + (mrow >> 6) * 8192;
+#pragma unroll
+                    for (int bp = 0; bp < 2; ++bp) {  // 8-token blocks 2 bp (matrices 0, 1), 2 bp + 1 (2, 3)
+                        const float* r = f + 8 * bp;
+                        const int token = 32 * hf + 8 * (2 * bp + (j >> 1)) + i;
+                        stmatrix_x4_trans(smem_u32(tile + sw128_off(token, (mrow & 63) >> 3)),
+                                          pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]),
+                                          pack_bf16(r[6], r[7]));
+                    }
                 }
                 fence_proxy_async();  // the tile is read by the TMA store
                 wg_sync(1, kThreadsP);
@@ -528,7 +533,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_commit();
                 }
             } else {
-                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + m;
+                float ov[32];
+                tmem_ld32(tl + colo, ov);
+                __nv_bfloat16* op = (__nv_bfloat16*)p.o + (t0 * Hv + h) * dv + row;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int nn = 32 * hf + e;
