@@ -78,10 +78,10 @@ constexpr int kUIssuer = 96;  // group P's second MMA issuer (warp 3; thread 0 i
 constexpr int kTmemCols = 512;
 // TMEM column map (lane = row of the M = 128 MMA)
 constexpr uint32_t kColH = 0;     // H^T, fp32 state: lane dv, column dk     [0, 128)
-constexpr uint32_t kColR1 = 128;  // Q K^T (lanes 0-63), then W^T (group P)   [128, 192)
+constexpr uint32_t kColR1 = 128;  // Q K^T (lanes 0-63)                       [128, 192)
 constexpr uint32_t kColR2 = 192;  // 2 x (Ut^T -> U^T), by chunk parity      [192, 320)
-constexpr uint32_t kColO = 320;   // 2 x O^T = H^T (diag(Gam) Q)^T + U^T P^T,  [320, 448)
-                                  // by chunk parity
+constexpr uint32_t kColO = 320;   // O^T = H^T (diag(Gam) Q)^T + U^T P^T        [320, 384)
+constexpr uint32_t kColW = 384;   // W^T (group P)                              [384, 448)
 constexpr uint32_t kColHb = 448;  // bf16 H^T, A operand (K pairs per column) [448, 512)
 // U^T in bf16 (A operand of MMA_UP / MMA_H) overwrites the first 32 columns of its R2 buffer.
 
@@ -96,7 +96,7 @@ constexpr uint32_t kVec = 163840;      // 4 x 2 KB of per-token vectors, by chun
 constexpr uint32_t kVecStride = 512;   // floats per buffer
 constexpr uint32_t kOst = kVec + 4 * kVecStride * 4;  // 16 KB bf16 o tile [dv atom][64 tokens][128 B]
 constexpr uint32_t kRed = kOst + 16384;                // 16 floats
-constexpr uint32_t kBar = kRed + 64;   // 9 mbarriers + TMEM base
+constexpr uint32_t kBar = kRed + 64;   // 10 mbarriers + TMEM base
 constexpr uint32_t kSmemBytes = kBar + 128 + 1024;    // + alignment slack
 static_assert(kBwu + 4 * kTImgBytes <= kWt && kWt + 16384 <= kVec, "shared-memory regions overlap");
 
@@ -252,8 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bar_wt_full = bars + 4;  // W^T of chunk k in smem, Ut^T of chunk k in TMEM
     uint64_t* bar_wt_empty = bars + 5; // MMA_HW of chunk k has read W^T
     uint64_t* bar_s_done = bars + 6;   // [2] group S finished chunk k (parity buffers free)
-    uint64_t* bar_mma_u = bars + 8;    // MMA_U completions (group P's second issuer)
-    uint32_t* tmem_slot = (uint32_t*)(bars + 9);
+    uint64_t* bar_mma_u = bars + 8;    // MMA_U and MMA_W completions (group P's second issuer)
+    uint64_t* bar_o_free = bars + 9;   // group P has read chunk j's O^T out (arrival j)
+    uint32_t* tmem_slot = (uint32_t*)(bars + 10);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hv = p.Hv, dv = 128, dk = 128;
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- set-up: barriers, TMEM
     if (tid == 0) {
-        for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 10; ++i) mbar_init(&bars[i], 1);
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -502,7 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int cc = chunk_ofn(kk);
             const int64_t t0 = bos + (int64_t)cc * kChunk;
             const int lc = (int)min((int64_t)kChunk, len - (int64_t)cc * kChunk);
-            const uint32_t colo = kColO + 64 * (kk & 1) + 32 * hf;
+            // the last step's O^T goes to R1 (free by then), so that it need not wait for the read-out
+            // of the step before
+            const uint32_t colo = (kk == nk - 1 ? kColR1 : kColO) + 32 * hf;
             tc_fence_after();
             if (lc == kChunk) {
                 const int j = lane >> 3, i = lane & 7;  // this lane addresses stored row i of matrix j
@@ -526,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 fence_proxy_async();  // the tile is read by the TMA store
+                tc_fence_before();    // O^T has been read (group S may overwrite it once told)
                 wg_sync(1, kThreadsP);
                 if (t == 0) {
                     tma_store_3d(&tm_o, sm + kOst, 0, h, (int)t0);
@@ -541,6 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int nn = 32 * hf + e;
                     if (nn < lc) op[(int64_t)nn * Hv * dv] = __float2bfloat16_rn(ov[e]);
                 }
+                tc_fence_before();
+                wg_sync(1, kThreadsP);
             }
         };
 
@@ -564,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wg_and(1, kThreadsP, mbar_wait(&bar_s_done[stage], ((k - 2) >> 1) & 1));
                 if (!ok) break;
                 if (emits(k - 2)) epilogue(k - 2);
+                if (t == 0) mbar_arrive(bar_o_free);  // arrival k - 2: O^T of chunk k - 2 is out
             }
             ok = wg_and(1, kThreadsP, mbar_wait(&bar_tma[stage], (k >> 1) & 1));
             if (!ok) break;
@@ -583,13 +590,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(bar_mma_p);
             }
-            if (with_v && t == kUIssuer) {  // MMA_U: Ut^T = V^T Bu^T (R2[stage]) from a second issuer,
-                                            // on its own barrier, while MMA1 runs
+            if (t == kUIssuer) {  // MMA_U: Ut^T = V^T Bu^T (R2[stage]), unless the walk has v = 0, and
+                                  // MMA_W: W^T = K^T Bw^T (its own columns), from a second issuer on
+                                  // its own barrier while MMA1 runs
                 tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
-                                desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
+                for (int j = 0; j < 4; ++j) {
+                    if (with_v)
+                        mma_bf16_ss(tmem + kColR2 + 64 * stage, desc_sw128(sV + j * 2048, 8192, 1024),
+                                    desc_sw128(sBwu + kTImgBytes + j * 32, 16, 1024), id_mn_n64, j > 0);
+                    mma_bf16_ss(tmem + kColW, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
+                                desc_sw128(sBwu + j * 32, 16, 1024), id_mn_n64, j > 0);
+                }
                 mma_commit(bar_mma_u);
             }
             if (warp == 2 && k + 1 < nk) {  // the next chunk's gates, while MMA1 runs
@@ -661,27 +673,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             wg_sync(1, kThreadsP);
 
-            if (t == 0) {  // MMA_W: W^T = K^T Bw^T (R1, once P has read Q K^T from it)
-                tc_fence_after();
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_bf16_ss(tmem + kColR1, desc_sw128(sQK + 8192 + j * 2048, 16384, 1024),
-                                desc_sw128(sBwu + j * 32, 16, 1024), id_mn_n64, j > 0);
-                mma_commit(bar_mma_p);
-            }
             {  // W^T and Ut^T are in TMEM, and Wt is free once MMA_HW of chunk k-1 has read it
-                bool w = mbar_wait(bar_mma_p, ph);
-                if (with_v) w = w && mbar_wait(bar_mma_u, phu);
+                bool w = mbar_wait(bar_mma_u, phu);
                 if (k >= 1) w = w && mbar_wait(bar_wt_empty, (k - 1) & 1);
                 ok = wg_and(1, kThreadsP, w);
-                ph ^= 1;
-                if (with_v) phu ^= 1;
+                phu ^= 1;
                 if (!ok) break;
             }
             tc_fence_after();
             {  // W^T (lane = dk index) -> bf16 rows of the MN-major B operand of MMA_HW
                 float v[32];
-                tmem_ld32(tl + kColR1 + 32 * hf, v);
+                tmem_ld32(tl + kColW + 32 * hf, v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] = -v[e];  // MMA_HW accumulates -H^T W^T
                 store_row32(sm + kWt, row, 4 * hf, v);
@@ -738,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool emit = fin && c >= c0 && !args.himg;
             const uint32_t sQK = sbase + kStageQK + stage * 32768;
             const uint32_t colR2 = kColR2 + 64 * stage;
-            const uint32_t colO = kColO + 64 * stage;
+            const uint32_t colO = k == nk - 1 ? kColR1 : kColO;  // the last step's: R1 (group P is done with it)
 
             ok = wg_and(2, kThreadsS, mbar_wait(bar_wt_full, k & 1));
             if (!ok) break;
@@ -816,7 +818,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st32u(tl + colR2 + 32, w);
             }
             tc_fence_before();
-            wg_sync(2, kThreadsS);
+            // O^T of chunk k-1 has been read out by group P (its arrival k-1) before MMA_O rewrites
+            // the buffer; chunks without outputs write none, and the last step writes R1
+            ok = wg_and(2, kThreadsS, !(emit && k >= 1 && k < nk - 1) || mbar_wait(bar_o_free, (k - 1) & 1));
+            if (!ok) break;
             if (m == 0) {  // MMA_O: O^T = H^T (diag(Gam) Q)^T + U^T P^T;  MMA_H: H^T += (U^T diag(decay)) K
                 tc_fence_after();
                 if (emit) {
