@@ -592,7 +592,9 @@ __global__ void __launch_bounds__(kNT, 1)
             store_row32(sm + bWt, m, 4 * hh, v);
             {
                 // rows past the sequence end hold the next sequence's q and dO: zero them here
-                const int r = tid >> 2, a = (tid >> 1) & 1, part = tid & 1;
+                // thread: row tid % 64 of dk half (tid / 64) % 2, 16-byte chunks 4 part .. 4 part + 3;
+                // the eight lanes of a quarter warp take eight rows of one half (distinct banks)
+                const int r = tid & 63, a = (tid >> 6) & 1, part = tid >> 7;
                 const float gmul = r < lc ? vGam[r] : 0.f;
                 const uint4* src = reinterpret_cast<const uint4*>(sm + bQK + a * 16384 + r * 128);
                 uint4* dst = reinterpret_cast<uint4*>(sm + bBw + a * 8192 + r * 128);
