@@ -652,11 +652,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     store_row32(sm + kPt + stage * 8192, r, 4 * hf, v);
                 }
             } else if (emit) {
-                // thread li: q row li % 64 of dk half li / 64, so that the eight lanes of a quarter
-                // warp touch eight rows of one half, whose rotated 16-byte chunks fall on distinct banks
                 const int li = ((warp >> 2) << 6) | ((warp & 1) << 5) | lane;  // 0..127
-                const int srow = li & 63;
-                uint8_t* qrow = sm + kStageQK + stage * 32768 + (li >> 6) * 16384 + srow * 128;
+                const int srow = li >> 1;
+                uint8_t* qrow = sm + kStageQK + stage * 32768 + (li & 1) * 16384 + srow * 128;
                 const float gmul = vec[128 + srow];
 #pragma unroll
                 for (int i8 = 0; i8 < 8; ++i8) {
